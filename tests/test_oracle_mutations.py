@@ -1,0 +1,86 @@
+"""Plant plausible mistakes in copies of the oracle and check the pins catch them.
+
+Each mutant is a textual edit of ``oracle/oracle.c`` compiled into a
+temporary library; the pin tests are then run against it and at least one
+must fail.  The real oracle is untouched.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
+
+MUTANTS = {
+    "gqa_group_modulo": ("int g = h / r;", "int g = h % p->n_kv_head;"),
+    "scale_dropped": ("double s = p->scale * dot;", "double s = dot;"),
+    "causal_excludes_diagonal": ("int P = ctx + a;                                   /* absolute position */",
+                                 "int P = ctx + a - (a > 0);"),
+    "chunk_top_left_aligned": ("int P = ctx + a;", "int P = a;"),
+    "softmax_sign_flipped": ("w[j] = exp(w[j] - m);", "w[j] = exp(m - w[j]);"),
+    "k_and_v_swapped": ("const uint16_t *krow = kv_row(p, i, j, g, 0);",
+                        "const uint16_t *krow = kv_row(p, i, j, g, 1);"),
+    "wrong_kv_head_row": ("return base + (row * G + (size_t)g) * d;", "return base + (row * G) * d;"),
+    "prefix_boundary_off_by_one": ("if (j >= ctx) {", "if (j > ctx) {"),
+    "cache_slot_wrong": ("size_t slot = (size_t)(j % p->block_size);",
+                         "size_t slot = (size_t)((j + 1) % p->block_size);"),
+    "v_written_over_k": ("uint16_t *vd = kv_cache + (((size_t)page * 2 + 1)",
+                         "uint16_t *vd = kv_cache + (((size_t)page * 2 + 0)"),
+    "no_normalisation": ("for (int j = 0; j <= P; ++j) w[j] /= l;", "for (int j = 0; j <= P; ++j) w[j] /= 1.0;"),
+    "value_column_fixed": ("out[x] += w[j] * bf16_bits_to_double(vrow[x]);",
+                           "out[x] += w[j] * bf16_bits_to_double(vrow[0]);"),
+}
+
+# pins run against each mutant (the cheap ones; the byte-count pin is run separately)
+PIN_CALLS = [
+    lambda: pins.test_softmax_rows_sum_to_one([5, 70, 1], 6, 3, 32),
+    lambda: pins.test_softmax_weights_chunked_sum_to_one(),
+    lambda: pins.test_first_row_outputs_v0_exactly(),
+    lambda: pins.test_identical_keys_give_prefix_mean(),
+    lambda: pins.test_gqa_equals_mha_with_repeated_kv(8, 2),
+    lambda: pins.test_brute_force_tiny([3, 7, 1], 2, 1, 3),
+    lambda: pins.test_matches_torch_sdpa_fp64([300, 129, 2], 8, 2, 32),
+    lambda: pins.test_chunk_matches_torch_sdpa_with_explicit_mask(),
+    lambda: pins.test_chunked_equals_unchunked(100, 16),
+    lambda: pins.test_block_table_invariance_and_gather(),
+    lambda: pins.test_chunk_prefix_read_through_table(),
+]
+
+
+def _all_pins_pass() -> bool:
+    for call in PIN_CALLS:
+        try:
+            call()
+        except (AssertionError, RuntimeError):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    assert SRC.count(old) >= 1, f"mutation anchor for {name} not found"
+    src = tmp_path / "oracle_mutant.c"
+    src.write_text(SRC.replace(old, new, 1))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, str(src), "-o", str(lib), "-lm"])
+    handle = oracle._swap_library(str(lib))
+    try:
+        assert not _all_pins_pass(), f"mutant {name} passed every pin"
+    finally:
+        oracle._restore_library(handle)
+
+
+def test_unmutated_copy_passes(tmp_path):
+    src = tmp_path / "oracle_copy.c"
+    src.write_text(SRC)
+    lib = tmp_path / "liboracle_copy.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, str(src), "-o", str(lib), "-lm"])
+    handle = oracle._swap_library(str(lib))
+    try:
+        assert _all_pins_pass()
+    finally:
+        oracle._restore_library(handle)
