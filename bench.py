@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of libprefill's causal prefill attention on B200.
+
+One step = one prefill_attn call over the 8k-token GQA prompt (s=8192,
+n_head=32, n_kv_head=8, head_dim=128, paged cache block_size=16): scheduling,
+Q/K/V staging, S=QK^T, causal block rule, online softmax, P.V, output store
+and the fused paged KV write.  The chunked-prefill workload (16 chunks of 512
+tokens, prefix gathered from the cache) and the other shapes are measured too
+and reported under "workloads" (not the headline).
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_prefill_attention_b200 import _lib  # noqa: E402
+from causal_prefill_attention_b200 import workloads as W  # noqa: E402
+
+HEADLINE = "gqa_s8192_h32g8_d128"
+METRIC = "prefill attention TFLOP/s & % of B200 BF16 tensor peak; prompt tokens/s"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(bf16=d["bf16_tflops"], bf16_sustained=d.get("bf16_tflops_sustained"), hbm=d["hbm_gbs"],
+                    source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ device runners
+class PlainRunner:
+    """prefill_attn over one workload, inputs resident in HBM."""
+
+    def __init__(self, w: W.Workload, stream):
+        self.w = w
+        d = torch.device("cuda")
+        self.q, self.k, self.v = w.q.to(d), w.k.to(d), w.v.to(d)
+        self.cu, self.bt = w.cu_seqlens.to(d), w.block_table.to(d)
+        self.cache = w.empty_cache().to(d)
+        self.out = torch.empty_like(self.q)
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+        self.stream = stream
+        self.launches = 1
+        self.flops = w.causal_flops()
+        self.tokens = w.total_tokens
+
+    def step(self):
+        _lib.prefill_attn(self.q, self.k, self.v, self.cu, self.w.max_seqlen, self.w.scale, self.out, self.cache,
+                          self.bt, status=self.status, stream=self.stream)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
+
+
+class ChunkedRunner:
+    """The chunked workload: one call per 512-token chunk, in order."""
+
+    def __init__(self, w: W.Workload, chunk: int, stream):
+        self.w = w
+        d = torch.device("cuda")
+        self.parts = []
+        for q, k, v, cu, ctx, bt in W.chunk_views(w, chunk):
+            self.parts.append((q.to(d), k.to(d), v.to(d), cu.to(d), ctx.to(d), int(cu[-1]), int(ctx[0]),
+                               torch.empty(q.shape, dtype=torch.bfloat16, device=d)))
+        self.bt = w.block_table.to(d)
+        self.cache = w.empty_cache().to(d)
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+        self.stream = stream
+        self.launches = len(self.parts)
+        self.flops = w.causal_flops()   # same total as the unchunked prompt
+        self.tokens = w.total_tokens
+
+    def step(self):
+        for q, k, v, cu, ctx, L, c, out in self.parts:
+            _lib.prefill_attn_chunked(q, k, v, cu, ctx, L, c, self.w.scale, out, self.cache, self.bt,
+                                      status=self.status, stream=self.stream)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
+
+
+def time_steps(runner, steps, warmup, stream, flush):
+    for _ in range(warmup):
+        runner.step()
+    torch.cuda.synchronize()
+    runner.check_status()
+    durs = []
+    for _ in range(steps):
+        flush.add_(1)  # write > L2 so every step starts cold
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        runner.step()
+        b.record(stream)
+        durs.append((a, b))
+    torch.cuda.synchronize()
+    runner.check_status()
+    return [a.elapsed_time(b) for a, b in durs]
+
+
+def e2e_plain(w: W.Workload, steps, warmup, stream):
+    """Same metric through the C ABI with pinned host buffers: H2D of the step's
+    inputs and D2H of its output inside the timed region."""
+    d = torch.device("cuda")
+    host = {n: t.pin_memory() for n, t in
+            dict(q=w.q, k=w.k, v=w.v, cu=w.cu_seqlens, bt=w.block_table).items()}
+    dev = {n: torch.empty_like(t, device=d) for n, t in host.items()}
+    cache = w.empty_cache().to(d)
+    out = torch.empty_like(dev["q"])
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out.numel() * out.element_size()
+
+    def one():
+        with torch.cuda.stream(stream):
+            for n in host:
+                dev[n].copy_(host[n], non_blocking=True)
+            _lib.prefill_attn(dev["q"], dev["k"], dev["v"], dev["cu"], w.max_seqlen, w.scale, out, cache, dev["bt"],
+                              status=status, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
+    """Time the oracle on random (row, head) pairs of the workload until about
+    budget_s seconds of CPU work; return (TFLOP/s, cores, description)."""
+    import oracle  # test infrastructure: only the CPU-baseline / reference legs use it
+    rng = np.random.default_rng(seed)
+    done_flops, elapsed, nrows = 0.0, 0.0, 0
+    batch = 64
+    while elapsed < budget_s:
+        rows = rng.integers(0, w.total_tokens, batch)
+        heads = rng.integers(0, w.n_head, batch)
+        starts = w.cu_seqlens.numpy()
+        pos = rows - starts[np.searchsorted(starts, rows, side="right") - 1]
+        t0 = time.perf_counter()
+        oracle.attention_rows(w.q, w.k, w.v, w.cu_seqlens, w.n_head, w.n_kv_head, w.head_dim, w.scale,
+                              rows.tolist(), heads.tolist())
+        elapsed += time.perf_counter() - t0
+        done_flops += float(np.sum(4.0 * w.head_dim * (pos + 1)))
+        nrows += batch
+    desc = (f"{nrows} random (row, head) output rows of {w.name} through the fp64 oracle "
+            f"({elapsed:.1f} s); FLOPs counted as 4*head_dim*(keys) per row, the causal count")
+    return done_flops / elapsed / 1e12, oracle.num_threads(), desc, elapsed
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return reference_arm(args)
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    _lib.load()
+    stream = torch.cuda.current_stream()
+    w = W.named_workload(HEADLINE)
+    runner = PlainRunner(w, stream)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    pk = peaks()
+
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        durs = time_steps(runner, args.steps, args.warmup, stream, flush)
+    torch.cuda.synchronize()
+    total_ms = sum(durs)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms = total_ms / args.steps
+    tflops = runner.flops / (ms * 1e-3) / 1e12
+    value = tflops * world  # replicas: every rank runs the same work
+    tokens_s = runner.tokens / (ms * 1e-3) * world
+
+    e2e_ms, h2d, d2h = e2e_plain(w, max(3, args.steps // 2), 3, stream)
+    e2e_tflops = runner.flops / (e2e_ms * 1e-3) / 1e12 * world
+
+    extra = {}
+    if not args.no_extra and rank == 0:
+        for name in W.NAMED:
+            if name == HEADLINE:
+                continue
+            wx = W.named_workload(name)
+            rx = ChunkedRunner(wx, wx.chunk, stream) if wx.chunk else PlainRunner(wx, stream)
+            dx = time_steps(rx, max(5, args.steps // 2), 3, stream, flush)
+            mx = statistics.median(dx)
+            extra[name] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
+                           "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches}
+            del rx, wx
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1:
+        v, cores, desc, el = oracle_sample(w, args.cpu_budget)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC,
+            "value": round(value, 3),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic: seeded randn bf16 Q/K/V, sentinel-filled paged cache, shuffled block table",
+            "config": {"workload": HEADLINE, "s": 8192, "n_head": 32, "n_kv_head": 8, "head_dim": 128,
+                       "block_size": 16, "num_seqs": 1, "causal": True,
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "pct_of_peak": round(100.0 * tflops / pk["bf16"], 2),
+            "prompt_tokens_per_s": round(tokens_s, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": pk["bf16"], "unit": "TFLOP/s",
+                         "frac": round(tflops / pk["bf16"], 4), "traffic": None,
+                         "peak_source": f"{pk['source']} bf16 burst (kernel timed alone)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_tflops, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": runner.launches * args.steps,
+            "clocks": clocks,
+            "workloads": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def reference_arm(args):
+    """The fp64 CPU oracle on the headline workload, each step a bounded sample."""
+    w = W.named_workload(HEADLINE)
+    per_step = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
+    vals = []
+    for s in range(args.warmup + args.steps):
+        v, cores, desc, el = oracle_sample(w, per_step, seed=s)
+        if s >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    # ms for one whole step of the workload at the sampled rate
+    ms = w.causal_flops() / (value * 1e12) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": HEADLINE, "s": 8192, "n_head": 32, "n_kv_head": 8, "head_dim": 128,
+                   "block_size": 16, "num_seqs": 1, "causal": True},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,133 @@
+"""ctypes binding of libprefill's C ABI (include/prefill.h).
+
+Argument marshalling only: tensors are turned into device pointers and sizes,
+and every step of the computation runs in the CUDA kernels behind the ABI.
+There is no fallback: if the shared library is missing, loading fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libprefill.so")
+
+STATUS_NAMES = {
+    0: "PREFILL_OK", 1: "PREFILL_ERR_NULL", 2: "PREFILL_ERR_SHAPE", 3: "PREFILL_ERR_UNSUPPORTED",
+    4: "PREFILL_ERR_BLOCK_TABLE", 5: "PREFILL_ERR_CUDA", 6: "PREFILL_ERR_TIMEOUT", 7: "PREFILL_ERR_ALIGNMENT",
+}
+EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
+            "prefill_num_kv_blocks", "prefill_kv_block_rule")
+
+_lib = None
+
+
+class PrefillError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libprefill.so from the package directory (raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libprefill.so not built at {LIB_PATH}; run causal_prefill_attention_b200.build")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.prefill_attn.argtypes = [P, P, P, I, P, I, I, I, I, I, F, P, P, I, P, I, I, P, P]
+        lib.prefill_attn.restype = I
+        lib.prefill_attn_chunked.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, I, P, I, I, P, P]
+        lib.prefill_attn_chunked.restype = I
+        lib.prefill_status_string.argtypes = [I]
+        lib.prefill_status_string.restype = ctypes.c_char_p
+        lib.prefill_num_kv_blocks.argtypes = [I, I, I, I, I]
+        lib.prefill_num_kv_blocks.restype = I
+        lib.prefill_kv_block_rule.argtypes = [I, I, I, I, I, I, P, P]
+        lib.prefill_kv_block_rule.restype = I
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().prefill_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check_bf16(name, t, ndim):
+    if t.dtype != torch.bfloat16 or t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous {ndim}-d bfloat16 tensor")
+
+
+def _check_i32(name, t):
+    if t.dtype != torch.int32 or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous int32 tensor")
+
+
+def prefill_attn(q, k, v, cu_seqlens, max_seqlen: int, scale: float, out, kv_cache, block_table,
+                 status: Optional[torch.Tensor] = None, stream=None, raise_on_error: bool = True) -> int:
+    """Causal prefill attention + paged KV write (C ABI ``prefill_attn``).
+
+    q/out [T, n_head, head_dim], k/v [T, n_kv_head, head_dim], kv_cache
+    [num_blocks, 2, block_size, n_kv_head, head_dim] (bf16, CUDA);
+    cu_seqlens int32 [B+1], block_table int32 [B, max_blocks_per_seq].
+    """
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3)
+    _check_bf16("out", out, 3), _check_bf16("kv_cache", kv_cache, 5)
+    _check_i32("cu_seqlens", cu_seqlens), _check_i32("block_table", block_table)
+    T, H, D = q.shape
+    G = k.shape[1]
+    rc = load().prefill_attn(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1, int(max_seqlen),
+        H, G, D, float(scale), _ptr(out), _ptr(kv_cache), kv_cache.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "prefill_attn")
+    return rc
+
+
+def prefill_attn_chunked(q, k, v, cu_seqlens_q, context_lens, max_q_len: int, max_context_len: int,
+                         scale: float, out, kv_cache, block_table, status: Optional[torch.Tensor] = None,
+                         stream=None, raise_on_error: bool = True) -> int:
+    """Chunked prefill (C ABI ``prefill_attn_chunked``): each chunk attends to
+    ``context_lens[i]`` cached tokens plus itself, then appends its K/V."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3)
+    _check_bf16("out", out, 3), _check_bf16("kv_cache", kv_cache, 5)
+    _check_i32("cu_seqlens_q", cu_seqlens_q), _check_i32("context_lens", context_lens)
+    _check_i32("block_table", block_table)
+    T, H, D = q.shape
+    G = k.shape[1]
+    rc = load().prefill_attn_chunked(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(cu_seqlens_q), _ptr(context_lens), cu_seqlens_q.numel() - 1,
+        int(max_q_len), int(max_context_len), H, G, D, float(scale), _ptr(out), _ptr(kv_cache),
+        kv_cache.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "prefill_attn_chunked")
+    return rc
+
+
+def num_kv_blocks(qb: int, ctx: int, n: int, bm: int = 128, bn: int = 128) -> int:
+    return load().prefill_num_kv_blocks(qb, ctx, n, bm, bn)
+
+
+def kv_block_rule(qb: int, j: int, ctx: int, n: int, bm: int = 128, bn: int = 128):
+    """(kind, col_limit[bm], key_begin): kind 0 = unmasked, 1 = masked, -1 = out of range."""
+    lim = (ctypes.c_int32 * bm)()
+    kb = ctypes.c_int32(0)
+    kind = load().prefill_kv_block_rule(qb, j, ctx, n, bm, bn, lim, ctypes.byref(kb))
+    return kind, list(lim), kb.value

@@ -1,0 +1,163 @@
+// api.cu -- the C ABI of libprefill (include/prefill.h): host-side argument
+// checks, TMA tensor-map encoding, kernel launch.  Allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/prefill.h"
+#include "block_rule.h"
+#include "params.h"
+
+namespace {
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims innermost first, strides in bytes
+// for dims 1..rank-1.  Out-of-range boxes are filled with zeros.
+bool encode(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+            const cuuint32_t *box) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total, const int32_t *cu,
+        const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
+        int n_kv_head, int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *cache, int num_blocks,
+        const int32_t *bt, int mbps, int bs, int32_t *status, prefill_stream_t stream) {
+    if (!q || !k || !v || !cu || !out || !cache || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
+    if (total < 0 || num_seqs < 0 || max_q < 0 || max_ctx < 0) return PREFILL_ERR_SHAPE;
+    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (bs != 16 && bs != 32 && bs != 64 && bs != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (!(std::isfinite(scale) && scale > 0.f)) return PREFILL_ERR_UNSUPPORTED;
+    if (num_blocks < 1 || mbps < 1) return PREFILL_ERR_BLOCK_TABLE;
+    // each bound must fit the table; the exact per-sequence check (context +
+    // chunk length) runs on the device, where the lengths are
+    if (max_ctx > (long long)mbps * bs || max_q > (long long)mbps * bs) return PREFILL_ERR_BLOCK_TABLE;
+    if (num_seqs > 65535 || n_head > 65535) return PREFILL_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * 2 * bs * n_kv_head * head_dim > (1ll << 40)) return PREFILL_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cache))
+        return PREFILL_ERR_ALIGNMENT;
+    if (total == 0 || num_seqs == 0 || max_q == 0) return PREFILL_OK;
+
+    pf::TensorMaps maps;
+    const cuuint64_t D = head_dim, H = n_head, G = n_kv_head, T = total;
+    {
+        const cuuint64_t dims[3] = {D, H, T}, strides[2] = {D * 2, H * D * 2};
+        const cuuint32_t box[3] = {64, 1, 128};
+        if (!encode(&maps.q, q, 3, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[3] = {D, G, T}, strides[2] = {D * 2, G * D * 2};
+        const cuuint32_t box[3] = {64, 1, 128};
+        if (!encode(&maps.k, k, 3, dims, strides, box)) return PREFILL_ERR_CUDA;
+        if (!encode(&maps.v, v, 3, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[4] = {D, G, (cuuint64_t)bs, (cuuint64_t)num_blocks * 2};
+        const cuuint64_t strides[3] = {D * 2, G * D * 2, (cuuint64_t)bs * G * D * 2};
+        const cuuint32_t box[4] = {64, 1, (cuuint32_t)bs, 1};
+        if (!encode(&maps.cache, cache, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+
+    pf::FwdParams p;
+    p.k = k;
+    p.v = v;
+    p.out = out;
+    p.cache = cache;
+    p.cu_seqlens = cu;
+    p.context_lens = chunked ? ctx_lens : nullptr;
+    p.block_table = bt;
+    p.status = status;
+    p.num_seqs = num_seqs;
+    p.n_head = n_head;
+    p.n_kv_head = n_kv_head;
+    p.group = n_head / n_kv_head;
+    p.total = total;
+    p.num_blocks = num_blocks;
+    p.mbps = mbps;
+    p.block_size = bs;
+    p.max_q = max_q;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    int e = pf::launch_fwd_v0(maps, p, head_dim, stream);
+    return e == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int prefill_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_tokens,
+                 const int32_t *cu_seqlens, int num_seqs, int max_seqlen, int n_head, int n_kv_head, int head_dim,
+                 float scale, prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks,
+                 const int32_t *block_table, int max_blocks_per_seq, int block_size, int32_t *status_dev,
+                 prefill_stream_t stream) {
+    return run(q, k, v, total_tokens, cu_seqlens, nullptr, false, num_seqs, max_seqlen, 0, n_head, n_kv_head,
+               head_dim, scale, out, kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
+               status_dev, stream);
+}
+
+int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,
+                         const int32_t *cu_seqlens_q, const int32_t *context_lens, int num_seqs, int max_q_len,
+                         int max_context_len, int n_head, int n_kv_head, int head_dim, float scale,
+                         prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks, const int32_t *block_table,
+                         int max_blocks_per_seq, int block_size, int32_t *status_dev, prefill_stream_t stream) {
+    return run(q, k, v, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len, n_head,
+               n_kv_head, head_dim, scale, out, kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
+               status_dev, stream);
+}
+
+const char *prefill_status_string(int s) {
+    switch (s) {
+        case PREFILL_OK: return "ok";
+        case PREFILL_ERR_NULL: return "a required pointer is NULL";
+        case PREFILL_ERR_SHAPE: return "inconsistent sizes";
+        case PREFILL_ERR_UNSUPPORTED: return "unsupported head_dim, block_size or scale";
+        case PREFILL_ERR_BLOCK_TABLE: return "block table entry out of range or table too short";
+        case PREFILL_ERR_CUDA: return "CUDA launch or driver failure";
+        case PREFILL_ERR_TIMEOUT: return "device pipeline wait exceeded its limit";
+        case PREFILL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int prefill_num_kv_blocks(int qb, int ctx, int n, int bm, int bn) {
+    if (bm < 1 || bn < 1 || ctx < 0 || n < 0) return 0;
+    return pf::num_kv_blocks(qb, ctx, n, bm, bn);
+}
+
+int prefill_kv_block_rule(int qb, int j, int ctx, int n, int bm, int bn, int32_t *col_limit, int32_t *key_begin) {
+    if (bm < 1 || bn < 1 || ctx < 0 || n < 0 || j < 0 || j >= prefill_num_kv_blocks(qb, ctx, n, bm, bn)) return -1;
+    const pf::KvBlock b = pf::kv_block(qb, j, ctx, n, bm, bn);
+    if (key_begin) *key_begin = b.key_begin;
+    if (col_limit)
+        for (int r = 0; r < bm; ++r) col_limit[r] = b.full ? bn : pf::col_limit(b, r, bn);
+    return b.full ? 0 : 1;
+}
+
+}  // extern "C"

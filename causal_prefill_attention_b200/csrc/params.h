@@ -1,0 +1,39 @@
+// params.h -- launch parameters shared by the host API and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+namespace pf {
+
+struct FwdParams {
+    const uint16_t *k;            // [T][G][D] this call's keys (for the cache write)
+    const uint16_t *v;            // [T][G][D]
+    uint16_t *out;                // [T][H][D]
+    uint16_t *cache;              // [NB][2][bs][G][D]
+    const int32_t *cu_seqlens;    // [B+1]
+    const int32_t *context_lens;  // [B] or nullptr (plain prefill)
+    const int32_t *block_table;   // [B][mbps]
+    int32_t *status;              // nullable
+    int num_seqs;
+    int n_head;
+    int n_kv_head;
+    int group;                    // n_head / n_kv_head
+    int total;                    // rows of q/k/v/out
+    int num_blocks;
+    int mbps;                     // max_blocks_per_seq
+    int block_size;
+    int max_q;                    // bound on every sequence (chunk) length
+    float scale_log2;             // scale * log2(e)
+};
+
+struct TensorMaps {
+    CUtensorMap q;      // {D, H, T}, box {64, 1, 128}
+    CUtensorMap k;      // {D, G, T}, box {64, 1, 128}
+    CUtensorMap v;      // {D, G, T}, box {64, 1, 128}
+    CUtensorMap cache;  // {D, G, bs, 2*NB}, box {64, 1, bs, 1}
+};
+
+// Launchers (defined per kernel file); return a cudaError_t value.
+int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
+
+}  // namespace pf

@@ -1,0 +1,168 @@
+/*
+ * prefill.h -- C ABI of libprefill: causal prefill attention (MHA / GQA) for
+ * NVIDIA B200 (sm_100a), fused with the paged KV-cache write.
+ *
+ * What a call computes, for every sequence i of a packed batch, every query
+ * row a of that sequence and every query head h:
+ *
+ *   P    = ctx_i + a                  absolute position (ctx_i = 0 for prefill_attn)
+ *   g    = h / (n_head / n_kv_head)   kv head shared by a contiguous group of query heads
+ *   s_j  = scale * <q[a][h], k_j[g]>  for keys j = 0 .. P   (causal: later keys are skipped)
+ *   out[a][h] = sum_j softmax(s)_j * v_j[g]
+ *
+ * and it writes every token's K and V rows into its page of the KV cache.
+ *
+ * Sources (page address and section):
+ *   hncyxsy.com/news/270449 §2.2  head split: (s, h) viewed as (s, n_head, head_dim), head_dim last
+ *   hncyxsy.com/news/270449 §2.3  per-head scores, causal upper-triangle mask, softmax, times V
+ *   hncyxsy.com/news/270449 §3.1  scores divided by sqrt(head_dim); mask by block-index control flow
+ *   hncyxsy.com/news/270449 §3.2  online softmax: per-block max and exp-sum, old results rescaled
+ *   hncyxsy.com/news/270449 §3.3  heads merged back to (s, h) by flattening (s, n_head, head_dim)
+ *   hncyxsy.com/news/270449 §3.4  GQA: several query heads share one K/V head
+ *   hncyxsy.com/news/270449 §4.2  KV cache in fixed-size blocks; the write is fused, not a copy kernel
+ *   hncyxsy.com/news/270449 §4.3  query blocks x kv blocks; skip / unmasked / column-masked blocks
+ *   hncyxsy.com/news/227904 §2.1  chunked prefill: a chunk attends to all earlier K/V
+ *   hncyxsy.com/news/227904 §3.4  page table maps a sequence's logical pages to physical blocks
+ *   lnwmold.com/news/496245 §3.3  block size 16, prefill chunk 512 (workload shapes)
+ *
+ * Layouts (all row-major, contiguous, little-endian bf16 = IEEE bfloat16 bits):
+ *   q, out    [total_tokens][n_head][head_dim]
+ *   k, v      [total_tokens][n_kv_head][head_dim]
+ *   kv_cache  [num_blocks][2][block_size][n_kv_head][head_dim]   ([.][0] = K page, [.][1] = V page)
+ *   block_table  int32 [num_seqs][max_blocks_per_seq]; logical page p of sequence i
+ *                (positions p*block_size .. p*block_size+block_size-1) lives in
+ *                physical block block_table[i][p].  Entries past a sequence's last
+ *                page are never read.
+ *   cu_seqlens   int32 [num_seqs + 1]; sequence i owns packed rows
+ *                cu_seqlens[i] .. cu_seqlens[i+1]-1 (non-decreasing, cu_seqlens[0] = 0).
+ *
+ * Ownership: every pointer argument is caller-owned DEVICE memory, except where
+ * stated.  The library allocates no device memory per call, keeps nothing after
+ * return, and enqueues its work asynchronously on `stream` (the legacy default
+ * stream if NULL).  It writes `out`, the cache slots of the tokens it processes,
+ * and `*status_dev`; nothing else.  Inputs must stay valid until the work on
+ * `stream` completes.
+ *
+ * Errors: argument problems that the host can see are returned synchronously
+ * and nothing is launched.  Problems only the device can see (a block-table
+ * entry outside [0, num_blocks), a sequence longer than the bound given, a
+ * decreasing cu_seqlens, a pipeline wait that ran past its limit) make the
+ * affected work skip its memory accesses and set `*status_dev` to the first
+ * such code (atomic compare-and-swap from PREFILL_OK); the caller zeroes it
+ * before the call and reads it after synchronising.  With status_dev == NULL
+ * such problems are still skipped but not reported.
+ *
+ * Preconditions (stated, not checked): no physical block appears twice in the
+ * block table (within or across sequences); input values are finite.
+ */
+#ifndef LIBPREFILL_PREFILL_H
+#define LIBPREFILL_PREFILL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Raw bfloat16 storage (the 16 high bits of an IEEE binary32). */
+typedef uint16_t prefill_bf16;
+/* Same object as a CUDA runtime cudaStream_t / driver CUstream. */
+typedef struct CUstream_st *prefill_stream_t;
+
+typedef enum {
+    PREFILL_OK = 0,
+    PREFILL_ERR_NULL = 1,         /* a required pointer is NULL */
+    PREFILL_ERR_SHAPE = 2,        /* inconsistent sizes or a sequence longer than the bound given */
+    PREFILL_ERR_UNSUPPORTED = 3,  /* head_dim, block_size or scale outside the supported set */
+    PREFILL_ERR_BLOCK_TABLE = 4,  /* block-table entry outside [0, num_blocks) or table too short */
+    PREFILL_ERR_CUDA = 5,         /* launch or driver failure */
+    PREFILL_ERR_TIMEOUT = 6,      /* a device-side pipeline wait exceeded its iteration limit */
+    PREFILL_ERR_ALIGNMENT = 7     /* a pointer is not 16-byte aligned */
+} prefill_status;
+
+/*
+ * prefill_attn -- causal prefill attention over whole prompts, fused with the
+ * paged KV write (hncyxsy.com/news/270449 §3.1-§4.3; hncyxsy.com/news/227904 §3.4).
+ *
+ *   q, k, v        device, layouts above, total_tokens rows each
+ *   total_tokens   rows in q/k/v/out (= cu_seqlens[num_seqs]); 0 is a no-op
+ *   cu_seqlens     device int32 [num_seqs + 1]
+ *   num_seqs       >= 1 (0 is a no-op)
+ *   max_seqlen     upper bound on every sequence length (host value; sizes the grid)
+ *   n_head, n_kv_head   n_head % n_kv_head == 0
+ *   head_dim       64 or 128
+ *   scale          finite, > 0 (normally 1/sqrt(head_dim))
+ *   out            device, written: [total_tokens][n_head][head_dim] bf16
+ *   kv_cache       device, written at the slots of this call's tokens only
+ *   num_blocks     physical blocks in kv_cache (>= 1)
+ *   block_table    device int32 [num_seqs][max_blocks_per_seq]
+ *   block_size     16, 32, 64 or 128 tokens per block
+ *   status_dev     device int32 (nullable), see Errors above
+ *   stream         CUDA stream to enqueue on
+ * Requires max_seqlen <= max_blocks_per_seq * block_size.
+ * Returns a prefill_status.
+ */
+int prefill_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                 int total_tokens, const int32_t *cu_seqlens, int num_seqs, int max_seqlen,
+                 int n_head, int n_kv_head, int head_dim, float scale,
+                 prefill_bf16 *out,
+                 prefill_bf16 *kv_cache, int num_blocks,
+                 const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                 int32_t *status_dev, prefill_stream_t stream);
+
+/*
+ * prefill_attn_chunked -- chunked prefill (hncyxsy.com/news/227904 §2.1): each
+ * sequence's query chunk attends to the context_lens[i] tokens already in the
+ * cache (gathered through block_table) plus itself, causally, with the chunk
+ * aligned at the end: chunk row a sits at absolute position context_lens[i] + a.
+ * The chunk's own K/V are then appended to the cache at those positions.
+ *
+ *   q, k, v        device, the chunk's rows only: total_q rows
+ *   cu_seqlens_q   device int32 [num_seqs + 1] over the chunk rows
+ *   context_lens   device int32 [num_seqs]: cached tokens before each chunk
+ *   max_q_len      upper bound on every chunk length (host)
+ *   max_context_len  upper bound on every context length (host)
+ *   the rest as for prefill_attn.
+ * The cached prefix is read as it stands before the call (the slots this call
+ * writes are all at positions >= context_lens[i]).
+ * Requires max_q_len <= max_blocks_per_seq * block_size and max_context_len <=
+ * max_blocks_per_seq * block_size; a sequence whose context_lens[i] + chunk
+ * length exceeds the table is skipped on the device and reported as
+ * PREFILL_ERR_BLOCK_TABLE.
+ */
+int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                         int total_q, const int32_t *cu_seqlens_q, const int32_t *context_lens,
+                         int num_seqs, int max_q_len, int max_context_len,
+                         int n_head, int n_kv_head, int head_dim, float scale,
+                         prefill_bf16 *out,
+                         prefill_bf16 *kv_cache, int num_blocks,
+                         const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                         int32_t *status_dev, prefill_stream_t stream);
+
+/* Human-readable name of a prefill_status value (static storage). */
+const char *prefill_status_string(int status);
+
+/*
+ * Causal block rule (hncyxsy.com/news/270449 §4.3), exported so that host code
+ * and tests can check the exact rule the kernels use.  Host-only, no GPU needed.
+ *
+ * A query block covers chunk rows [qb*bm, qb*bm + bm).  Its kv blocks are
+ * numbered j = 0 .. prefill_num_kv_blocks()-1: first the cached prefix
+ * (positions [j*bn, j*bn + bn) intersected with [0, ctx)), then the chunk's own
+ * keys in blocks of bn aligned to the chunk start, up to the diagonal block.
+ * Blocks above the diagonal are not numbered (never issued).
+ *
+ * prefill_kv_block_rule returns 0 if every (row < n, key) pair of block j is
+ * visible (no mask), 1 if it is partly masked, -1 if j is out of range; for a
+ * masked block it writes, for each row r of the query block, the number of
+ * leading visible key columns to col_limit[r] (bm entries; may be NULL).
+ * Its key range starts at absolute position *key_begin (may be NULL).
+ */
+int prefill_num_kv_blocks(int qb, int ctx, int n, int bm, int bn);
+int prefill_kv_block_rule(int qb, int j, int ctx, int n, int bm, int bn,
+                          int32_t *col_limit, int32_t *key_begin);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIBPREFILL_PREFILL_H */

@@ -1,0 +1,125 @@
+"""CPU tests of the C ABI: the library loads, exports what the header declares,
+rejects bad arguments before any launch, and its causal block rule matches the
+brute-force mask.  No compute call is made (there may be no GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from causal_prefill_attention_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "prefill.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(prefill_[a-z_0-9]+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert "prefill_attn" in names and "prefill_attn_chunked" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(_lib.EXPORTED) <= set(names)
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert _lib.status_string(s)
+    assert _lib.status_string(99) == "unknown status"
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _call(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, total=128, cu=FAKE, num_seqs=1, max_seqlen=128, H=4, G=4, D=128,
+             scale=0.088, out=FAKE, cache=FAKE, nb=8, bt=FAKE, mbps=8, bs=16, status=None, stream=None)
+    a.update(over)
+    return lib.prefill_attn(a["q"], a["k"], a["v"], a["total"], a["cu"], a["num_seqs"], a["max_seqlen"], a["H"],
+                            a["G"], a["D"], a["scale"], a["out"], a["cache"], a["nb"], a["bt"], a["mbps"], a["bs"],
+                            a["status"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(cu=None), 1), (dict(bt=None), 1), (dict(cache=None), 1),
+    (dict(H=6, G=4), 2), (dict(G=0), 2), (dict(total=-1), 2),
+    (dict(D=96), 3), (dict(D=256), 3), (dict(bs=8), 3), (dict(bs=24), 3),
+    (dict(scale=0.0), 3), (dict(scale=float("nan")), 3), (dict(scale=float("inf")), 3), (dict(scale=-1.0), 3),
+    (dict(max_seqlen=129), 4), (dict(nb=0), 4), (dict(mbps=0), 4),
+    (dict(q=FAKE + 8), 7), (dict(out=FAKE + 2), 7),
+])
+def test_host_validation_rejects_before_launch(lib, over, code):
+    assert _call(lib, **over) == code
+
+
+def test_empty_call_is_a_noop(lib):
+    assert _call(lib, total=0) == 0
+    assert _call(lib, num_seqs=0) == 0
+
+
+def test_chunked_validation(lib):
+    P = FAKE
+    args = [P, P, P, 512, P, P, 1, 512, 7680, 32, 8, 128, 0.088, P, P, 512, P, 512, 16, None, None]
+    a = list(args)
+    a[5] = None  # context_lens
+    assert lib.prefill_attn_chunked(*a) == 1
+    a = list(args)
+    a[8] = 8193  # the context bound alone exceeds the table
+    assert lib.prefill_attn_chunked(*a) == 4
+    a = list(args)
+    a[7] = 8193  # the chunk bound alone exceeds the table
+    assert lib.prefill_attn_chunked(*a) == 4
+
+
+# ---------------------------------------------------------------- P11: block rule vs brute force
+def _brute_visible(ctx, n):
+    """visible[a, p] for chunk rows a < n and absolute key positions p < ctx + n."""
+    a = np.arange(n)[:, None]
+    p = np.arange(ctx + n)[None, :]
+    return p <= ctx + a
+
+
+@pytest.mark.parametrize("bm,bn", [(128, 128), (64, 64), (128, 64), (64, 128)])
+def test_block_rule_matches_brute_force_mask(lib, bm, bn):
+    rng = np.random.default_rng(5)
+    cases = [(0, n) for n in (1, 2, 3, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 256, 300)]
+    cases += [(int(c), int(n)) for c, n in zip(rng.integers(0, 400, 40), rng.integers(1, 300, 40))]
+    cases += [(128, 128), (512, 512), (130, 5), (1, 1)]
+    for ctx, n in cases:
+        vis = _brute_visible(ctx, n)
+        covered = np.zeros_like(vis, dtype=np.int32)
+        for qb in range(-(-n // bm)):
+            rows = np.arange(qb * bm, min(qb * bm + bm, n))
+            nkv = _lib.num_kv_blocks(qb, ctx, n, bm, bn)
+            for j in range(nkv):
+                kind, lim, kb = _lib.kv_block_rule(qb, j, ctx, n, bm, bn)
+                assert kind in (0, 1)
+                for r_i, a in enumerate(rows):
+                    r = a - qb * bm
+                    cols = kb + np.arange(bn)
+                    in_range = cols < ctx + n
+                    want = np.zeros(bn, dtype=bool)
+                    want[in_range] = vis[a, cols[in_range]]
+                    # prefix blocks stop at ctx; chunk blocks never include prefix columns
+                    if j < -(-ctx // bn):
+                        want &= cols < ctx
+                    got = np.arange(bn) < lim[r]
+                    assert np.array_equal(got, want), (ctx, n, qb, j, a)
+                    if kind == 0:
+                        assert want.all()
+                    covered[a, cols[got]] += 1
+            assert _lib.kv_block_rule(qb, nkv, ctx, n, bm, bn)[0] == -1
+        # every visible pair is covered by exactly one issued block; no invisible pair is
+        assert np.array_equal(covered, vis.astype(np.int32)), (ctx, n)
