@@ -5,6 +5,8 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <cstdint>
 #include <mutex>
 
@@ -40,6 +42,17 @@ bool encode(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims, c
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// The pipelined kernel runs unless LIBPREFILL_KERNEL=simple selects the
+// one-CTA-per-block kernel (used to compare the two on the same inputs).
+bool use_pipelined() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("LIBPREFILL_KERNEL");
+        v = (e && std::strcmp(e, "simple") == 0) ? 0 : 1;
+    }
+    return v == 1;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -104,7 +117,9 @@ int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int
     p.max_q = max_q;
     p.scale_log2 = scale * 1.4426950408889634f;
 
-    int e = pf::launch_fwd_v0(maps, p, head_dim, stream);
+    int e = (use_pipelined() && pf::fwd_pipelined_supported(p, head_dim))
+                ? pf::launch_fwd(maps, p, head_dim, stream)
+                : pf::launch_fwd_v0(maps, p, head_dim, stream);
     return e == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 

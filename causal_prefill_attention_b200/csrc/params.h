@@ -34,6 +34,10 @@ struct TensorMaps {
 };
 
 // Launchers (defined per kernel file); return a cudaError_t value.
+// Pipelined warp-specialised kernel (prefill_fwd.cu) and the sizes it takes.
+int launch_fwd(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
+bool fwd_pipelined_supported(const FwdParams &p, int head_dim);
+// One-CTA-per-query-block kernel (prefill_fwd_v0.cu): no size limits.
 int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
 
 }  // namespace pf

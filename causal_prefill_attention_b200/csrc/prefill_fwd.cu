@@ -1,0 +1,618 @@
+// prefill_fwd.cu -- pipelined, warp-specialised causal prefill attention for
+// sm_100a, fused with the paged KV-cache write.
+//
+// The method is the tiled attention of hncyxsy.com/news/270449 §3.2 and §4.3:
+// Q split into query blocks, K/V into kv blocks, a running row max and exp-sum
+// per query row, old partial results rescaled when the max grows, P.V
+// accumulated, and blocks above the causal diagonal never issued.  Only the
+// final output and the KV cache reach HBM.
+//
+// B200 mapping (the pages target A100; this is a redesign, not their kernel):
+//   * persistent grid, one CTA per SM; a work item is a pair of consecutive
+//     128-row query blocks of one (sequence, head); items are ordered longest
+//     first on the device from cu_seqlens and dealt to CTAs in zigzag order.
+//   * warps 0-3 / 4-7: softmax for query block 0 / 1 (one TMEM lane = one
+//     row per thread); they also apply the (lazy) rescale of O and store the
+//     final O / l.  Warp 8: TMA producer (Q blocks, K/V ring of NST stages,
+//     paged prefix gather).  Warp 9: tcgen05 MMA issuer.  Warp 10: paged KV
+//     writer.  Warp 11: idle.
+//   * TMEM (512 columns): S0 | S1 | O0 | O1, 128 columns each; P (bf16) is
+//     written over the first 64 columns of its S and read by the P.V MMA
+//     directly from TMEM.
+//   * MMA order per kv block j: PV0(j), S0(j+1), PV1(j), S1(j+1), so the
+//     softmax of one query block overlaps the tensor-core work of the other.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <math_constants.h>
+
+#include "block_rule.h"
+#include "params.h"
+#include "sm100.cuh"
+#include "../../include/prefill.h"
+
+namespace pf {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NST = 4;  // K/V ring stages (each one K or one V tile)
+constexpr int NTHREADS = 384;
+constexpr int WARP_PRODUCER = 8, WARP_MMA = 9, WARP_WRITER = 10;
+constexpr uint32_t CHUNK = 128 * 128;  // 128 rows x 64 bf16, 128B-swizzled
+// Threshold (log2 units) before the running max is moved and O rescaled;
+// between moves P can reach 2^8, well inside fp32 / bf16 range.
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct Lay {
+    static constexpr int NCH = D / 64;
+    static constexpr uint32_t TILE = NCH * CHUNK;
+    static constexpr uint32_t Q0 = 0, Q1 = TILE, KV = 2 * TILE;
+    static constexpr uint32_t BAR = KV + NST * TILE;
+    // barrier slots
+    static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NST, B_SFULL = 4 + 2 * NST,
+                         B_PFULL = 6 + 2 * NST, B_OFULL = 8 + 2 * NST, B_OEMPTY = 10 + 2 * NST,
+                         NBAR = 12 + 2 * NST;
+    static constexpr uint32_t TMEM_SLOT = BAR + NBAR * 8, ABORT = TMEM_SLOT + 4;
+    static constexpr uint32_t SCHED = BAR + 256;
+};
+
+// ------------------------------------------------------------------ schedule
+struct Item {
+    int i, h, g, qb0, c0, n, ctx;
+    int nk0, nk1;  // kv blocks visited by query block 0 / 1
+    int two;       // second query block present
+    __device__ __forceinline__ int nk(int s) const { return s ? nk1 : nk0; }
+    __device__ __forceinline__ int nmax() const { return nk0 > nk1 ? nk0 : nk1; }
+};
+
+__device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
+    const int c0 = p.cu_seqlens[i], c1 = p.cu_seqlens[i + 1];
+    const int n = c1 - c0;
+    const int ctx = p.context_lens ? p.context_lens[i] : 0;
+    const bool bl = n < 0 || n > p.max_q || c0 < 0 || c1 > p.total;
+    const bool bc = ctx < 0 || (long long)ctx + n > (long long)p.mbps * p.block_size;
+    if (bl || bc) {
+        *bad = true;
+        return 0;
+    }
+    return cdiv(n, 2 * BM);
+}
+
+// Work items are ordered by pair index p descending (the longest causal rows
+// first), then by sequence (longest first), then head.  T[p] counts the items
+// with pair index >= p (T[P] = 0), so pair index p owns items [T[p+1], T[p]);
+// perm lists sequences by pair count, descending, ties by index, so the first
+// A(p) entries are exactly the sequences that own pair index p.
+__device__ __forceinline__ Item decode_item(const FwdParams &p, const int *T, const uint16_t *perm, int P, int u) {
+    int lo = 0, hi = P - 1;  // largest pi with T[pi] > u
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (T[mid] > u) lo = mid; else hi = mid - 1;
+    }
+    const int pi = lo;
+    const int v = u - T[pi + 1];
+    const int k = v / p.n_head;
+    Item it;
+    it.h = v - k * p.n_head;
+    it.i = perm[k];
+    it.g = it.h / p.group;
+    it.qb0 = 2 * pi;
+    it.c0 = p.cu_seqlens[it.i];
+    it.n = p.cu_seqlens[it.i + 1] - it.c0;
+    it.ctx = p.context_lens ? p.context_lens[it.i] : 0;
+    it.two = (it.qb0 + 1) * BM < it.n;
+    it.nk0 = num_kv_blocks(it.qb0, it.ctx, it.n, BM, BN);
+    it.nk1 = it.two ? num_kv_blocks(it.qb0 + 1, it.ctx, it.n, BM, BN) : 0;
+    return it;
+}
+
+__device__ __forceinline__ int zigzag(int k, int c, int G) { return k * G + ((k & 1) ? (G - 1 - c) : c); }
+
+// ------------------------------------------------------------------ waits
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort) {
+#pragma unroll 1
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
+__device__ __forceinline__ void setmaxnreg_dec88() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_cache,
+                   const FwdParams p, const int P) {
+    using L = Lay<D>;
+    constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+    constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    volatile int *abort = reinterpret_cast<volatile int *>(gbase + L::ABORT);
+    int *T = reinterpret_cast<int *>(gbase + L::SCHED);
+    int *cur = T + (P + 1);
+    uint16_t *perm = reinterpret_cast<uint16_t *>(cur + (P + 1));
+    auto bar = [&](int idx) -> uint32_t { return base + L::BAR + 8u * idx; };
+
+    // ---------------- set-up: barriers, TMEM, schedule
+    if (tid == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_cache);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(L::B_QFULL + s), 1);
+            mbar_init(bar(L::B_QEMPTY + s), 1);
+            mbar_init(bar(L::B_SFULL + s), 1);
+            mbar_init(bar(L::B_PFULL + s), 4);
+            mbar_init(bar(L::B_OFULL + s), 1);
+            mbar_init(bar(L::B_OEMPTY + s), 4);
+        }
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar(L::B_KVFULL + s), 1);
+            mbar_init(bar(L::B_KVEMPTY + s), 1);
+        }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(base + L::TMEM_SLOT, 512);
+        tmem_relinquish();
+    }
+    for (int x = tid; x <= P; x += NTHREADS) cur[x] = 0;
+    __syncthreads();
+    {
+        bool bad = false;
+        for (int i = tid; i < p.num_seqs; i += NTHREADS) {
+            const int c = seq_pairs(p, i, &bad);
+            if (c > 0) atomicAdd(&cur[c], 1);
+        }
+        if (bad && blockIdx.x == 0) report(p.status, PREFILL_ERR_SHAPE);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // Two suffix scans over c = P .. 0 in one pass:
+        //   A(c) = sequences with more than c pairs (= those owning pair index c)
+        //        = bucket start of pair count c in the sorted order;
+        //   T[c] = items with pair index >= c = n_head * sum_{c' >= c} A(c').
+        int carry_a = 0, carry_t = 0;
+        for (int top = P; top >= 0; top -= 32) {
+            const int c = top - lane;
+            const int hc = c >= 0 ? cur[c] : 0;
+            int incl = hc;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += t;
+            }
+            const int a = c >= 0 ? carry_a + incl - hc : 0;
+            int incl_a = a;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl_a, off);
+                if (lane >= off) incl_a += t;
+            }
+            __syncwarp();
+            if (c >= 0) {
+                T[c] = (carry_t + incl_a) * p.n_head;
+                cur[c] = a;
+            }
+            carry_a += __shfl_sync(0xffffffffu, incl, 31);
+            carry_t += __shfl_sync(0xffffffffu, incl_a, 31);
+        }
+        __syncwarp();
+        // stable counting sort of sequences by pair count, descending
+        for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
+            const int i = b0 + lane;
+            bool bad = false;
+            const int c = i < p.num_seqs ? seq_pairs(p, i, &bad) : 0;
+            const unsigned act = __ballot_sync(0xffffffffu, c > 0);
+            if (c > 0) {
+                const unsigned grp = __match_any_sync(act, c);
+                const int rank = __popc(grp & ((1u << lane) - 1u));
+                perm[cur[c] + rank] = (uint16_t)i;
+                __syncwarp(grp);
+                if (rank == 0) cur[c] += __popc(grp);
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int total = T[0];
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gbase + L::TMEM_SLOT);
+    const int G = gridDim.x, cta = blockIdx.x;
+
+    if (warp < 8) {
+        // ================= softmax / rescale / epilogue for query block s
+        setmaxnreg_inc208();
+        const int s = warp >> 2;
+        const int row = tid & 127;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + 128u * s + lane_off;
+        const uint32_t tO = tmem + 256u + 128u * s + lane_off;
+        const uint32_t b_sfull = bar(L::B_SFULL + s), b_pfull = bar(L::B_PFULL + s);
+        const uint32_t b_ofull = bar(L::B_OFULL + s), b_oempty = bar(L::B_OEMPTY + s);
+        const float sl2 = p.scale_log2;
+        const float thr = kRescaleLog2 / sl2;  // the threshold in raw score units
+        uint32_t ph_s = 0, ph_o = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int u = zigzag(k, cta, G);
+            if (u >= total) break;
+            const Item it = decode_item(p, T, perm, P, u);
+            if (s == 1 && !it.two) continue;
+            const int qb = it.qb0 + s;
+            const int nk = it.nk(s);
+            float m_run = -CUDART_INF_F, l_run = 0.f;
+            for (int j = 0; j < nk; ++j) {
+                if (!wait_bar(b_sfull, ph_s, abort)) { ok = false; break; }
+                ph_s ^= 1;
+                tc_fence_after();
+                float x[BN];
+                {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int c4 = 0; c4 < BN / 32; ++c4) {
+                        tmem_ld32(tS + c4 * 32, r);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(r[c]);
+                    }
+                }
+                const KvBlock kb = kv_block(qb, j, it.ctx, it.n, BM, BN);
+                if (!kb.full) {
+                    const int lim = col_limit(kb, row, BN);
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        if (c >= lim) x[c] = -CUDART_INF_F;
+                }
+                float mt = x[0];
+#pragma unroll
+                for (int c = 1; c < BN; ++c) mt = fmaxf(mt, x[c]);
+                const bool need = mt > m_run + thr;
+                float m_new = need ? fmaxf(m_run, mt) : m_run;
+                if (m_new == -CUDART_INF_F) m_new = 0.f;
+                const float alpha = need ? ex2((m_run - m_new) * sl2) : 1.f;
+                const float nms = -m_new * sl2;
+                float sum = 0.f;
+                {
+                    uint32_t pw[32];
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const float p0 = ex2(fmaf(x[half * 64 + 2 * c], sl2, nms));
+                            const float p1 = ex2(fmaf(x[half * 64 + 2 * c + 1], sl2, nms));
+                            sum += p0 + p1;
+                            pw[c] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st32(tS + half * 32, pw);
+                    }
+                }
+                l_run = l_run * alpha + sum;
+                m_run = m_new;
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        tmem_ld32(tO + cc * 32, r);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+                        tmem_st32(tO + cc * 32, r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_pfull);
+            }
+            if (!ok) break;
+            // final O / l -> bf16 rows of out
+            if (!wait_bar(b_ofull, ph_o, abort)) { ok = false; break; }
+            ph_o ^= 1;
+            tc_fence_after();
+            const int a = qb * BM + row;
+            const float inv_l = 1.f / l_run;
+            uint16_t *dst = p.out + ((size_t)(it.c0 + a) * p.n_head + it.h) * D;
+            {
+                uint32_t r[32];
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    tmem_ld32(tO + cc * 32, r);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
+                    if (a < it.n) {
+                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_oempty);
+        }
+        if (!ok && (tid & 127) == 0) report(p.status, PREFILL_ERR_TIMEOUT);
+    } else {
+        setmaxnreg_dec88();
+        if (warp == WARP_PRODUCER) {
+            // ================= TMA producer (all lanes loop; lane 0 issues)
+            const int bs = p.block_size;
+            int stage = 0;
+            uint32_t phase = 0, ph_qe = 0;  // bit s: phase of Q block s
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int u = zigzag(k, cta, G);
+                if (u >= total) break;
+                const Item it = decode_item(p, T, perm, P, u);
+                const int ns = it.two ? 2 : 1;
+                for (int s = 0; s < ns; ++s) {
+                    if (!wait_bar(bar(L::B_QEMPTY + s), ((ph_qe >> s) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    ph_qe ^= 1u << s;
+                    if (lane == 0) {
+                        const uint32_t b = bar(L::B_QFULL + s);
+                        mbar_expect_tx(b, L::TILE);
+#pragma unroll
+                        for (int ch = 0; ch < L::NCH; ++ch)
+                            tma_load_3d(base + (s ? L::Q1 : L::Q0) + ch * CHUNK, &tm_q, b, ch * 64, it.h,
+                                        it.c0 + (it.qb0 + s) * BM);
+                    }
+                }
+                const int nmax = it.nmax();
+                for (int j = 0; j < nmax && ok; ++j) {
+                    const KvBlock kb = kv_block(it.qb0, j, it.ctx, it.n, BM, BN);
+                    for (int t = 0; t < 2; ++t) {  // t = 0: K, t = 1: V
+                        if (!wait_bar(bar(L::B_KVEMPTY + stage), phase ^ 1, abort)) { ok = false; break; }
+                        const uint32_t dst = base + L::KV + stage * L::TILE;
+                        const uint32_t b = bar(L::B_KVFULL + stage);
+                        if (!kb.prefix) {
+                            if (lane == 0) {
+                                mbar_expect_tx(b, L::TILE);
+#pragma unroll
+                                for (int ch = 0; ch < L::NCH; ++ch)
+                                    tma_load_3d(dst + ch * CHUNK, t ? &tm_v : &tm_k, b, ch * 64, it.g,
+                                                it.c0 + kb.src_row);
+                            }
+                        } else {
+                            // prefix: whole pages by TMA; the rest of the block (a partly
+                            // valid page, rows past the prefix) by plain loads and zeros
+                            const int npos = kb.lim_const;
+                            const int full_pages = npos / bs;
+                            const int r0 = full_pages * bs;
+                            if (r0 < BN) {
+                                const int units = (BN - r0) * 8 * L::NCH;
+                                for (int x = lane; x < units; x += 32) {
+                                    const int rr = r0 + x / (8 * L::NCH);
+                                    const int ch = (x / 8) % L::NCH;
+                                    const int un = x % 8;
+                                    uint4 val = make_uint4(0, 0, 0, 0);
+                                    if (rr < npos) {
+                                        const int P_ = kb.key_begin + rr;
+                                        const int page = p.block_table[(size_t)it.i * p.mbps + P_ / bs];
+                                        if (page >= 0 && page < p.num_blocks) {
+                                            const size_t off =
+                                                ((((size_t)page * 2 + t) * bs + P_ % bs) * p.n_kv_head + it.g) * D +
+                                                ch * 64 + un * 8;
+                                            val = *reinterpret_cast<const uint4 *>(p.cache + off);
+                                        } else {
+                                            report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                                        }
+                                    }
+                                    uint8_t *d = gbase + (dst - base) + ch * CHUNK + rr * 128 + ((un ^ (rr & 7)) << 4);
+                                    *reinterpret_cast<uint4 *>(d) = val;
+                                }
+                                fence_proxy_async_smem();
+                                __syncwarp();
+                            }
+                            if (lane == 0) {
+                                mbar_expect_tx(b, (uint32_t)(full_pages * bs * 128 * L::NCH));
+                                for (int pg = 0; pg < full_pages; ++pg) {
+                                    int page = p.block_table[(size_t)it.i * p.mbps + kb.key_begin / bs + pg];
+                                    if (page < 0 || page >= p.num_blocks) {
+                                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                                        page = p.num_blocks;  // outside the map: zero fill
+                                    }
+#pragma unroll
+                                    for (int ch = 0; ch < L::NCH; ++ch)
+                                        tma_load_4d(dst + ch * CHUNK + pg * bs * 128, &tm_cache, b, ch * 64, it.g, 0,
+                                                    page * 2 + t);
+                                }
+                            }
+                        }
+                        if (++stage == NST) { stage = 0; phase ^= 1; }
+                    }
+                }
+            }
+            if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
+        } else if (warp == WARP_MMA) {
+            // ================= tcgen05 MMA issuer (lane 0)
+            if (lane == 0) {
+                int stage = 0;
+                // per-query-block phase bits (bit s) and "O already used" bits
+                uint32_t phase = 0, ph_qf = 0, ph_pf = 0, ph_oe = 0, used = 0;
+                bool ok = true;
+                auto kv_wait = [&](int st, uint32_t ph) { return wait_bar(bar(L::B_KVFULL + st), ph, abort); };
+                auto issue_s = [&](int s, int kst) {
+                    const uint32_t q = base + (s ? L::Q1 : L::Q0), kk_ = base + L::KV + kst * L::TILE;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+                        mma_ss(tmem + 128u * s, smem_desc_sw128(q + off, 16, 1024),
+                               smem_desc_sw128(kk_ + off, 16, 1024), IDESC_QK, kk > 0);
+                    }
+                };
+                auto issue_pv = [&](int s, int vst, bool acc) {
+                    const uint32_t vv = base + L::KV + vst * L::TILE;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_ts(tmem + 256u + 128u * s, tmem + 128u * s + kk * 8,
+                               smem_desc_sw128(vv + kk * 2048, CHUNK, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                };
+                for (int k = 0; ok; ++k) {
+                    const int u = zigzag(k, cta, G);
+                    if (u >= total) break;
+                    const Item it = decode_item(p, T, perm, P, u);
+                    const int ns = it.two ? 2 : 1;
+                    const int nmax = it.nmax();
+                    for (int s = 0; s < ns && ok; ++s) {
+                        ok = wait_bar(bar(L::B_QFULL + s), (ph_qf >> s) & 1u, abort);
+                        ph_qf ^= 1u << s;
+                    }
+                    if (!ok) break;
+                    // K_0
+                    int kst = stage;
+                    uint32_t kph = phase;
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
+                    if (!kv_wait(kst, kph)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int s = 0; s < ns; ++s) {
+                        issue_s(s, kst);
+                        tc_commit(bar(L::B_SFULL + s));
+                    }
+                    tc_commit(bar(L::B_KVEMPTY + kst));
+                    for (int j = 0; j < nmax && ok; ++j) {
+                        const int vst = stage;
+                        const uint32_t vph = phase;
+                        if (++stage == NST) { stage = 0; phase ^= 1; }
+                        int nst = -1;
+                        uint32_t nph = 0;
+                        if (j + 1 < nmax) {
+                            nst = stage;
+                            nph = phase;
+                            if (++stage == NST) { stage = 0; phase ^= 1; }
+                        }
+                        if (!kv_wait(vst, vph)) { ok = false; break; }
+                        bool next_ready = false;
+                        for (int s = 0; s < ns; ++s) {
+                            if (j >= it.nk(s)) continue;
+                            if (!wait_bar(bar(L::B_PFULL + s), (ph_pf >> s) & 1u, abort)) { ok = false; break; }
+                            ph_pf ^= 1u << s;
+                            if (j == 0 && ((used >> s) & 1u)) {
+                                if (!wait_bar(bar(L::B_OEMPTY + s), (ph_oe >> s) & 1u, abort)) { ok = false; break; }
+                                ph_oe ^= 1u << s;
+                            }
+                            tc_fence_after();
+                            issue_pv(s, vst, j > 0);
+                            if (j + 1 < it.nk(s)) {
+                                if (!next_ready) {
+                                    if (!kv_wait(nst, nph)) { ok = false; break; }
+                                    tc_fence_after();
+                                    next_ready = true;
+                                }
+                                issue_s(s, nst);
+                                tc_commit(bar(L::B_SFULL + s));
+                            } else {
+                                tc_commit(bar(L::B_OFULL + s));
+                                tc_commit(bar(L::B_QEMPTY + s));
+                            }
+                        }
+                        if (!ok) break;
+                        tc_commit(bar(L::B_KVEMPTY + vst));
+                        if (nst >= 0) {
+                            if (!next_ready) {  // no slot needed K_{j+1}: still wait so the stage is consumed in order
+                                if (!kv_wait(nst, nph)) { ok = false; break; }
+                            }
+                            tc_commit(bar(L::B_KVEMPTY + nst));
+                        }
+                    }
+                    used |= it.two ? 3u : 1u;
+                }
+                if (!ok) report(p.status, PREFILL_ERR_TIMEOUT);
+            }
+            __syncwarp();
+        } else if (warp == WARP_WRITER) {
+            // ================= paged KV write of each item's tokens (one query head per group)
+            constexpr int U = D * 2 / 16;  // 16-byte units per row
+            const int bs = p.block_size;
+            for (int k = 0;; ++k) {
+                const int u = zigzag(k, cta, G);
+                if (u >= total) break;
+                const Item it = decode_item(p, T, perm, P, u);
+                if (it.h % p.group) continue;
+                const int a0 = it.qb0 * BM;
+                const int a1 = min(a0 + 2 * BM, it.n);
+                const size_t G_ = p.n_kv_head;
+                for (int x = lane; x < (a1 - a0) * U; x += 32) {
+                    const int a = a0 + x / U, un = x % U;
+                    const int P_ = it.ctx + a;
+                    const int page = p.block_table[(size_t)it.i * p.mbps + P_ / bs];
+                    if (page < 0 || page >= p.num_blocks) {
+                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                        continue;
+                    }
+                    const size_t src = ((size_t)(it.c0 + a) * G_ + it.g) * D;
+                    const size_t dk = ((((size_t)page * 2 + 0) * bs + P_ % bs) * G_ + it.g) * D;
+                    const size_t dv = ((((size_t)page * 2 + 1) * bs + P_ % bs) * G_ + it.g) * D;
+                    const uint4 kval = reinterpret_cast<const uint4 *>(p.k + src)[un];
+                    const uint4 vval = reinterpret_cast<const uint4 *>(p.v + src)[un];
+                    reinterpret_cast<uint4 *>(p.cache + dk)[un] = kval;
+                    reinterpret_cast<uint4 *>(p.cache + dv)[un] = vval;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+size_t smem_bytes(int P, int num_seqs) {
+    return Lay<D>::SCHED + (size_t)(P + 1) * 8 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int D>
+int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
+    const int P = cdiv(p.max_q, 2 * BM);
+    const size_t smem = smem_bytes<D>(P, p.num_seqs);
+    cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return (int)e;
+    const long long items_bound = (long long)p.num_seqs * p.n_head * P;
+    const int grid = (int)(items_bound < sm_count() ? items_bound : sm_count());
+    prefill_fwd_kernel<D><<<grid, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache, p, P);
+    return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+// Sizes the pipelined kernel handles (its schedule lives in shared memory).
+bool fwd_pipelined_supported(const FwdParams &p, int head_dim) {
+    const int P = cdiv(p.max_q, 2 * BM);
+    if (P > 2048 || p.num_seqs > 4096) return false;
+    const size_t smem = head_dim == 64 ? smem_bytes<64>(P, p.num_seqs) : smem_bytes<128>(P, p.num_seqs);
+    return smem <= 227 * 1024;
+}
+
+int launch_fwd(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream) {
+    if (head_dim == 64) return launch<64>(maps, p, stream);
+    return launch<128>(maps, p, stream);
+}
+
+}  // namespace pf
