@@ -173,7 +173,7 @@ def time_steps(runner, steps, warmup, stream, flush):
     return [a.elapsed_time(b) for a, b in durs]
 
 
-def e2e_plain(w: W.Workload, steps, warmup, stream):
+def e2e_run(w: W.Workload, steps, warmup, stream):
     """Same metric through the C ABI with pinned host buffers: H2D of the step's
     inputs and D2H of its output inside the timed region."""
     d = torch.device("cuda")
@@ -186,13 +186,25 @@ def e2e_plain(w: W.Workload, steps, warmup, stream):
     status = torch.zeros(1, dtype=torch.int32, device=d)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out.numel() * out.element_size()
+    chunks = []
+    if w.chunk:
+        for c0 in range(0, w.total_tokens, w.chunk):
+            L = min(w.chunk, w.total_tokens - c0)
+            chunks.append((c0, L, torch.tensor([0, L], dtype=torch.int32, device=d),
+                           torch.tensor([c0], dtype=torch.int32, device=d)))
 
     def one():
         with torch.cuda.stream(stream):
             for n in host:
                 dev[n].copy_(host[n], non_blocking=True)
-            _lib.prefill_attn(dev["q"], dev["k"], dev["v"], dev["cu"], w.max_seqlen, w.scale, out, cache, dev["bt"],
-                              status=status, stream=stream)
+            if not w.chunk:
+                _lib.prefill_attn(dev["q"], dev["k"], dev["v"], dev["cu"], w.max_seqlen, w.scale, out, cache,
+                                  dev["bt"], status=status, stream=stream)
+            else:
+                for c0, L, cu, ctx in chunks:
+                    sl = slice(c0, c0 + L)
+                    _lib.prefill_attn_chunked(dev["q"][sl], dev["k"][sl], dev["v"][sl], cu, ctx, L, c0, w.scale,
+                                              out[sl], cache, dev["bt"], status=status, stream=stream)
             out_h.copy_(out, non_blocking=True)
 
     for _ in range(warmup):
@@ -242,6 +254,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--workload", default=HEADLINE, choices=list(W.NAMED),
+                    help="workload timed as the step (default: the 8k GQA prompt)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -264,8 +278,8 @@ def main():
 
     _lib.load()
     stream = torch.cuda.current_stream()
-    w = W.named_workload(HEADLINE)
-    runner = PlainRunner(w, stream)
+    w = W.named_workload(args.workload)
+    runner = ChunkedRunner(w, w.chunk, stream) if w.chunk else PlainRunner(w, stream)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     pk = peaks()
 
@@ -286,13 +300,13 @@ def main():
     value = tflops * world  # replicas: every rank runs the same work
     tokens_s = runner.tokens / (ms * 1e-3) * world
 
-    e2e_ms, h2d, d2h = e2e_plain(w, max(3, args.steps // 2), 3, stream)
+    e2e_ms, h2d, d2h = e2e_run(w, max(3, args.steps // 2), 3, stream)
     e2e_tflops = runner.flops / (e2e_ms * 1e-3) / 1e12 * world
 
     extra = {}
     if not args.no_extra and rank == 0:
         for name in W.NAMED:
-            if name == HEADLINE:
+            if name == args.workload:
                 continue
             wx = W.named_workload(name)
             rx = ChunkedRunner(wx, wx.chunk, stream) if wx.chunk else PlainRunner(wx, stream)
@@ -323,10 +337,7 @@ def main():
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic: seeded randn bf16 Q/K/V, sentinel-filled paged cache, shuffled block table",
-            "config": {"workload": HEADLINE, "s": 8192, "n_head": 32, "n_kv_head": 8, "head_dim": 128,
-                       "block_size": 16, "num_seqs": 1, "causal": True,
-                       "l2": "flushed before every timed step (256 MiB write)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "config": config_of(w, world),
             "pct_of_peak": round(100.0 * tflops / pk["bf16"], 2),
             "prompt_tokens_per_s": round(tokens_s, 1),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": pk["bf16"], "unit": "TFLOP/s",
@@ -346,9 +357,16 @@ def main():
     return 0
 
 
+def config_of(w: W.Workload, world: int) -> dict:
+    return {"workload": w.name, "tokens": w.total_tokens, "num_seqs": w.num_seqs, "max_seqlen": w.max_seqlen,
+            "n_head": w.n_head, "n_kv_head": w.n_kv_head, "head_dim": w.head_dim, "block_size": w.block_size,
+            "chunk": w.chunk, "causal": True, "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 def reference_arm(args):
-    """The fp64 CPU oracle on the headline workload, each step a bounded sample."""
-    w = W.named_workload(HEADLINE)
+    """The fp64 CPU oracle on the same workload, each step a bounded sample."""
+    w = W.named_workload(args.workload)
     per_step = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
     vals = []
     for s in range(args.warmup + args.steps):
@@ -362,8 +380,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": HEADLINE, "s": 8192, "n_head": 32, "n_kv_head": 8, "head_dim": 128,
-                   "block_size": 16, "num_seqs": 1, "causal": True},
+        "config": config_of(w, 1),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: {desc}"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

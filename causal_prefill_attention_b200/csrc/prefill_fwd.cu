@@ -15,7 +15,9 @@
 //     row per thread); they also apply the (lazy) rescale of O and store the
 //     final O / l.  Warp 8: TMA producer (Q blocks, K/V ring of NST stages,
 //     paged prefix gather).  Warp 9: tcgen05 MMA issuer.  Warp 10: paged KV
-//     writer.  Warp 11: idle.
+//     writer, a second consumer of the K/V ring that stores each item's own
+//     K/V tiles from shared memory into their cache pages (TMA stores).
+//     Warp 11: idle.
 //   * TMEM (512 columns): S0 | S1 | O0 | O1, 128 columns each; P (bf16) is
 //     written over the first 64 columns of its S and read by the P.V MMA
 //     directly from TMEM.
@@ -79,25 +81,33 @@ __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
     return cdiv(n, 2 * BM);
 }
 
-// Work items are ordered by pair index p descending (the longest causal rows
-// first), then by sequence (longest first), then head.  T[p] counts the items
-// with pair index >= p (T[P] = 0), so pair index p owns items [T[p+1], T[p]);
-// perm lists sequences by pair count, descending, ties by index, so the first
-// A(p) entries are exactly the sequences that own pair index p.
-__device__ __forceinline__ Item decode_item(const FwdParams &p, const int *T, const uint16_t *perm, int P, int u) {
-    int lo = 0, hi = P - 1;  // largest pi with T[pi] > u
+// Work items are ordered sequence-major: sequences by pair count, descending
+// (ties by index), then the pair index p descending, then the head.  Longest
+// causal rows come first (a longest-processing-time order for the persistent
+// grid) and the items of one sequence run close together in time, so its K/V
+// stays in L2 while its heads and pairs reuse it.
+//   cnt[c]   sequences with exactly c pairs            (c = 1 .. P)
+//   start[c] sequences with more than c pairs          (= first sorted slot of bucket c)
+//   B[c]     items of sequences with more than c pairs (= first item of bucket c)
+//   perm     sequence indices sorted by pair count, descending, stable
+__device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, const int *start, const uint16_t *perm,
+                                            int P, int u) {
+    int lo = 1, hi = P;  // smallest c in [1, P] with B[c] <= u
     while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (T[mid] > u) lo = mid; else hi = mid - 1;
+        const int mid = (lo + hi) >> 1;
+        if (B[mid] <= u) hi = mid; else lo = mid + 1;
     }
-    const int pi = lo;
-    const int v = u - T[pi + 1];
-    const int k = v / p.n_head;
+    const int c = lo;
+    const int v = u - B[c];
+    const int per_seq = p.n_head * c;
+    const int ks = v / per_seq;
+    const int w = v - ks * per_seq;
+    const int pw = w / p.n_head;
     Item it;
-    it.h = v - k * p.n_head;
-    it.i = perm[k];
+    it.h = w - pw * p.n_head;
+    it.i = perm[start[c] + ks];
     it.g = it.h / p.group;
-    it.qb0 = 2 * pi;
+    it.qb0 = 2 * (c - 1 - pw);
     it.c0 = p.cu_seqlens[it.i];
     it.n = p.cu_seqlens[it.i + 1] - it.c0;
     it.ctx = p.context_lens ? p.context_lens[it.i] : 0;
@@ -140,8 +150,9 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     volatile int *abort = reinterpret_cast<volatile int *>(gbase + L::ABORT);
-    int *T = reinterpret_cast<int *>(gbase + L::SCHED);
-    int *cur = T + (P + 1);
+    int *B = reinterpret_cast<int *>(gbase + L::SCHED);  // [P + 1]
+    int *start = B + (P + 1);                            // [P + 1]
+    int *cur = start + (P + 1);                          // [P + 1]
     uint16_t *perm = reinterpret_cast<uint16_t *>(cur + (P + 1));
     auto bar = [&](int idx) -> uint32_t { return base + L::BAR + 8u * idx; };
 
@@ -161,7 +172,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int s = 0; s < NST; ++s) {
             mbar_init(bar(L::B_KVFULL + s), 1);
-            mbar_init(bar(L::B_KVEMPTY + s), 1);
+            mbar_init(bar(L::B_KVEMPTY + s), 2);  // MMA commit + KV writer
         }
         *abort = 0;
         fence_mbar_init();
@@ -182,34 +193,29 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     __syncthreads();
     if (warp == 0) {
-        // Two suffix scans over c = P .. 0 in one pass:
-        //   A(c) = sequences with more than c pairs (= those owning pair index c)
-        //        = bucket start of pair count c in the sorted order;
-        //   T[c] = items with pair index >= c = n_head * sum_{c' >= c} A(c').
-        int carry_a = 0, carry_t = 0;
+        // Suffix scans over c = P .. 0 (lane 0 holds the largest c of a chunk):
+        //   start[c] = sum_{c' > c} cnt[c'],  B[c] = n_head * sum_{c' > c} c' cnt[c'].
+        int carry_s = 0, carry_b = 0;
         for (int top = P; top >= 0; top -= 32) {
             const int c = top - lane;
             const int hc = c >= 0 ? cur[c] : 0;
-            int incl = hc;
+            int incl = hc, inclw = hc * (c >= 0 ? c : 0);
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int t = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += t;
+                const int tw = __shfl_up_sync(0xffffffffu, inclw, off);
+                if (lane >= off) {
+                    incl += t;
+                    inclw += tw;
+                }
             }
-            const int a = c >= 0 ? carry_a + incl - hc : 0;
-            int incl_a = a;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, incl_a, off);
-                if (lane >= off) incl_a += t;
-            }
-            __syncwarp();
             if (c >= 0) {
-                T[c] = (carry_t + incl_a) * p.n_head;
-                cur[c] = a;
+                start[c] = carry_s + incl - hc;
+                cur[c] = carry_s + incl - hc;
+                B[c] = (carry_b + inclw - hc * c) * p.n_head;
             }
-            carry_a += __shfl_sync(0xffffffffu, incl, 31);
-            carry_t += __shfl_sync(0xffffffffu, incl_a, 31);
+            carry_s += __shfl_sync(0xffffffffu, incl, 31);
+            carry_b += __shfl_sync(0xffffffffu, inclw, 31);
         }
         __syncwarp();
         // stable counting sort of sequences by pair count, descending
@@ -231,7 +237,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const int total = T[0];
+    const int total = B[0];
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gbase + L::TMEM_SLOT);
     const int G = gridDim.x, cta = blockIdx.x;
 
@@ -252,7 +258,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int k = 0; ok; ++k) {
             const int u = zigzag(k, cta, G);
             if (u >= total) break;
-            const Item it = decode_item(p, T, perm, P, u);
+            const Item it = decode_item(p, B, start, perm, P, u);
             if (s == 1 && !it.two) continue;
             const int qb = it.qb0 + s;
             const int nk = it.nk(s);
@@ -263,13 +269,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tc_fence_after();
                 float x[BN];
                 {
-                    uint32_t r[32];
+                    uint32_t r[BN];
+                    tmem_ld128(tS, r);
 #pragma unroll
-                    for (int c4 = 0; c4 < BN / 32; ++c4) {
-                        tmem_ld32(tS + c4 * 32, r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(r[c]);
-                    }
+                    for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(r[c]);
                 }
                 const KvBlock kb = kv_block(qb, j, it.ctx, it.n, BM, BN);
                 if (!kb.full) {
@@ -278,29 +281,44 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int c = 0; c < BN; ++c)
                         if (c >= lim) x[c] = -CUDART_INF_F;
                 }
-                float mt = x[0];
+                // row max: four independent chains of 3-input max
+                float mt;
+                {
+                    float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
 #pragma unroll
-                for (int c = 1; c < BN; ++c) mt = fmaxf(mt, x[c]);
+                    for (int c = 4; c < BN - 4; c += 8) {
+                        a0 = max3(a0, x[c], x[c + 1]);
+                        a1 = max3(a1, x[c + 2], x[c + 3]);
+                        a2 = max3(a2, x[c + 4], x[c + 5]);
+                        a3 = max3(a3, x[c + 6], x[c + 7]);
+                    }
+                    a0 = max3(a0, x[BN - 4], x[BN - 3]);
+                    a1 = max3(a1, x[BN - 2], x[BN - 1]);
+                    mt = fmaxf(max3(a0, a1, a2), a3);
+                }
                 const bool need = mt > m_run + thr;
                 float m_new = need ? fmaxf(m_run, mt) : m_run;
                 if (m_new == -CUDART_INF_F) m_new = 0.f;
                 const float alpha = need ? ex2((m_run - m_new) * sl2) : 1.f;
                 const float nms = -m_new * sl2;
-                float sum = 0.f;
+                // P = 2^(S*scale*log2e - m*scale*log2e): packed FMA, ex2, packed sums
+                float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
                 {
                     uint32_t pw[32];
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) {
-                            const float p0 = ex2(fmaf(x[half * 64 + 2 * c], sl2, nms));
-                            const float p1 = ex2(fmaf(x[half * 64 + 2 * c + 1], sl2, nms));
-                            sum += p0 + p1;
+                            float y0, y1;
+                            fma2(y0, y1, x[half * 64 + 2 * c], x[half * 64 + 2 * c + 1], sl2, sl2, nms, nms);
+                            const float p0 = ex2(y0), p1 = ex2(y1);
+                            if (c & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
                             pw[c] = pack_bf16x2(p0, p1);
                         }
                         tmem_st32(tS + half * 32, pw);
                     }
                 }
+                const float sum = (sa0 + sa1) + (sb0 + sb1);
                 l_run = l_run * alpha + sum;
                 m_run = m_new;
                 if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -359,7 +377,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item(p, T, perm, P, u);
+                const Item it = decode_item(p, B, start, perm, P, u);
                 const int ns = it.two ? 2 : 1;
                 for (int s = 0; s < ns; ++s) {
                     if (!wait_bar(bar(L::B_QEMPTY + s), ((ph_qe >> s) & 1u) ^ 1u, abort)) { ok = false; break; }
@@ -466,7 +484,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int k = 0; ok; ++k) {
                     const int u = zigzag(k, cta, G);
                     if (u >= total) break;
-                    const Item it = decode_item(p, T, perm, P, u);
+                    const Item it = decode_item(p, B, start, perm, P, u);
                     const int ns = it.two ? 2 : 1;
                     const int nmax = it.nmax();
                     for (int s = 0; s < ns && ok; ++s) {
@@ -536,34 +554,78 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             __syncwarp();
         } else if (warp == WARP_WRITER) {
-            // ================= paged KV write of each item's tokens (one query head per group)
-            constexpr int U = D * 2 / 16;  // 16-byte units per row
+            // ================= paged KV write, fused with the K/V staging: the writer
+            // consumes every stage of the ring; the item's own (diagonal) K and V
+            // tiles are stored from shared memory straight into their cache pages,
+            // whole pages by TMA, a ragged last page (or pages not aligned to the
+            // tile) by plain stores.  One query head per kv group writes.
             const int bs = p.block_size;
-            for (int k = 0;; ++k) {
+            const size_t G_ = p.n_kv_head;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item(p, T, perm, P, u);
-                if (it.h % p.group) continue;
-                const int a0 = it.qb0 * BM;
-                const int a1 = min(a0 + 2 * BM, it.n);
-                const size_t G_ = p.n_kv_head;
-                for (int x = lane; x < (a1 - a0) * U; x += 32) {
-                    const int a = a0 + x / U, un = x % U;
-                    const int P_ = it.ctx + a;
-                    const int page = p.block_table[(size_t)it.i * p.mbps + P_ / bs];
-                    if (page < 0 || page >= p.num_blocks) {
-                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
-                        continue;
+                const Item it = decode_item(p, B, start, perm, P, u);
+                const int nmax = it.nmax();
+                const int np = cdiv(it.ctx, BN);
+                const bool writes = (it.h % p.group) == 0;
+                for (int j = 0; j < nmax && ok; ++j) {
+                    const int jc = j - np;  // chunk block index (negative: prefix)
+                    const bool own = writes && (jc == it.qb0 || (it.two && jc == it.qb0 + 1));
+                    for (int t = 0; t < 2; ++t) {
+                        if (!wait_bar(bar(L::B_KVFULL + stage), phase, abort)) { ok = false; break; }
+                        if (own) {
+                            const uint32_t src = base + L::KV + stage * L::TILE;
+                            const int a0 = jc * BN;                      // first chunk row of the tile
+                            const int rows = min(BN, it.n - a0);         // valid rows
+                            const int P0 = it.ctx + a0;                  // absolute position of row 0
+                            const bool aligned = (P0 % bs) == 0;
+                            const int tma_rows = aligned ? (rows / bs) * bs : 0;
+                            if (lane == 0 && tma_rows > 0) {
+                                for (int r = 0; r < tma_rows; r += bs) {
+                                    const int page = p.block_table[(size_t)it.i * p.mbps + (P0 + r) / bs];
+                                    if (page < 0 || page >= p.num_blocks) {
+                                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                                        continue;
+                                    }
+#pragma unroll
+                                    for (int ch = 0; ch < L::NCH; ++ch)
+                                        tma_store_4d(&tm_cache, src + ch * CHUNK + r * 128, ch * 64, it.g, 0,
+                                                     page * 2 + t);
+                                }
+                                bulk_commit();
+                            }
+                            // remaining rows one 16-byte unit per lane step
+                            const int units = (rows - tma_rows) * 8 * L::NCH;
+                            for (int x = lane; x < units; x += 32) {
+                                const int rr = tma_rows + x / (8 * L::NCH);
+                                const int ch = (x / 8) % L::NCH;
+                                const int un = x % 8;
+                                const int P_ = P0 + rr;
+                                const int page = p.block_table[(size_t)it.i * p.mbps + P_ / bs];
+                                if (page < 0 || page >= p.num_blocks) {
+                                    report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                                    continue;
+                                }
+                                const uint4 val = *reinterpret_cast<const uint4 *>(
+                                    gbase + (src - base) + ch * CHUNK + rr * 128 + ((un ^ (rr & 7)) << 4));
+                                const size_t off =
+                                    ((((size_t)page * 2 + t) * bs + P_ % bs) * G_ + it.g) * D + ch * 64 + un * 8;
+                                *reinterpret_cast<uint4 *>(p.cache + off) = val;
+                            }
+                            if (lane == 0 && tma_rows > 0) bulk_wait_read0();
+                            __syncwarp();
+                        }
+                        if (lane == 0) mbar_arrive(bar(L::B_KVEMPTY + stage));
+                        if (++stage == NST) { stage = 0; phase ^= 1; }
                     }
-                    const size_t src = ((size_t)(it.c0 + a) * G_ + it.g) * D;
-                    const size_t dk = ((((size_t)page * 2 + 0) * bs + P_ % bs) * G_ + it.g) * D;
-                    const size_t dv = ((((size_t)page * 2 + 1) * bs + P_ % bs) * G_ + it.g) * D;
-                    const uint4 kval = reinterpret_cast<const uint4 *>(p.k + src)[un];
-                    const uint4 vval = reinterpret_cast<const uint4 *>(p.v + src)[un];
-                    reinterpret_cast<uint4 *>(p.cache + dk)[un] = kval;
-                    reinterpret_cast<uint4 *>(p.cache + dv)[un] = vval;
                 }
             }
+            if (lane == 0) bulk_wait0();  // stores complete before the kernel ends
+            if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
+            __syncwarp();
         }
     }
 
@@ -574,7 +636,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 template <int D>
 size_t smem_bytes(int P, int num_seqs) {
-    return Lay<D>::SCHED + (size_t)(P + 1) * 8 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
+    return Lay<D>::SCHED + (size_t)(P + 1) * 12 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
 }
 
 int sm_count() {
