@@ -44,6 +44,12 @@ constexpr uint32_t CHUNK = 128 * 128;  // 128 rows x 64 bf16, 128B-swizzled
 // Threshold (log2 units) before the running max is moved and O rescaled;
 // between moves P can reach 2^8, well inside fp32 / bf16 range.
 constexpr float kRescaleLog2 = 8.0f;
+// Which of the 32 column pairs in each 64-column half of an unmasked block take
+// their exponentials on the FMA pipe (exp2_fma2) instead of MUFU (ex2).
+#ifndef PF_EXP2_EMU_MASK
+#define PF_EXP2_EMU_MASK 0x00000000u
+#endif
+constexpr uint32_t kEmuMask = PF_EXP2_EMU_MASK;
 
 template <int D>
 struct Lay {
@@ -51,13 +57,112 @@ struct Lay {
     static constexpr uint32_t TILE = NCH * CHUNK;
     static constexpr uint32_t Q0 = 0, Q1 = TILE, KV = 2 * TILE;
     static constexpr uint32_t BAR = KV + NST * TILE;
-    // barrier slots
+    // barrier slots; P is handed over in two halves (columns 0..63 -> PA, 64..127 -> PB)
     static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NST, B_SFULL = 4 + 2 * NST,
-                         B_PFULL = 6 + 2 * NST, B_OFULL = 8 + 2 * NST, B_OEMPTY = 10 + 2 * NST,
-                         NBAR = 12 + 2 * NST;
+                         B_PA = 6 + 2 * NST, B_PB = 8 + 2 * NST, B_OFULL = 10 + 2 * NST, B_OEMPTY = 12 + 2 * NST,
+                         NBAR = 14 + 2 * NST;
     static constexpr uint32_t TMEM_SLOT = BAR + NBAR * 8, ABORT = TMEM_SLOT + 4;
     static constexpr uint32_t SCHED = BAR + 256;
+    static_assert(ABORT + 4 <= SCHED, "barrier area overflow");
 };
+
+// P = 2^(S*scale*log2e - m*scale*log2e) for 64 columns (half h) of one row:
+// packed FMA, exponentials, packed row sums into (sa*, sb*), bf16 pairs in pw.
+template <int h, bool kEmu>
+__device__ __forceinline__ void exp_half(const float (&x)[BN], float sl2, float nms, uint32_t (&pw)[32], float &sa0,
+                                         float &sa1, float &sb0, float &sb1) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        float y0, y1, p0, p1;
+        fma2(y0, y1, x[h * 64 + 2 * c], x[h * 64 + 2 * c + 1], sl2, sl2, nms, nms);
+        if (kEmu && ((kEmuMask >> c) & 1u)) {
+            exp2_fma2(y0, y1, p0, p1);
+        } else {
+            p0 = ex2(y0);
+            p1 = ex2(y1);
+        }
+        if (c & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
+        pw[c] = pack_bf16x2(p0, p1);
+    }
+}
+
+// Row max of 128 scores: four independent chains of 3-input max.
+__device__ __forceinline__ float rowmax128(const float (&x)[BN]) {
+    float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+#pragma unroll
+    for (int c = 4; c < BN - 4; c += 8) {
+        a0 = max3(a0, x[c], x[c + 1]);
+        a1 = max3(a1, x[c + 2], x[c + 3]);
+        a2 = max3(a2, x[c + 4], x[c + 5]);
+        a3 = max3(a3, x[c + 6], x[c + 7]);
+    }
+    a0 = max3(a0, x[BN - 4], x[BN - 3]);
+    a1 = max3(a1, x[BN - 2], x[BN - 1]);
+    return fmaxf(max3(a0, a1, a2), a3);
+}
+
+// Online softmax of one kv block for one row (one thread), then P to TMEM in
+// two halves, each announced on its own barrier so that the P.V MMA can start
+// on the first half while the second is computed.
+//
+// The exponentials are taken against the running max m_run without waiting
+// for this block's max: the running max only moves when the block max exceeds
+// it by more than the threshold (2^8 in P), and only then is half 0 redone
+// and O rescaled.  Blocks whose max stays below that bound give P up to 2^8,
+// which the final O / l divides out exactly (same max for P and l).
+template <int D, bool kFull>
+__device__ __forceinline__ void softmax_block(const float (&x)[BN], int j, float sl2, float thr, float &m_run,
+                                              float &l_run, uint32_t tS, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
+                                              int lane) {
+    const bool first = j == 0;
+    float mt = first ? rowmax128(x) : 0.f;
+    float m_ref = first ? mt : m_run;
+    if (m_ref == -CUDART_INF_F) m_ref = 0.f;  // nothing visible yet (cannot happen under causal masking)
+    float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+    {
+        uint32_t pw[32];
+        exp_half<0, kFull>(x, sl2, -m_ref * sl2, pw, sa0, sa1, sb0, sb1);
+        tmem_st32(tS, pw);
+    }
+    float m_new = m_ref, alpha = first ? 0.f : 1.f;
+    if (!first) {
+        mt = rowmax128(x);
+        const bool need = mt > m_run + thr;
+        if (__any_sync(0xffffffffu, need)) {
+            // the max moved by more than the threshold: redo half 0 (stored again
+            // over the first attempt) and rescale O before P.V touches it
+            m_new = need ? mt : m_run;
+            alpha = ex2((m_run - m_new) * sl2);
+            sa0 = sa1 = sb0 = sb1 = 0.f;
+            {
+                uint32_t pw[32];
+                exp_half<0, kFull>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
+                tmem_st32(tS, pw);
+            }
+#pragma unroll 1
+            for (int cc = 0; cc < D / 16; ++cc) {
+                uint32_t r[16];
+                tmem_ld16(tO + cc * 16, r);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+                tmem_st16(tO + cc * 16, r);
+            }
+        }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_pa);
+    uint32_t pw[32];
+    exp_half<1, kFull>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
+    tmem_st32(tS + 32, pw);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_pb);
+    l_run = l_run * alpha + ((sa0 + sa1) + (sb0 + sb1));
+    m_run = m_new;
+}
 
 // ------------------------------------------------------------------ schedule
 struct Item {
@@ -166,7 +271,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar(L::B_QFULL + s), 1);
             mbar_init(bar(L::B_QEMPTY + s), 1);
             mbar_init(bar(L::B_SFULL + s), 1);
-            mbar_init(bar(L::B_PFULL + s), 4);
+            mbar_init(bar(L::B_PA + s), 4);
+            mbar_init(bar(L::B_PB + s), 4);
             mbar_init(bar(L::B_OFULL + s), 1);
             mbar_init(bar(L::B_OEMPTY + s), 4);
         }
@@ -249,7 +355,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + 128u * s + lane_off;
         const uint32_t tO = tmem + 256u + 128u * s + lane_off;
-        const uint32_t b_sfull = bar(L::B_SFULL + s), b_pfull = bar(L::B_PFULL + s);
+        const uint32_t b_sfull = bar(L::B_SFULL + s), b_pa = bar(L::B_PA + s), b_pb = bar(L::B_PB + s);
         const uint32_t b_ofull = bar(L::B_OFULL + s), b_oempty = bar(L::B_OEMPTY + s);
         const float sl2 = p.scale_log2;
         const float thr = kRescaleLog2 / sl2;  // the threshold in raw score units
@@ -281,60 +387,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int c = 0; c < BN; ++c)
                         if (c >= lim) x[c] = -CUDART_INF_F;
                 }
-                // row max: four independent chains of 3-input max
-                float mt;
-                {
-                    float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
-#pragma unroll
-                    for (int c = 4; c < BN - 4; c += 8) {
-                        a0 = max3(a0, x[c], x[c + 1]);
-                        a1 = max3(a1, x[c + 2], x[c + 3]);
-                        a2 = max3(a2, x[c + 4], x[c + 5]);
-                        a3 = max3(a3, x[c + 6], x[c + 7]);
-                    }
-                    a0 = max3(a0, x[BN - 4], x[BN - 3]);
-                    a1 = max3(a1, x[BN - 2], x[BN - 1]);
-                    mt = fmaxf(max3(a0, a1, a2), a3);
-                }
-                const bool need = mt > m_run + thr;
-                float m_new = need ? fmaxf(m_run, mt) : m_run;
-                if (m_new == -CUDART_INF_F) m_new = 0.f;
-                const float alpha = need ? ex2((m_run - m_new) * sl2) : 1.f;
-                const float nms = -m_new * sl2;
-                // P = 2^(S*scale*log2e - m*scale*log2e): packed FMA, ex2, packed sums
-                float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-                {
-                    uint32_t pw[32];
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            float y0, y1;
-                            fma2(y0, y1, x[half * 64 + 2 * c], x[half * 64 + 2 * c + 1], sl2, sl2, nms, nms);
-                            const float p0 = ex2(y0), p1 = ex2(y1);
-                            if (c & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
-                            pw[c] = pack_bf16x2(p0, p1);
-                        }
-                        tmem_st32(tS + half * 32, pw);
-                    }
-                }
-                const float sum = (sa0 + sa1) + (sb0 + sb1);
-                l_run = l_run * alpha + sum;
-                m_run = m_new;
-                if (j > 0 && __any_sync(0xffffffffu, need)) {
-                    uint32_t r[32];
-#pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        tmem_ld32(tO + cc * 32, r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-                        tmem_st32(tO + cc * 32, r);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(b_pfull);
+                if (kb.full) softmax_block<D, true>(x, j, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
+                else softmax_block<D, false>(x, j, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
             }
             if (!ok) break;
             // final O / l -> bf16 rows of out
@@ -458,100 +512,108 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
         } else if (warp == WARP_MMA) {
-            // ================= tcgen05 MMA issuer (lane 0)
-            if (lane == 0) {
-                int stage = 0;
-                // per-query-block phase bits (bit s) and "O already used" bits
-                uint32_t phase = 0, ph_qf = 0, ph_pf = 0, ph_oe = 0, used = 0;
-                bool ok = true;
-                auto kv_wait = [&](int st, uint32_t ph) { return wait_bar(bar(L::B_KVFULL + st), ph, abort); };
-                auto issue_s = [&](int s, int kst) {
-                    const uint32_t q = base + (s ? L::Q1 : L::Q0), kk_ = base + L::KV + kst * L::TILE;
+            // ================= tcgen05 MMA issuer: the whole warp runs the loop with
+            // warp-uniform descriptors; one elected lane issues each instruction.
+            int stage = 0;
+            // per-query-block phase bits (bit s) and "O already used" bits
+            uint32_t phase = 0, ph_qf = 0, ph_pf = 0, ph_oe = 0, used = 0;
+            bool ok = true;
+            auto wait_all = [&](uint32_t b, uint32_t par) {
+                return __all_sync(0xffffffffu, wait_bar(b, par, abort));
+            };
+            const uint64_t dq0 = smem_desc_sw128(base + L::Q0, 16, 1024);
+            const uint64_t dq1 = smem_desc_sw128(base + L::Q1, 16, 1024);
+            auto issue_s = [&](int s, int kst) {
+                const uint64_t dq = s ? dq1 : dq0;
+                const uint64_t dk = smem_desc_sw128(base + L::KV + kst * L::TILE, 16, 1024);
+                const uint32_t d = tmem + 128u * s;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-                        mma_ss(tmem + 128u * s, smem_desc_sw128(q + off, 16, 1024),
-                               smem_desc_sw128(kk_ + off, 16, 1024), IDESC_QK, kk > 0);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+                    mma_ss_elect(d, dq + off, dk + off, IDESC_QK, kk > 0);
+                }
+            };
+            // k-steps [k0, k0 + 4) of O_s += P_s V (16 keys each): one half of P
+            auto issue_pv = [&](int s, int vst, bool acc, int k0) {
+                const uint64_t dv = smem_desc_sw128(base + L::KV + vst * L::TILE, CHUNK, 1024);
+                const uint32_t d = tmem + 256u + 128u * s, a = tmem + 128u * s;
+#pragma unroll
+                for (int kk = k0; kk < k0 + BN / 32; ++kk)
+                    mma_ts_elect(d, a + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            };
+            for (int k = 0; ok; ++k) {
+                const int u = zigzag(k, cta, G);
+                if (u >= total) break;
+                const Item it = decode_item(p, B, start, perm, P, u);
+                const int ns = it.two ? 2 : 1;
+                const int nmax = it.nmax();
+                for (int s = 0; s < ns && ok; ++s) {
+                    ok = wait_all(bar(L::B_QFULL + s), (ph_qf >> s) & 1u);
+                    ph_qf ^= 1u << s;
+                }
+                if (!ok) break;
+                // K_0
+                const int kst = stage;
+                const uint32_t kph = phase;
+                if (++stage == NST) { stage = 0; phase ^= 1; }
+                if (!wait_all(bar(L::B_KVFULL + kst), kph)) { ok = false; break; }
+                tc_fence_after();
+                for (int s = 0; s < ns; ++s) {
+                    issue_s(s, kst);
+                    tc_commit_elect(bar(L::B_SFULL + s));
+                }
+                tc_commit_elect(bar(L::B_KVEMPTY + kst));
+                for (int j = 0; j < nmax && ok; ++j) {
+                    const int vst = stage;
+                    const uint32_t vph = phase;
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
+                    int nst = -1;
+                    uint32_t nph = 0;
+                    if (j + 1 < nmax) {
+                        nst = stage;
+                        nph = phase;
+                        if (++stage == NST) { stage = 0; phase ^= 1; }
                     }
-                };
-                auto issue_pv = [&](int s, int vst, bool acc) {
-                    const uint32_t vv = base + L::KV + vst * L::TILE;
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tmem + 256u + 128u * s, tmem + 128u * s + kk * 8,
-                               smem_desc_sw128(vv + kk * 2048, CHUNK, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-                };
-                for (int k = 0; ok; ++k) {
-                    const int u = zigzag(k, cta, G);
-                    if (u >= total) break;
-                    const Item it = decode_item(p, B, start, perm, P, u);
-                    const int ns = it.two ? 2 : 1;
-                    const int nmax = it.nmax();
-                    for (int s = 0; s < ns && ok; ++s) {
-                        ok = wait_bar(bar(L::B_QFULL + s), (ph_qf >> s) & 1u, abort);
-                        ph_qf ^= 1u << s;
+                    if (!wait_all(bar(L::B_KVFULL + vst), vph)) { ok = false; break; }
+                    bool next_ready = false;
+                    for (int s = 0; s < ns; ++s) {
+                        if (j >= it.nk(s)) continue;
+                        if (!wait_all(bar(L::B_PA + s), (ph_pf >> s) & 1u)) { ok = false; break; }
+                        if (j == 0 && ((used >> s) & 1u)) {
+                            if (!wait_all(bar(L::B_OEMPTY + s), (ph_oe >> s) & 1u)) { ok = false; break; }
+                            ph_oe ^= 1u << s;
+                        }
+                        tc_fence_after();
+                        issue_pv(s, vst, j > 0, 0);
+                        if (!wait_all(bar(L::B_PB + s), (ph_pf >> s) & 1u)) { ok = false; break; }
+                        ph_pf ^= 1u << s;
+                        tc_fence_after();
+                        issue_pv(s, vst, j > 0, BN / 32);
+                        if (j + 1 < it.nk(s)) {
+                            if (!next_ready) {
+                                if (!wait_all(bar(L::B_KVFULL + nst), nph)) { ok = false; break; }
+                                tc_fence_after();
+                                next_ready = true;
+                            }
+                            issue_s(s, nst);
+                            tc_commit_elect(bar(L::B_SFULL + s));
+                        } else {
+                            tc_commit_elect(bar(L::B_OFULL + s));
+                            tc_commit_elect(bar(L::B_QEMPTY + s));
+                        }
                     }
                     if (!ok) break;
-                    // K_0
-                    int kst = stage;
-                    uint32_t kph = phase;
-                    if (++stage == NST) { stage = 0; phase ^= 1; }
-                    if (!kv_wait(kst, kph)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int s = 0; s < ns; ++s) {
-                        issue_s(s, kst);
-                        tc_commit(bar(L::B_SFULL + s));
+                    tc_commit_elect(bar(L::B_KVEMPTY + vst));
+                    if (nst >= 0) {
+                        if (!next_ready) {  // no query block needed K_{j+1}: still consume the stage in order
+                            if (!wait_all(bar(L::B_KVFULL + nst), nph)) { ok = false; break; }
+                        }
+                        tc_commit_elect(bar(L::B_KVEMPTY + nst));
                     }
-                    tc_commit(bar(L::B_KVEMPTY + kst));
-                    for (int j = 0; j < nmax && ok; ++j) {
-                        const int vst = stage;
-                        const uint32_t vph = phase;
-                        if (++stage == NST) { stage = 0; phase ^= 1; }
-                        int nst = -1;
-                        uint32_t nph = 0;
-                        if (j + 1 < nmax) {
-                            nst = stage;
-                            nph = phase;
-                            if (++stage == NST) { stage = 0; phase ^= 1; }
-                        }
-                        if (!kv_wait(vst, vph)) { ok = false; break; }
-                        bool next_ready = false;
-                        for (int s = 0; s < ns; ++s) {
-                            if (j >= it.nk(s)) continue;
-                            if (!wait_bar(bar(L::B_PFULL + s), (ph_pf >> s) & 1u, abort)) { ok = false; break; }
-                            ph_pf ^= 1u << s;
-                            if (j == 0 && ((used >> s) & 1u)) {
-                                if (!wait_bar(bar(L::B_OEMPTY + s), (ph_oe >> s) & 1u, abort)) { ok = false; break; }
-                                ph_oe ^= 1u << s;
-                            }
-                            tc_fence_after();
-                            issue_pv(s, vst, j > 0);
-                            if (j + 1 < it.nk(s)) {
-                                if (!next_ready) {
-                                    if (!kv_wait(nst, nph)) { ok = false; break; }
-                                    tc_fence_after();
-                                    next_ready = true;
-                                }
-                                issue_s(s, nst);
-                                tc_commit(bar(L::B_SFULL + s));
-                            } else {
-                                tc_commit(bar(L::B_OFULL + s));
-                                tc_commit(bar(L::B_QEMPTY + s));
-                            }
-                        }
-                        if (!ok) break;
-                        tc_commit(bar(L::B_KVEMPTY + vst));
-                        if (nst >= 0) {
-                            if (!next_ready) {  // no slot needed K_{j+1}: still wait so the stage is consumed in order
-                                if (!kv_wait(nst, nph)) { ok = false; break; }
-                            }
-                            tc_commit(bar(L::B_KVEMPTY + nst));
-                        }
-                    }
-                    used |= it.two ? 3u : 1u;
                 }
-                if (!ok) report(p.status, PREFILL_ERR_TIMEOUT);
+                used |= it.two ? 3u : 1u;
             }
+            if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
             __syncwarp();
         } else if (warp == WARP_WRITER) {
             // ================= paged KV write, fused with the K/V staging: the writer

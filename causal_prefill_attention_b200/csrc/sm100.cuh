@@ -141,6 +141,37 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// Elected-lane variants: called by a whole converged warp; elect.sync picks
+// one lane (the same one every time for a full, converged warp) to issue the
+// instruction, so the operands stay warp-uniform.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
 // Instruction descriptor for kind::f16: bf16 A and B, fp32 accumulator,
 // M x N tile; a_mn / b_mn select MN-major (transposed) operands.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
@@ -215,6 +246,26 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
 #undef PF_R8
 #undef PF_O32
 
+// 16-column variants (fewer live registers).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -253,6 +304,34 @@ __device__ __forceinline__ void add2(float &a0, float &a1, float b0, float b1) {
         "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
         : "+f"(a0), "+f"(a1)
         : "f"(b0), "f"(b1));
+}
+
+// 2^y0, 2^y1 on the FMA pipe, for y in [-125, 127] (inputs below -125 are
+// clamped: the result is then 2^-125 instead of ~0).  Cody-Waite style range
+// reduction (Cody & Waite, "Software Manual for the Elementary Functions",
+// 1980): y = j + f with j = round(y), obtained by adding 1.5 * 2^23 so that the
+// integer lands in the low mantissa bits, and f in [-1/2, 1/2]; 2^f from a
+// cubic fitted for this code by Lawson's iteratively reweighted least squares
+// (max relative error 8.4e-5 evaluated in fp32 Horner form); j is then added
+// to the exponent field.  Used to move part of the exponentials off MUFU.
+__device__ __forceinline__ void exp2_fma2(float y0, float y1, float &r0, float &r1) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0.999919593334198f, c1 = 0.6932621598243713f, c2 = 0.24271413683891296f,
+                    c3 = 0.055212993174791336f;
+    y0 = fmaxf(y0, -125.f);
+    y1 = fmaxf(y1, -125.f);
+    float t0 = y0, t1 = y1;
+    add2(t0, t1, kMagic, kMagic);  // round(y) in the low bits of t
+    float j0 = t0, j1 = t1;
+    add2(j0, j1, -kMagic, -kMagic);  // round(y) as a float
+    float f0, f1;
+    fma2(f0, f1, j0, j1, -1.f, -1.f, y0, y1);  // f = y - round(y)
+    float p0, p1;
+    fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+    fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ void report(int32_t *status, int code) {
