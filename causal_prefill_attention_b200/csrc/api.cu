@@ -79,16 +79,21 @@ int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int
 
     pf::TensorMaps maps;
     const cuuint64_t D = head_dim, H = n_head, G = n_kv_head, T = total;
+    // q / k / v: {64 columns, head, token, 64-column chunk}; the chunk is the
+    // outermost dimension (stride 128 B), so one box {64, 1, 128, D/64} lands a
+    // whole 128-row tile chunk-major: D/64 blocks of 128 rows x 128 B, each
+    // 128-byte swizzled -- the layout the MMA descriptors expect.
+    const cuuint64_t NCH = D / 64;
     {
-        const cuuint64_t dims[3] = {D, H, T}, strides[2] = {D * 2, H * D * 2};
-        const cuuint32_t box[3] = {64, 1, 128};
-        if (!encode(&maps.q, q, 3, dims, strides, box)) return PREFILL_ERR_CUDA;
+        const cuuint64_t dims[4] = {64, H, T, NCH}, strides[3] = {D * 2, H * D * 2, 128};
+        const cuuint32_t box[4] = {64, 1, 128, (cuuint32_t)NCH};
+        if (!encode(&maps.q, q, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
     {
-        const cuuint64_t dims[3] = {D, G, T}, strides[2] = {D * 2, G * D * 2};
-        const cuuint32_t box[3] = {64, 1, 128};
-        if (!encode(&maps.k, k, 3, dims, strides, box)) return PREFILL_ERR_CUDA;
-        if (!encode(&maps.v, v, 3, dims, strides, box)) return PREFILL_ERR_CUDA;
+        const cuuint64_t dims[4] = {64, G, T, NCH}, strides[3] = {D * 2, G * D * 2, 128};
+        const cuuint32_t box[4] = {64, 1, 128, (cuuint32_t)NCH};
+        if (!encode(&maps.k, k, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
+        if (!encode(&maps.v, v, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
     {
         const cuuint64_t dims[4] = {D, G, (cuuint64_t)bs, (cuuint64_t)num_blocks * 2};

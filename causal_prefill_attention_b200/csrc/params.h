@@ -27,9 +27,9 @@ struct FwdParams {
 };
 
 struct TensorMaps {
-    CUtensorMap q;      // {D, H, T}, box {64, 1, 128}
-    CUtensorMap k;      // {D, G, T}, box {64, 1, 128}
-    CUtensorMap v;      // {D, G, T}, box {64, 1, 128}
+    CUtensorMap q;      // {64, H, T, D/64} (chunk outermost), box {64, 1, 128, D/64}
+    CUtensorMap k;      // {64, G, T, D/64}, box {64, 1, 128, D/64}
+    CUtensorMap v;      // {64, G, T, D/64}, box {64, 1, 128, D/64}
     CUtensorMap cache;  // {D, G, bs, 2*NB}, box {64, 1, bs, 1}
 };
 

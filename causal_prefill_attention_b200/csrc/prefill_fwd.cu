@@ -37,7 +37,10 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int NST = 4;  // K/V ring stages (each one K or one V tile)
+#ifndef PF_KV_STAGES
+#define PF_KV_STAGES 4
+#endif
+constexpr int NST = PF_KV_STAGES;  // K/V ring stages (each one K or one V tile)
 constexpr int NTHREADS = 384;
 constexpr int WARP_PRODUCER = 8, WARP_MMA = 9, WARP_WRITER = 10;
 constexpr uint32_t CHUNK = 128 * 128;  // 128 rows x 64 bf16, 128B-swizzled
@@ -235,8 +238,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
-__device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
-__device__ __forceinline__ void setmaxnreg_dec88() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
+// Register split (the launch gives 384 threads x 168 = 64,512 registers):
+// softmax warpgroups 2 x 128 x 200 + control warpgroup 128 x 104 = 64,512.
+__device__ __forceinline__ void setmaxnreg_softmax() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;"); }
+__device__ __forceinline__ void setmaxnreg_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;"); }
 
 // ------------------------------------------------------------------ kernel
 template <int D>
@@ -349,7 +354,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (warp < 8) {
         // ================= softmax / rescale / epilogue for query block s
-        setmaxnreg_inc208();
+        setmaxnreg_softmax();
         const int s = warp >> 2;
         const int row = tid & 127;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -421,12 +426,15 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         if (!ok && (tid & 127) == 0) report(p.status, PREFILL_ERR_TIMEOUT);
     } else {
-        setmaxnreg_dec88();
+        setmaxnreg_control();
         if (warp == WARP_PRODUCER) {
             // ================= TMA producer (all lanes loop; lane 0 issues)
             const int bs = p.block_size;
             int stage = 0;
             uint32_t phase = 0, ph_qe = 0;  // bit s: phase of Q block s
+            // stages / Q buffers filled at least once, and the phase of their last
+            // fill: drained before exit so that no copy is in flight when the CTA ends
+            uint32_t kv_filled = 0, kv_lastph = 0, q_filled = 0, q_lastph = 0;
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
@@ -435,14 +443,13 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int ns = it.two ? 2 : 1;
                 for (int s = 0; s < ns; ++s) {
                     if (!wait_bar(bar(L::B_QEMPTY + s), ((ph_qe >> s) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    q_filled |= 1u << s;
+                    q_lastph = (q_lastph & ~(1u << s)) | (((ph_qe >> s) & 1u) << s);
                     ph_qe ^= 1u << s;
                     if (lane == 0) {
                         const uint32_t b = bar(L::B_QFULL + s);
                         mbar_expect_tx(b, L::TILE);
-#pragma unroll
-                        for (int ch = 0; ch < L::NCH; ++ch)
-                            tma_load_3d(base + (s ? L::Q1 : L::Q0) + ch * CHUNK, &tm_q, b, ch * 64, it.h,
-                                        it.c0 + (it.qb0 + s) * BM);
+                        tma_load_4d(base + (s ? L::Q1 : L::Q0), &tm_q, b, 0, it.h, it.c0 + (it.qb0 + s) * BM, 0);
                     }
                 }
                 const int nmax = it.nmax();
@@ -452,13 +459,12 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         if (!wait_bar(bar(L::B_KVEMPTY + stage), phase ^ 1, abort)) { ok = false; break; }
                         const uint32_t dst = base + L::KV + stage * L::TILE;
                         const uint32_t b = bar(L::B_KVFULL + stage);
+                        kv_filled |= 1u << stage;
+                        kv_lastph = (kv_lastph & ~(1u << stage)) | (phase << stage);
                         if (!kb.prefix) {
                             if (lane == 0) {
                                 mbar_expect_tx(b, L::TILE);
-#pragma unroll
-                                for (int ch = 0; ch < L::NCH; ++ch)
-                                    tma_load_3d(dst + ch * CHUNK, t ? &tm_v : &tm_k, b, ch * 64, it.g,
-                                                it.c0 + kb.src_row);
+                                tma_load_4d(dst, t ? &tm_v : &tm_k, b, 0, it.g, it.c0 + kb.src_row, 0);
                             }
                         } else {
                             // prefix: whole pages by TMA; the rest of the block (a partly
@@ -510,6 +516,12 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                 }
             }
+            // drain: every copy this warp issued has landed before the CTA can exit
+            // (immediate on the normal path, where the consumers waited for them)
+            for (int st = 0; st < NST; ++st)
+                if ((kv_filled >> st) & 1u) mbar_wait(bar(L::B_KVFULL + st), (kv_lastph >> st) & 1u);
+            for (int s = 0; s < 2; ++s)
+                if ((q_filled >> s) & 1u) mbar_wait(bar(L::B_QFULL + s), (q_lastph >> s) & 1u);
             if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
         } else if (warp == WARP_MMA) {
             // ================= tcgen05 MMA issuer: the whole warp runs the loop with

@@ -92,9 +92,7 @@ prefill_fwd_v0_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ---- Q block
     if (tid == 0) {
         mbar_expect_tx(bar_load, L::TILE);
-#pragma unroll
-        for (int ch = 0; ch < L::NCH; ++ch)
-            tma_load_3d(sQ + ch * CHUNK_BYTES, &tm_q, bar_load, ch * 64, h, c0 + qb * BM);
+        tma_load_4d(sQ, &tm_q, bar_load, 0, h, c0 + qb * BM, 0);
     }
     ok = __syncthreads_and(mbar_wait(bar_load, ph_load));
     ph_load ^= 1;
@@ -126,11 +124,8 @@ prefill_fwd_v0_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             } else {
                 mbar_expect_tx(bar_load, 2u * L::TILE);
-#pragma unroll
-                for (int ch = 0; ch < L::NCH; ++ch) {
-                    tma_load_3d(sK + ch * CHUNK_BYTES, &tm_k, bar_load, ch * 64, g, c0 + kb.src_row);
-                    tma_load_3d(sV + ch * CHUNK_BYTES, &tm_v, bar_load, ch * 64, g, c0 + kb.src_row);
-                }
+                tma_load_4d(sK, &tm_k, bar_load, 0, g, c0 + kb.src_row, 0);
+                tma_load_4d(sV, &tm_v, bar_load, 0, g, c0 + kb.src_row, 0);
             }
         }
         ok = __syncthreads_and(mbar_wait(bar_load, ph_load));
