@@ -36,6 +36,20 @@ METRIC = "prefill attention TFLOP/s & % of B200 BF16 tensor peak; prompt tokens/
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
 
+def kernel_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    record, if the kernel sources are unchanged since it was taken; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    h = hashlib.sha256()
+    for f in rec["source_files"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return rec["traffic_bytes"] if h.hexdigest()[:16] == rec["source_sha256_16"] else None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -59,7 +73,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (FileNotFoundError, OSError):
             self.proc = None
         return self
@@ -249,7 +263,7 @@ def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -341,7 +355,9 @@ def main():
             "pct_of_peak": round(100.0 * tflops / pk["bf16"], 2),
             "prompt_tokens_per_s": round(tokens_s, 1),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": pk["bf16"], "unit": "TFLOP/s",
-                         "frac": round(tflops / pk["bf16"], 4), "traffic": None,
+                         "frac": round(tflops / pk["bf16"], 4),
+                         "traffic": kernel_traffic() if args.workload == HEADLINE else None,
+                         "algorithmic_bytes": (4 * w.n_head + 8 * w.n_kv_head) * w.head_dim * w.total_tokens,
                          "peak_source": f"{pk['source']} bf16 burst (kernel timed alone)"},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_tflops, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),

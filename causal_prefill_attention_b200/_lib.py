@@ -19,7 +19,7 @@ STATUS_NAMES = {
     4: "PREFILL_ERR_BLOCK_TABLE", 5: "PREFILL_ERR_CUDA", 6: "PREFILL_ERR_TIMEOUT", 7: "PREFILL_ERR_ALIGNMENT",
 }
 EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
-            "prefill_num_kv_blocks", "prefill_kv_block_rule")
+            "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall")
 
 _lib = None
 
@@ -48,6 +48,8 @@ def load() -> ctypes.CDLL:
         lib.prefill_num_kv_blocks.restype = I
         lib.prefill_kv_block_rule.argtypes = [I, I, I, I, I, I, P, P]
         lib.prefill_kv_block_rule.restype = I
+        lib.prefill_test_inject_stall.argtypes = [I]
+        lib.prefill_test_inject_stall.restype = None
         _lib = lib
     return _lib
 
@@ -119,6 +121,12 @@ def prefill_attn_chunked(q, k, v, cu_seqlens_q, context_lens, max_q_len: int, ma
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "prefill_attn_chunked")
     return rc
+
+
+def inject_stall(enable: bool = True) -> None:
+    """Test hook: the next pipelined launch withholds one Q tile so that a
+    bounded device wait expires and the call reports PREFILL_ERR_TIMEOUT."""
+    load().prefill_test_inject_stall(1 if enable else 0)
 
 
 def num_kv_blocks(qb: int, ctx: int, n: int, bm: int = 128, bn: int = 128) -> int:

@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/prefill.h"
@@ -54,6 +55,8 @@ bool use_pipelined() {
     }
     return v == 1;
 }
+
+std::atomic<int> g_test_stall{0};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -121,6 +124,7 @@ int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int
     p.block_size = bs;
     p.max_q = max_q;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.test_stall = g_test_stall.exchange(0);
 
     int e = (use_pipelined() && pf::fwd_pipelined_supported(p, head_dim))
                 ? pf::launch_fwd(maps, p, head_dim, stream)
@@ -151,6 +155,8 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
                n_kv_head, head_dim, scale, out, kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
                status_dev, stream);
 }
+
+void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }
 
 const char *prefill_status_string(int s) {
     switch (s) {

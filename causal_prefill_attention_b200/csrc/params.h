@@ -24,6 +24,7 @@ struct FwdParams {
     int block_size;
     int max_q;                    // bound on every sequence (chunk) length
     float scale_log2;             // scale * log2(e)
+    int test_stall;               // test hook: withhold one Q tile (see prefill_test_inject_stall)
 };
 
 struct TensorMaps {

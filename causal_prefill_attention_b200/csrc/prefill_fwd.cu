@@ -228,12 +228,10 @@ __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, co
 __device__ __forceinline__ int zigzag(int k, int c, int G) { return k * G + ((k & 1) ? (G - 1 - c) : c); }
 
 // ------------------------------------------------------------------ waits
+// Bounded wait that also stops when another role has given up; the first
+// role to run out of time raises the CTA's abort flag.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort) {
-#pragma unroll 1
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *abort) return false;
-    }
+    if (mbar_wait(bar, parity, abort)) return true;
     *abort = 1;
     return false;
 }
@@ -443,6 +441,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int ns = it.two ? 2 : 1;
                 for (int s = 0; s < ns; ++s) {
                     if (!wait_bar(bar(L::B_QEMPTY + s), ((ph_qe >> s) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    if (p.test_stall && cta == 0 && k == 0 && s == 0) {
+                        // test hook: withhold this Q tile so that the MMA warp's wait expires
+                        ph_qe ^= 1u << s;
+                        continue;
+                    }
                     q_filled |= 1u << s;
                     q_lastph = (q_lastph & ~(1u << s)) | (((ph_qe >> s) & 1u) << s);
                     ph_qe ^= 1u << s;

@@ -1,7 +1,7 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
 // attention kernels use: mbarriers, TMA tensor loads, tcgen05 MMA / TMEM.
 //
-// Every wait on an mbarrier is bounded: after kSpinLimit failed polls it gives
+// Every wait on an mbarrier is bounded in time: after about a second it gives
 // up and the caller records PREFILL_ERR_TIMEOUT instead of hanging the GPU.
 #pragma once
 #include <cstdint>
@@ -9,10 +9,9 @@
 
 namespace pf {
 
-// ~4M polls; each poll of try_wait may suspend the thread for a short,
-// hardware-chosen time, so the limit is well above any legitimate wait
-// (microseconds) and well below a watchdog (seconds).
-constexpr uint32_t kSpinLimit = 1u << 22;
+// Every wait gives up after about one second of wall-clock time (far above
+// any legitimate wait, which lasts microseconds, and far below a watchdog).
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -43,12 +42,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for the phase with the given parity to complete; false after
+// kWaitLimitNs, or as soon as *abort becomes non-zero (when abort is given).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int *abort = nullptr) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-    return false;
+        if ((i & 255u) == 0) {
+            if (abort && *abort) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        }
+    }
 }
 
 // ------------------------------------------------------------------ fences

@@ -139,6 +139,18 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
                          const int32_t *block_table, int max_blocks_per_seq, int block_size,
                          int32_t *status_dev, prefill_stream_t stream);
 
+/*
+ * Test hook for the failure path (no counterpart on the pages).  With enable
+ * != 0, the next prefill_attn / prefill_attn_chunked launch that uses the
+ * pipelined kernel withholds its first Q tile in CTA 0, so that the consumer's
+ * bounded wait (about one second) expires: every role of the kernel then stops,
+ * drains its copies, frees its tensor memory and returns, and *status_dev
+ * reads PREFILL_ERR_TIMEOUT.  The hook resets itself after one launch.  It makes
+ * no fault and no hang; it exists so tests can check that a stalled pipeline is
+ * reported and that the CUDA context stays usable.
+ */
+void prefill_test_inject_stall(int enable);
+
 /* Human-readable name of a prefill_status value (static storage). */
 const char *prefill_status_string(int status);
 
