@@ -9,7 +9,9 @@
 #include <cstring>
 #include <cstdint>
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "../../include/prefill.h"
 #include "block_rule.h"
@@ -57,6 +59,38 @@ bool use_pipelined() {
 }
 
 std::atomic<int> g_test_stall{0};
+
+// Split-KV workspace: one device buffer per (device, stream), allocated on the
+// first call that splits and grown when a larger call needs more.  Kept for
+// later calls; a separate buffer per stream keeps concurrent streams apart.
+struct Workspace {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<std::pair<int, void *>, Workspace> g_ws;
+
+void *split_workspace(size_t bytes, void *stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    Workspace &w = g_ws[{dev, stream}];
+    if (w.bytes < bytes) {
+        if (w.ptr) {
+            cudaStreamSynchronize(static_cast<cudaStream_t>(stream));  // earlier calls may still read it
+            cudaFree(w.ptr);
+            w.ptr = nullptr;
+            w.bytes = 0;
+        }
+        if (cudaMalloc(&w.ptr, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            w.ptr = nullptr;
+            return nullptr;
+        }
+        w.bytes = bytes;
+    }
+    return w.ptr;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -125,10 +159,28 @@ int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int
     p.max_q = max_q;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.test_stall = g_test_stall.exchange(0);
+    p.max_ctx = (int)max_ctx;
+    p.nsplit = 1;
+    p.part_o = nullptr;
+    p.part_ml = nullptr;
 
-    int e = (use_pipelined() && pf::fwd_pipelined_supported(p, head_dim))
-                ? pf::launch_fwd(maps, p, head_dim, stream)
-                : pf::launch_fwd_v0(maps, p, head_dim, stream);
+    int e;
+    if (use_pipelined() && pf::fwd_pipelined_supported(p, head_dim)) {
+        p.nsplit = pf::fwd_choose_splits(p);
+        if (p.nsplit > 1) {
+            const size_t o_bytes = (size_t)p.nsplit * p.total * p.n_head * head_dim * sizeof(float);
+            char *ws = static_cast<char *>(split_workspace(pf::fwd_split_workspace_bytes(p, head_dim), stream));
+            if (ws) {
+                p.part_o = reinterpret_cast<float *>(ws);
+                p.part_ml = reinterpret_cast<float *>(ws + o_bytes);
+            } else {
+                p.nsplit = 1;  // no workspace: run unsplit
+            }
+        }
+        e = pf::launch_fwd(maps, p, head_dim, stream);
+    } else {
+        e = pf::launch_fwd_v0(maps, p, head_dim, stream);
+    }
     return e == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 

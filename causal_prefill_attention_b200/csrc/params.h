@@ -25,6 +25,13 @@ struct FwdParams {
     int max_q;                    // bound on every sequence (chunk) length
     float scale_log2;             // scale * log2(e)
     int test_stall;               // test hook: withhold one Q tile (see prefill_test_inject_stall)
+    int max_ctx;                  // bound on every context length (chunked prefill; 0 otherwise)
+    // split-KV: kv ranges split into up to nsplit parts; the partial results go to
+    // part_o [nsplit][total][n_head][D] (fp32, unnormalised) and part_ml
+    // [nsplit][total][n_head][2] (running max in log2 units, exp-sum)
+    int nsplit;
+    float *part_o;
+    float *part_ml;
 };
 
 struct TensorMaps {
@@ -38,6 +45,9 @@ struct TensorMaps {
 // Pipelined warp-specialised kernel (prefill_fwd.cu) and the sizes it takes.
 int launch_fwd(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
 bool fwd_pipelined_supported(const FwdParams &p, int head_dim);
+// Split count for the pipelined kernel (1 = no split) and its workspace bytes.
+int fwd_choose_splits(const FwdParams &p);
+size_t fwd_split_workspace_bytes(const FwdParams &p, int head_dim);
 // One-CTA-per-query-block kernel (prefill_fwd_v0.cu): no size limits.
 int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
 

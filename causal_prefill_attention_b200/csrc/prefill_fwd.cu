@@ -114,10 +114,9 @@ __device__ __forceinline__ float rowmax128(const float (&x)[BN]) {
 // and O rescaled.  Blocks whose max stays below that bound give P up to 2^8,
 // which the final O / l divides out exactly (same max for P and l).
 template <int D, bool kFull>
-__device__ __forceinline__ void softmax_block(const float (&x)[BN], int j, float sl2, float thr, float &m_run,
+__device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, float sl2, float thr, float &m_run,
                                               float &l_run, uint32_t tS, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
                                               int lane) {
-    const bool first = j == 0;
     float mt = first ? rowmax128(x) : 0.f;
     float m_ref = first ? mt : m_run;
     if (m_ref == -CUDART_INF_F) m_ref = 0.f;  // nothing visible yet (cannot happen under causal masking)
@@ -172,9 +171,23 @@ struct Item {
     int i, h, g, qb0, c0, n, ctx;
     int nk0, nk1;  // kv blocks visited by query block 0 / 1
     int two;       // second query block present
+    // split of the kv range (split-KV): this item covers kv blocks [j_lo, j_hi)
+    int split, nsp, j_lo, j_hi;
+    bool skip;     // a split index beyond this pair's useful split count: no work
     __device__ __forceinline__ int nk(int s) const { return s ? nk1 : nk0; }
     __device__ __forceinline__ int nmax() const { return nk0 > nk1 ? nk0 : nk1; }
+    // end of query block s's blocks inside this split
+    __device__ __forceinline__ int end(int s) const { return nk(s) < j_hi ? nk(s) : j_hi; }
 };
+
+// Useful number of splits of a pair whose kv range has nmax blocks: at most
+// nsplit, and every split keeps at least kMinSplitBlocks blocks (so query block
+// 0, which ends one block before query block 1, always has work in every split).
+constexpr int kMinSplitBlocks = 4;
+__host__ __device__ __forceinline__ int useful_splits(int nmax, int nsplit) {
+    const int m = nmax / kMinSplitBlocks;
+    return nsplit < m ? nsplit : (m > 1 ? m : 1);
+}
 
 __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
     const int c0 = p.cu_seqlens[i], c1 = p.cu_seqlens[i + 1];
@@ -199,7 +212,9 @@ __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
 //   B[c]     items of sequences with more than c pairs (= first item of bucket c)
 //   perm     sequence indices sorted by pair count, descending, stable
 __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, const int *start, const uint16_t *perm,
-                                            int P, int u) {
+                                            int P, int u_split) {
+    const int u = u_split / p.nsplit;
+    const int split = u_split - u * p.nsplit;
     int lo = 1, hi = P;  // smallest c in [1, P] with B[c] <= u
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
@@ -222,6 +237,12 @@ __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, co
     it.two = (it.qb0 + 1) * BM < it.n;
     it.nk0 = num_kv_blocks(it.qb0, it.ctx, it.n, BM, BN);
     it.nk1 = it.two ? num_kv_blocks(it.qb0 + 1, it.ctx, it.n, BM, BN) : 0;
+    const int nmax = it.nmax();
+    it.nsp = useful_splits(nmax, p.nsplit);
+    it.split = split;
+    it.skip = split >= it.nsp;
+    it.j_lo = (split * nmax) / it.nsp;
+    it.j_hi = ((split + 1) * nmax) / it.nsp;
     return it;
 }
 
@@ -346,7 +367,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const int total = B[0];
+    const int total = B[0] * p.nsplit;
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gbase + L::TMEM_SLOT);
     const int G = gridDim.x, cta = blockIdx.x;
 
@@ -368,11 +389,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int u = zigzag(k, cta, G);
             if (u >= total) break;
             const Item it = decode_item(p, B, start, perm, P, u);
-            if (s == 1 && !it.two) continue;
+            if (it.skip || (s == 1 && !it.two)) continue;
             const int qb = it.qb0 + s;
-            const int nk = it.nk(s);
+            const int je = it.end(s);
             float m_run = -CUDART_INF_F, l_run = 0.f;
-            for (int j = 0; j < nk; ++j) {
+            for (int j = it.j_lo; j < je; ++j) {
                 if (!wait_bar(b_sfull, ph_s, abort)) { ok = false; break; }
                 ph_s ^= 1;
                 tc_fence_after();
@@ -390,8 +411,9 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int c = 0; c < BN; ++c)
                         if (c >= lim) x[c] = -CUDART_INF_F;
                 }
-                if (kb.full) softmax_block<D, true>(x, j, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
-                else softmax_block<D, false>(x, j, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
+                const bool first = j == it.j_lo;
+                if (kb.full) softmax_block<D, true>(x, first, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
+                else softmax_block<D, false>(x, first, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
             }
             if (!ok) break;
             // final O / l -> bf16 rows of out
@@ -399,6 +421,24 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ph_o ^= 1;
             tc_fence_after();
             const int a = qb * BM + row;
+            if (it.nsp > 1) {
+                // split-KV: unnormalised O, the running max (log2 units) and the
+                // exp-sum go to the workspace; the combine kernel merges the splits
+                const size_t prow = ((size_t)it.split * p.total + (it.c0 + a)) * p.n_head + it.h;
+                float *po = p.part_o + prow * D;
+                uint32_t r[32];
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    tmem_ld32(tO + cc * 32, r);
+                    if (a < it.n) {
+                        uint4 *d4 = reinterpret_cast<uint4 *>(po + cc * 32);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            d4[c] = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+                    }
+                }
+                if (a < it.n) *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_run * sl2, l_run);
+            } else {
             const float inv_l = 1.f / l_run;
             uint16_t *dst = p.out + ((size_t)(it.c0 + a) * p.n_head + it.h) * D;
             {
@@ -417,6 +457,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
                     }
                 }
+            }
             }
             tc_fence_before();
             __syncwarp();
@@ -438,6 +479,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
                 const Item it = decode_item(p, B, start, perm, P, u);
+                if (it.skip) continue;
                 const int ns = it.two ? 2 : 1;
                 for (int s = 0; s < ns; ++s) {
                     if (!wait_bar(bar(L::B_QEMPTY + s), ((ph_qe >> s) & 1u) ^ 1u, abort)) { ok = false; break; }
@@ -455,8 +497,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tma_load_4d(base + (s ? L::Q1 : L::Q0), &tm_q, b, 0, it.h, it.c0 + (it.qb0 + s) * BM, 0);
                     }
                 }
-                const int nmax = it.nmax();
-                for (int j = 0; j < nmax && ok; ++j) {
+                for (int j = it.j_lo; j < it.j_hi && ok; ++j) {
                     const KvBlock kb = kv_block(it.qb0, j, it.ctx, it.n, BM, BN);
                     for (int t = 0; t < 2; ++t) {  // t = 0: K, t = 1: V
                         if (!wait_bar(bar(L::B_KVEMPTY + stage), phase ^ 1, abort)) { ok = false; break; }
@@ -560,8 +601,9 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
                 const Item it = decode_item(p, B, start, perm, P, u);
+                if (it.skip) continue;
                 const int ns = it.two ? 2 : 1;
-                const int nmax = it.nmax();
+                const int j0 = it.j_lo, jend = it.j_hi;
                 for (int s = 0; s < ns && ok; ++s) {
                     ok = wait_all(bar(L::B_QFULL + s), (ph_qf >> s) & 1u);
                     ph_qf ^= 1u << s;
@@ -578,13 +620,13 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tc_commit_elect(bar(L::B_SFULL + s));
                 }
                 tc_commit_elect(bar(L::B_KVEMPTY + kst));
-                for (int j = 0; j < nmax && ok; ++j) {
+                for (int j = j0; j < jend && ok; ++j) {
                     const int vst = stage;
                     const uint32_t vph = phase;
                     if (++stage == NST) { stage = 0; phase ^= 1; }
                     int nst = -1;
                     uint32_t nph = 0;
-                    if (j + 1 < nmax) {
+                    if (j + 1 < jend) {
                         nst = stage;
                         nph = phase;
                         if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -592,19 +634,19 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (!wait_all(bar(L::B_KVFULL + vst), vph)) { ok = false; break; }
                     bool next_ready = false;
                     for (int s = 0; s < ns; ++s) {
-                        if (j >= it.nk(s)) continue;
+                        if (j >= it.end(s)) continue;
                         if (!wait_all(bar(L::B_PA + s), (ph_pf >> s) & 1u)) { ok = false; break; }
-                        if (j == 0 && ((used >> s) & 1u)) {
+                        if (j == j0 && ((used >> s) & 1u)) {
                             if (!wait_all(bar(L::B_OEMPTY + s), (ph_oe >> s) & 1u)) { ok = false; break; }
                             ph_oe ^= 1u << s;
                         }
                         tc_fence_after();
-                        issue_pv(s, vst, j > 0, 0);
+                        issue_pv(s, vst, j > j0, 0);
                         if (!wait_all(bar(L::B_PB + s), (ph_pf >> s) & 1u)) { ok = false; break; }
                         ph_pf ^= 1u << s;
                         tc_fence_after();
-                        issue_pv(s, vst, j > 0, BN / 32);
-                        if (j + 1 < it.nk(s)) {
+                        issue_pv(s, vst, j > j0, BN / 32);
+                        if (j + 1 < it.end(s)) {
                             if (!next_ready) {
                                 if (!wait_all(bar(L::B_KVFULL + nst), nph)) { ok = false; break; }
                                 tc_fence_after();
@@ -645,10 +687,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
                 const Item it = decode_item(p, B, start, perm, P, u);
-                const int nmax = it.nmax();
+                if (it.skip) continue;
                 const int np = cdiv(it.ctx, BN);
                 const bool writes = (it.h % p.group) == 0;
-                for (int j = 0; j < nmax && ok; ++j) {
+                for (int j = it.j_lo; j < it.j_hi && ok; ++j) {
                     const int jc = j - np;  // chunk block index (negative: prefix)
                     const bool own = writes && (jc == it.qb0 || (it.two && jc == it.qb0 + 1));
                     for (int t = 0; t < 2; ++t) {
@@ -711,6 +753,66 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp == WARP_MMA) tmem_dealloc(tmem, 512);
 }
 
+// Split-KV combine: one warp per (row, query head) merges the split partials,
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s
+// (the same merge rule the online softmax applies between kv blocks).
+template <int D>
+__global__ void __launch_bounds__(256) combine_splits_kernel(const FwdParams p) {
+    constexpr int E = D / 32;  // elements per lane
+    const long long wid = ((long long)blockIdx.x * 256 + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= (long long)p.total * p.n_head) return;
+    const int t = (int)(wid / p.n_head), h = (int)(wid % p.n_head);
+    int lo = 0, hi = p.num_seqs - 1;  // last sequence starting at or before row t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cu_seqlens[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    bool bad = false;
+    if (seq_pairs(p, lo, &bad) == 0) return;
+    const int c0 = p.cu_seqlens[lo], n = p.cu_seqlens[lo + 1] - c0;
+    const int a = t - c0;
+    if (a < 0 || a >= n) return;
+    const int ctx = p.context_lens ? p.context_lens[lo] : 0;
+    const int qb0 = (a / (2 * BM)) * 2;
+    const bool two = (qb0 + 1) * BM < n;
+    const int nmax = two ? num_kv_blocks(qb0 + 1, ctx, n, BM, BN) : num_kv_blocks(qb0, ctx, n, BM, BN);
+    const int nsp = useful_splits(nmax, p.nsplit);
+    if (nsp <= 1) return;  // this pair was not split: the attention kernel wrote the row
+    float m[8], l[8], M = -CUDART_INF_F;
+    for (int sp = 0; sp < nsp; ++sp) {
+        const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (((size_t)sp * p.total + t) * p.n_head + h) * 2);
+        m[sp] = ml.x;
+        l[sp] = ml.y;
+        M = fmaxf(M, ml.x);
+    }
+    float L = 0.f, acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int sp = 0; sp < nsp; ++sp) {
+        const float wgt = ex2(m[sp] - M);
+        L += wgt * l[sp];
+        const float *po = p.part_o + (((size_t)sp * p.total + t) * p.n_head + h) * D + lane * E;
+        float v[E];
+        if constexpr (E == 4) {
+            const float4 f = *reinterpret_cast<const float4 *>(po);
+            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+        } else {
+            const float2 f = *reinterpret_cast<const float2 *>(po);
+            v[0] = f.x; v[1] = f.y;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, v[e], acc[e]);
+    }
+    const float inv = 1.f / L;
+    uint16_t *dst = p.out + ((size_t)t * p.n_head + h) * D + lane * E;
+    if constexpr (E == 4) {
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    } else {
+        *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
+}
+
 template <int D>
 size_t smem_bytes(int P, int num_seqs) {
     return Lay<D>::SCHED + (size_t)(P + 1) * 12 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
@@ -734,8 +836,13 @@ int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
     cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     const long long items_bound = (long long)p.num_seqs * p.n_head * P;
-    const int grid = (int)(items_bound < sm_count() ? items_bound : sm_count());
-    prefill_fwd_kernel<D><<<grid, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache, p, P);
+    const long long items = items_bound * (p.nsplit > 0 ? p.nsplit : 1);
+    const int grid_s = (int)(items < sm_count() ? items : sm_count());
+    prefill_fwd_kernel<D><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache, p, P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
+    const long long warps = (long long)p.total * p.n_head;
+    combine_splits_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, (cudaStream_t)stream>>>(p);
     return (int)cudaGetLastError();
 }
 
@@ -747,6 +854,32 @@ bool fwd_pipelined_supported(const FwdParams &p, int head_dim) {
     if (P > 2048 || p.num_seqs > 4096) return false;
     const size_t smem = head_dim == 64 ? smem_bytes<64>(P, p.num_seqs) : smem_bytes<128>(P, p.num_seqs);
     return smem <= 227 * 1024;
+}
+
+int fwd_choose_splits(const FwdParams &p) {
+    // Split only when the call has fewer work items than SMs: pick the split
+    // count (up to 8) that minimises waves / splits, keeping >= kMinSplitBlocks
+    // blocks per split of the longest kv range.
+    const long long items = (long long)p.num_seqs * p.n_head * cdiv(p.max_q, 2 * BM);
+    const int sms = sm_count();
+    if (items <= 0 || items >= sms) return 1;
+    const int nk = cdiv(p.max_ctx, BN) + cdiv(p.max_q, BN);
+    int best = 1;
+    double best_cost = 1.0;  // waves per split at 1 split
+    for (int sp = 2; sp <= 8; ++sp) {
+        if (nk / sp < kMinSplitBlocks) break;
+        const double cost = (double)((items * sp + sms - 1) / sms) / sp;
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return best;
+}
+
+size_t fwd_split_workspace_bytes(const FwdParams &p, int head_dim) {
+    if (p.nsplit <= 1) return 0;
+    return (size_t)p.nsplit * p.total * p.n_head * ((size_t)head_dim + 2) * sizeof(float);
 }
 
 int launch_fwd(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream) {

@@ -37,11 +37,20 @@
  *                cu_seqlens[i] .. cu_seqlens[i+1]-1 (non-decreasing, cu_seqlens[0] = 0).
  *
  * Ownership: every pointer argument is caller-owned DEVICE memory, except where
- * stated.  The library allocates no device memory per call, keeps nothing after
- * return, and enqueues its work asynchronously on `stream` (the legacy default
- * stream if NULL).  It writes `out`, the cache slots of the tokens it processes,
- * and `*status_dev`; nothing else.  Inputs must stay valid until the work on
- * `stream` completes.
+ * stated.  Calls enqueue their work asynchronously on `stream` (the legacy
+ * default stream if NULL).  They write `out`, the cache slots of the tokens they
+ * process, and `*status_dev`; nothing else of the caller's.  Inputs must stay
+ * valid until the work on `stream` completes.
+ *
+ * Split-KV workspace: when a call has fewer work items than the GPU has SMs
+ * (typically a chunked-prefill chunk attending to a long cached prefix), the
+ * kv range of each item is split across CTAs and the partial results are
+ * merged by a second kernel on the same stream.  The partials live in a device
+ * workspace that the library allocates (cudaMalloc) on the first such call for
+ * a given (device, stream) and keeps for later calls, growing it when a larger
+ * call needs more; calls that do not split allocate nothing.  Size:
+ * splits x total rows x n_head x (head_dim + 2) x 4 bytes, splits <= 8.  If the
+ * allocation fails the call runs unsplit.
  *
  * Errors: argument problems that the host can see are returned synchronously
  * and nothing is launched.  Problems only the device can see (a block-table

@@ -178,3 +178,41 @@ def test_named_chunked_full_size():
                                          context_lens=[ctx], kv_cache=pre, block_table=w.block_table,
                                          block_size=16)
     U.compare_out(out[rows, heads], ref, "chunked full")
+
+
+# ------------------------------------------------------------ split-KV (few work items, long prefix)
+def _chunked_call(ctxs, lens, H, G, d, bs, seed):
+    full = W.make_workload([c + L for c, L in zip(ctxs, lens)], H, G, d, block_size=bs, seed=seed, extra_pages=2)
+    cache = full.empty_cache()
+    starts = full.cu_seqlens.tolist()
+    pre_k = torch.cat([full.k[s:s + c] for s, c in zip(starts, ctxs)])
+    pre_v = torch.cat([full.v[s:s + c] for s, c in zip(starts, ctxs)])
+    pre_cu = torch.tensor(np.concatenate([[0], np.cumsum(ctxs)]), dtype=torch.int32)
+    cache = oracle.kv_write(pre_k, pre_v, pre_cu, cache, full.block_table, bs)
+    sel = torch.cat([torch.arange(s + c, s + c + L) for s, c, L in zip(starts, ctxs, lens)])
+    q, k, v = full.q[sel].contiguous(), full.k[sel].contiguous(), full.v[sel].contiguous()
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    ctx = torch.tensor(ctxs, dtype=torch.int32)
+    ref_out = oracle.attention(q, k, v, cu, H, G, d, full.scale, context_lens=ctx, kv_cache=cache,
+                               block_table=full.block_table, block_size=bs)
+    ref_cache = oracle.kv_write(k, v, cu, cache, full.block_table, bs, context_lens=ctx)
+    cache_d = cache.cuda()
+    out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _lib.prefill_attn_chunked(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), ctx.cuda(), max(lens), max(ctxs), full.scale,
+                              out, cache_d, full.block_table.cuda(), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    U.assert_cache_bits_equal(cache_d.cpu(), ref_cache, "split-kv cache")
+    return U.compare_out(out.cpu(), ref_out, f"split-kv ctx={ctxs} lens={lens} d={d}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_split_kv_long_prefix(d):
+    """4 work items against a ~3k prefix: the kv range is split and merged."""
+    _chunked_call([3000], [300], 8, 2, d, 16, seed=71)
+
+
+def test_split_kv_mixed_batch():
+    """Pairs with long ranges split, short ones do not; both paths in one call."""
+    _chunked_call([2000, 50, 1500, 0], [200, 30, 129, 5], 4, 1, 128, 32, seed=72)
