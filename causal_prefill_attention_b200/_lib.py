@@ -17,9 +17,11 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libprefill.
 STATUS_NAMES = {
     0: "PREFILL_OK", 1: "PREFILL_ERR_NULL", 2: "PREFILL_ERR_SHAPE", 3: "PREFILL_ERR_UNSUPPORTED",
     4: "PREFILL_ERR_BLOCK_TABLE", 5: "PREFILL_ERR_CUDA", 6: "PREFILL_ERR_TIMEOUT", 7: "PREFILL_ERR_ALIGNMENT",
+    8: "PREFILL_ERR_SCRATCH_LIMIT",
 }
 EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
-            "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall")
+            "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall",
+            "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes")
 
 _lib = None
 
@@ -50,6 +52,10 @@ def load() -> ctypes.CDLL:
         lib.prefill_kv_block_rule.restype = I
         lib.prefill_test_inject_stall.argtypes = [I]
         lib.prefill_test_inject_stall.restype = None
+        lib.prefill_attn_chunked_noalloc.argtypes = lib.prefill_attn_chunked.argtypes
+        lib.prefill_attn_chunked_noalloc.restype = I
+        lib.prefill_noalloc_scratch_bytes.argtypes = []
+        lib.prefill_noalloc_scratch_bytes.restype = ctypes.c_size_t
         _lib = lib
     return _lib
 
@@ -120,6 +126,29 @@ def prefill_attn_chunked(q, k, v, cu_seqlens_q, context_lens, max_q_len: int, ma
         _ptr(status), _stream_ptr(stream))
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "prefill_attn_chunked")
+    return rc
+
+
+def prefill_attn_chunked_noalloc(q, k, v, cu_seqlens_q, context_lens, max_q_len: int, max_context_len: int,
+                                 scale: float, out, kv_cache, block_table, status: Optional[torch.Tensor] = None,
+                                 stream=None, raise_on_error: bool = True) -> int:
+    """``prefill_attn_chunked`` for callers that cannot allocate device memory
+    (C ABI ``prefill_attn_chunked_noalloc``): split-KV partials go to a fixed
+    32 MiB device array inside the library instead of a cudaMalloc'd workspace."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3)
+    _check_bf16("out", out, 3), _check_bf16("kv_cache", kv_cache, 5)
+    _check_i32("cu_seqlens_q", cu_seqlens_q), _check_i32("context_lens", context_lens)
+    _check_i32("block_table", block_table)
+    T, H, D = q.shape
+    G = k.shape[1]
+    rc = load().prefill_attn_chunked_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(cu_seqlens_q), _ptr(context_lens), cu_seqlens_q.numel() - 1,
+        int(max_q_len), int(max_context_len), H, G, D, float(scale), _ptr(out), _ptr(kv_cache),
+        kv_cache.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "prefill_attn_chunked_noalloc")
     return rc
 
 

@@ -94,10 +94,15 @@ void *split_workspace(size_t bytes, void *stream) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total, const int32_t *cu,
-        const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
-        int n_kv_head, int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *cache, int num_blocks,
-        const int32_t *bt, int mbps, int bs, int32_t *status, prefill_stream_t stream) {
+}  // namespace
+
+namespace pf {
+
+int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total, const int32_t *cu,
+                const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
+                int n_kv_head, int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *cache, int num_blocks,
+                const int32_t *bt, int mbps, int bs, int32_t *status, prefill_stream_t stream, void *scratch,
+                size_t scratch_bytes) {
     if (!q || !k || !v || !cu || !out || !cache || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
     if (total < 0 || num_seqs < 0 || max_q < 0 || max_ctx < 0) return PREFILL_ERR_SHAPE;
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
@@ -169,7 +174,9 @@ int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int
         p.nsplit = pf::fwd_choose_splits(p);
         if (p.nsplit > 1) {
             const size_t o_bytes = (size_t)p.nsplit * p.total * p.n_head * head_dim * sizeof(float);
-            char *ws = static_cast<char *>(split_workspace(pf::fwd_split_workspace_bytes(p, head_dim), stream));
+            const size_t need = pf::fwd_split_workspace_bytes(p, head_dim);
+            if (scratch && need > scratch_bytes) return PREFILL_ERR_SCRATCH_LIMIT;  // caller-supplied scratch too small
+            char *ws = static_cast<char *>(scratch ? scratch : split_workspace(need, stream));
             if (ws) {
                 p.part_o = reinterpret_cast<float *>(ws);
                 p.part_ml = reinterpret_cast<float *>(ws + o_bytes);
@@ -184,7 +191,7 @@ int run(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int
     return e == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 
-}  // namespace
+}  // namespace pf
 
 extern "C" {
 
@@ -193,9 +200,9 @@ int prefill_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf1
                  float scale, prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks,
                  const int32_t *block_table, int max_blocks_per_seq, int block_size, int32_t *status_dev,
                  prefill_stream_t stream) {
-    return run(q, k, v, total_tokens, cu_seqlens, nullptr, false, num_seqs, max_seqlen, 0, n_head, n_kv_head,
-               head_dim, scale, out, kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
-               status_dev, stream);
+    return pf::run_prefill(q, k, v, total_tokens, cu_seqlens, nullptr, false, num_seqs, max_seqlen, 0, n_head,
+                           n_kv_head, head_dim, scale, out, kv_cache, num_blocks, block_table, max_blocks_per_seq,
+                           block_size, status_dev, stream, nullptr, 0);
 }
 
 int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,
@@ -203,9 +210,9 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
                          int max_context_len, int n_head, int n_kv_head, int head_dim, float scale,
                          prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks, const int32_t *block_table,
                          int max_blocks_per_seq, int block_size, int32_t *status_dev, prefill_stream_t stream) {
-    return run(q, k, v, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len, n_head,
-               n_kv_head, head_dim, scale, out, kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
-               status_dev, stream);
+    return pf::run_prefill(q, k, v, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len,
+                           n_head, n_kv_head, head_dim, scale, out, kv_cache, num_blocks, block_table,
+                           max_blocks_per_seq, block_size, status_dev, stream, nullptr, 0);
 }
 
 void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }
@@ -220,6 +227,8 @@ const char *prefill_status_string(int s) {
         case PREFILL_ERR_CUDA: return "CUDA launch or driver failure";
         case PREFILL_ERR_TIMEOUT: return "device pipeline wait exceeded its limit";
         case PREFILL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case PREFILL_ERR_SCRATCH_LIMIT:
+            return "the call would need more split-KV scratch than the no-allocation entry point's static buffer holds";
         default: return "unknown status";
     }
 }

@@ -51,4 +51,13 @@ size_t fwd_split_workspace_bytes(const FwdParams &p, int head_dim);
 // One-CTA-per-query-block kernel (prefill_fwd_v0.cu): no size limits.
 int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
 
+// Host path shared by the C entry points (api.cu).  scratch / scratch_bytes:
+// caller-supplied split-KV scratch (nullptr: the library's own workspace);
+// a split that needs more than scratch_bytes returns PREFILL_ERR_SCRATCH_LIMIT.
+int run_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int total, const int32_t *cu,
+                const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
+                int n_kv_head, int head_dim, float scale, uint16_t *out, uint16_t *cache, int num_blocks,
+                const int32_t *bt, int mbps, int bs, int32_t *status, struct CUstream_st *stream, void *scratch,
+                size_t scratch_bytes);
+
 }  // namespace pf

@@ -67,6 +67,7 @@
 #ifndef LIBPREFILL_PREFILL_H
 #define LIBPREFILL_PREFILL_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -86,7 +87,8 @@ typedef enum {
     PREFILL_ERR_BLOCK_TABLE = 4,  /* block-table entry outside [0, num_blocks) or table too short */
     PREFILL_ERR_CUDA = 5,         /* launch or driver failure */
     PREFILL_ERR_TIMEOUT = 6,      /* a device-side pipeline wait exceeded its iteration limit */
-    PREFILL_ERR_ALIGNMENT = 7     /* a pointer is not 16-byte aligned */
+    PREFILL_ERR_ALIGNMENT = 7,    /* a pointer is not 16-byte aligned */
+    PREFILL_ERR_SCRATCH_LIMIT = 8 /* prefill_attn_chunked_noalloc: the split partials exceed its static buffer */
 } prefill_status;
 
 /*
@@ -147,6 +149,46 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
                          prefill_bf16 *kv_cache, int num_blocks,
                          const int32_t *block_table, int max_blocks_per_seq, int block_size,
                          int32_t *status_dev, prefill_stream_t stream);
+
+/*
+ * prefill_attn_chunked_noalloc -- prefill_attn_chunked for callers that cannot
+ * allocate device memory.  The pages have no counterpart: this is a deployment
+ * variant of the chunked call, not a step of the method.
+ *
+ * prefill_attn_chunked may split long kv ranges (split-KV) and then obtains a
+ * workspace with cudaMalloc.  Callers that cannot allow that -- code recorded
+ * into a CUDA graph by stream capture (cudaMalloc cannot be captured), serving
+ * engines that own all device memory through their own pool, processes whose
+ * device-memory budget is fixed at start-up -- use this entry point instead.
+ * It computes the same result with the same kernels, keeping the split
+ * partials in a fixed device array that is part of the library: 32 MiB
+ * (prefill_noalloc_scratch_bytes()) on every GPU that loads the library, held
+ * until the process exits.  It calls no cudaMalloc, cudaFree or allocating
+ * library routine.
+ *
+ *   Arguments, layouts and errors as for prefill_attn_chunked, plus:
+ *   PREFILL_ERR_SCRATCH_LIMIT  returned (before any launch) when the call would
+ *     split and its partials -- splits x total_q x n_head x (head_dim + 2) x 4
+ *     bytes -- do not fit the array.  Calls that do not split always fit.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  Every call uses the same array, which keeps the last call's
+ * contents (nothing in it needs to start at zero).  Calls whose GPU work
+ * overlaps -- on different streams, or unordered from different threads --
+ * race on the array: the caller must serialise them.
+ */
+int prefill_attn_chunked_noalloc(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                                 int total_q, const int32_t *cu_seqlens_q, const int32_t *context_lens,
+                                 int num_seqs, int max_q_len, int max_context_len,
+                                 int n_head, int n_kv_head, int head_dim, float scale,
+                                 prefill_bf16 *out,
+                                 prefill_bf16 *kv_cache, int num_blocks,
+                                 const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                                 int32_t *status_dev, prefill_stream_t stream);
+
+/* Size in bytes of prefill_attn_chunked_noalloc's fixed split-KV array. */
+size_t prefill_noalloc_scratch_bytes(void);
 
 /*
  * Test hook for the failure path (no counterpart on the pages).  With enable

@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for s in range(8):
+    for s in range(9):
         assert _lib.status_string(s)
     assert _lib.status_string(99) == "unknown status"
 
