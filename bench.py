@@ -187,6 +187,21 @@ def time_steps(runner, steps, warmup, stream, flush):
     return [a.elapsed_time(b) for a, b in durs]
 
 
+def aggregate(total_ms: float, steps: int, flops: float, tokens: int, world: int, dist=None, device="cuda"):
+    """Whole-job numbers from each rank's device-timed total: the slowest rank's
+    time (max over ranks) sets the step time; every rank runs the same work
+    (replicas), so the job's throughput is world x one replica's work / time.
+    Returns (ms per step, TFLOP/s of one replica, job TFLOP/s, job tokens/s)."""
+    if dist is not None and world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms = total_ms / steps
+    tflops = flops / (ms * 1e-3) / 1e12
+    return ms, tflops, tflops * world, tokens / (ms * 1e-3) * world
+
+
 def e2e_run(w: W.Workload, steps, warmup, stream):
     """Same metric through the C ABI with pinned host buffers: H2D of the step's
     inputs and D2H of its output inside the timed region."""
@@ -303,16 +318,7 @@ def main():
     with ClockSampler(local) as clk:
         durs = time_steps(runner, args.steps, args.warmup, stream, flush)
     torch.cuda.synchronize()
-    total_ms = sum(durs)
-    if dist:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        dist.barrier()
-    ms = total_ms / args.steps
-    tflops = runner.flops / (ms * 1e-3) / 1e12
-    value = tflops * world  # replicas: every rank runs the same work
-    tokens_s = runner.tokens / (ms * 1e-3) * world
+    ms, tflops, value, tokens_s = aggregate(sum(durs), args.steps, runner.flops, runner.tokens, world, dist, "cuda")
 
     e2e_ms, h2d, d2h = e2e_run(w, max(3, args.steps // 2), 3, stream)
     e2e_tflops = runner.flops / (e2e_ms * 1e-3) / 1e12 * world

@@ -258,9 +258,9 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 // Register split (the launch gives 384 threads x 168 = 64,512 registers):
-// softmax warpgroups 2 x 128 x 200 + control warpgroup 128 x 104 = 64,512.
-__device__ __forceinline__ void setmaxnreg_softmax() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;"); }
-__device__ __forceinline__ void setmaxnreg_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;"); }
+// softmax warpgroups 2 x 128 x 208 + control warpgroup 128 x 88 = 64,512.
+__device__ __forceinline__ void setmaxnreg_softmax() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
+__device__ __forceinline__ void setmaxnreg_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
 
 // ------------------------------------------------------------------ kernel
 template <int D>
@@ -541,19 +541,19 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 fence_proxy_async_smem();
                                 __syncwarp();
                             }
-                            if (lane == 0) {
-                                mbar_expect_tx(b, (uint32_t)(full_pages * bs * 128 * L::NCH));
-                                for (int pg = 0; pg < full_pages; ++pg) {
-                                    int page = p.block_table[(size_t)it.i * p.mbps + kb.key_begin / bs + pg];
-                                    if (page < 0 || page >= p.num_blocks) {
-                                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
-                                        page = p.num_blocks;  // outside the map: zero fill
-                                    }
-#pragma unroll
-                                    for (int ch = 0; ch < L::NCH; ++ch)
-                                        tma_load_4d(dst + ch * CHUNK + pg * bs * 128, &tm_cache, b, ch * 64, it.g, 0,
-                                                    page * 2 + t);
+                            // one (page, 64-column chunk) box per lane: a single thread pays
+                            // ~300 clocks per TMA issue, lanes issuing together overlap it
+                            if (lane == 0) mbar_expect_tx(b, (uint32_t)(full_pages * bs * 128 * L::NCH));
+                            __syncwarp();
+                            for (int x = lane; x < full_pages * L::NCH; x += 32) {
+                                const int pg = x / L::NCH, ch = x % L::NCH;
+                                int page = p.block_table[(size_t)it.i * p.mbps + kb.key_begin / bs + pg];
+                                if (page < 0 || page >= p.num_blocks) {
+                                    report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                                    page = p.num_blocks;  // outside the map: zero fill
                                 }
+                                tma_load_4d(dst + ch * CHUNK + pg * bs * 128, &tm_cache, b, ch * 64, it.g, 0,
+                                            page * 2 + t);
                             }
                         }
                         if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -702,20 +702,18 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             const int P0 = it.ctx + a0;                  // absolute position of row 0
                             const bool aligned = (P0 % bs) == 0;
                             const int tma_rows = aligned ? (rows / bs) * bs : 0;
-                            if (lane == 0 && tma_rows > 0) {
-                                for (int r = 0; r < tma_rows; r += bs) {
-                                    const int page = p.block_table[(size_t)it.i * p.mbps + (P0 + r) / bs];
-                                    if (page < 0 || page >= p.num_blocks) {
-                                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
-                                        continue;
-                                    }
-#pragma unroll
-                                    for (int ch = 0; ch < L::NCH; ++ch)
-                                        tma_store_4d(&tm_cache, src + ch * CHUNK + r * 128, ch * 64, it.g, 0,
-                                                     page * 2 + t);
+                            // one (page, chunk) store per lane, issued together
+                            const int nst = (tma_rows / bs) * L::NCH;
+                            for (int x = lane; x < nst; x += 32) {
+                                const int r = (x / L::NCH) * bs, ch = x % L::NCH;
+                                const int page = p.block_table[(size_t)it.i * p.mbps + (P0 + r) / bs];
+                                if (page < 0 || page >= p.num_blocks) {
+                                    report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                                    continue;
                                 }
-                                bulk_commit();
+                                tma_store_4d(&tm_cache, src + ch * CHUNK + r * 128, ch * 64, it.g, 0, page * 2 + t);
                             }
+                            if (lane < nst) bulk_commit();
                             // remaining rows one 16-byte unit per lane step
                             const int units = (rows - tma_rows) * 8 * L::NCH;
                             for (int x = lane; x < units; x += 32) {
@@ -734,7 +732,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                     ((((size_t)page * 2 + t) * bs + P_ % bs) * G_ + it.g) * D + ch * 64 + un * 8;
                                 *reinterpret_cast<uint4 *>(p.cache + off) = val;
                             }
-                            if (lane == 0 && tma_rows > 0) bulk_wait_read0();
+                            if (lane < nst) bulk_wait_read0();  // each issuing lane waits for its own stores
                             __syncwarp();
                         }
                         if (lane == 0) mbar_arrive(bar(L::B_KVEMPTY + stage));
@@ -742,7 +740,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                 }
             }
-            if (lane == 0) bulk_wait0();  // stores complete before the kernel ends
+            bulk_wait0();  // every lane's stores complete before the kernel ends
             if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
             __syncwarp();
         }
@@ -753,63 +751,84 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp == WARP_MMA) tmem_dealloc(tmem, 512);
 }
 
-// Split-KV combine: one warp per (row, query head) merges the split partials,
-// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s
-// (the same merge rule the online softmax applies between kv blocks).
+// Split-KV combine: one CTA per packed row t, one warp per query head (heads
+// strided by the warp count); the row's sequence and split count are found
+// once per CTA.  O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with
+// M = max_s m_s -- the merge rule the online softmax applies between blocks.
+constexpr int kCombineWarps = 16;
 template <int D>
-__global__ void __launch_bounds__(256) combine_splits_kernel(const FwdParams p) {
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(const FwdParams p) {
     constexpr int E = D / 32;  // elements per lane
-    const long long wid = ((long long)blockIdx.x * 256 + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (wid >= (long long)p.total * p.n_head) return;
-    const int t = (int)(wid / p.n_head), h = (int)(wid % p.n_head);
-    int lo = 0, hi = p.num_seqs - 1;  // last sequence starting at or before row t
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.cu_seqlens[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    bool bad = false;
-    if (seq_pairs(p, lo, &bad) == 0) return;
-    const int c0 = p.cu_seqlens[lo], n = p.cu_seqlens[lo + 1] - c0;
-    const int a = t - c0;
-    if (a < 0 || a >= n) return;
-    const int ctx = p.context_lens ? p.context_lens[lo] : 0;
-    const int qb0 = (a / (2 * BM)) * 2;
-    const bool two = (qb0 + 1) * BM < n;
-    const int nmax = two ? num_kv_blocks(qb0 + 1, ctx, n, BM, BN) : num_kv_blocks(qb0, ctx, n, BM, BN);
-    const int nsp = useful_splits(nmax, p.nsplit);
-    if (nsp <= 1) return;  // this pair was not split: the attention kernel wrote the row
-    float m[8], l[8], M = -CUDART_INF_F;
-    for (int sp = 0; sp < nsp; ++sp) {
-        const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (((size_t)sp * p.total + t) * p.n_head + h) * 2);
-        m[sp] = ml.x;
-        l[sp] = ml.y;
-        M = fmaxf(M, ml.x);
-    }
-    float L = 0.f, acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int sp = 0; sp < nsp; ++sp) {
-        const float wgt = ex2(m[sp] - M);
-        L += wgt * l[sp];
-        const float *po = p.part_o + (((size_t)sp * p.total + t) * p.n_head + h) * D + lane * E;
-        float v[E];
-        if constexpr (E == 4) {
-            const float4 f = *reinterpret_cast<const float4 *>(po);
-            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-        } else {
-            const float2 f = *reinterpret_cast<const float2 *>(po);
-            v[0] = f.x; v[1] = f.y;
+    __shared__ int s_nsp;
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        int lo = 0, hi = p.num_seqs - 1;  // last sequence starting at or before row t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.cu_seqlens[mid] <= t) lo = mid; else hi = mid - 1;
         }
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, v[e], acc[e]);
+        int nsp = 0;
+        bool bad = false;
+        if (seq_pairs(p, lo, &bad) > 0) {
+            const int c0 = p.cu_seqlens[lo], n = p.cu_seqlens[lo + 1] - c0;
+            const int a = t - c0;
+            if (a >= 0 && a < n) {
+                const int ctx = p.context_lens ? p.context_lens[lo] : 0;
+                const int qb0 = (a / (2 * BM)) * 2;
+                const bool two = (qb0 + 1) * BM < n;
+                const int nmax = two ? num_kv_blocks(qb0 + 1, ctx, n, BM, BN) : num_kv_blocks(qb0, ctx, n, BM, BN);
+                nsp = useful_splits(nmax, p.nsplit);
+            }
+        }
+        s_nsp = nsp;
     }
-    const float inv = 1.f / L;
-    uint16_t *dst = p.out + ((size_t)t * p.n_head + h) * D + lane * E;
-    if constexpr (E == 4) {
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-    } else {
-        *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    __syncthreads();
+    const int nsp = s_nsp;
+    if (nsp <= 1) return;  // row not split (the attention kernel wrote it) or not part of a valid sequence
+    for (int h = warp; h < p.n_head; h += kCombineWarps) {
+        const size_t base_row = (size_t)t * p.n_head + h;
+        const size_t stride_row = (size_t)p.total * p.n_head;
+        float M = -CUDART_INF_F;
+        float m[8], l[8];
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) {
+            if (sp < nsp) {
+                const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (base_row + sp * stride_row) * 2);
+                m[sp] = ml.x;
+                l[sp] = ml.y;
+                M = fmaxf(M, ml.x);
+            }
+        }
+        float L = 0.f, acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) {
+            if (sp < nsp) {
+                const float wgt = ex2(m[sp] - M);
+                L += wgt * l[sp];
+                const float *po = p.part_o + (base_row + sp * stride_row) * D + lane * E;
+                float v[E];
+                if constexpr (E == 4) {
+                    const float4 f = *reinterpret_cast<const float4 *>(po);
+                    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+                } else {
+                    const float2 f = *reinterpret_cast<const float2 *>(po);
+                    v[0] = f.x; v[1] = f.y;
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, v[e], acc[e]);
+            }
+        }
+        const float inv = 1.f / L;
+        uint16_t *dst = p.out + base_row * D + lane * E;
+        if constexpr (E == 4) {
+            *reinterpret_cast<uint2 *>(dst) =
+                make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+        } else {
+            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        }
     }
 }
 
@@ -841,8 +860,7 @@ int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
     prefill_fwd_kernel<D><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache, p, P);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
-    const long long warps = (long long)p.total * p.n_head;
-    combine_splits_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, (cudaStream_t)stream>>>(p);
+    combine_splits_kernel<D><<<(unsigned)p.total, 32 * kCombineWarps, 0, (cudaStream_t)stream>>>(p);
     return (int)cudaGetLastError();
 }
 
