@@ -37,10 +37,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-#ifndef PF_KV_STAGES
-#define PF_KV_STAGES 4
-#endif
-constexpr int NST = PF_KV_STAGES;  // K/V ring stages (each one K or one V tile)
+// K/V ring stages (each holds one K or one V tile): a template parameter of the
+// kernel, 5 when the shared-memory schedule leaves room for it, else 4.
 constexpr int NTHREADS = 384;
 constexpr int WARP_PRODUCER = 8, WARP_MMA = 9, WARP_WRITER = 10;
 constexpr uint32_t CHUNK = 128 * 128;  // 128 rows x 64 bf16, 128B-swizzled
@@ -54,7 +52,7 @@ constexpr float kRescaleLog2 = 8.0f;
 #endif
 constexpr uint32_t kEmuMask = PF_EXP2_EMU_MASK;
 
-template <int D>
+template <int D, int NST>
 struct Lay {
     static constexpr int NCH = D / 64;
     static constexpr uint32_t TILE = NCH * CHUNK;
@@ -263,12 +261,12 @@ __device__ __forceinline__ void setmaxnreg_softmax() { asm volatile("setmaxnreg.
 __device__ __forceinline__ void setmaxnreg_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
 
 // ------------------------------------------------------------------ kernel
-template <int D>
+template <int D, int NST>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_cache,
                    const FwdParams p, const int P) {
-    using L = Lay<D>;
+    using L = Lay<D, NST>;
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
 
@@ -832,10 +830,11 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(cons
     }
 }
 
-template <int D>
+template <int D, int NST>
 size_t smem_bytes(int P, int num_seqs) {
-    return Lay<D>::SCHED + (size_t)(P + 1) * 12 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
+    return Lay<D, NST>::SCHED + (size_t)(P + 1) * 12 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
 }
+constexpr size_t kMaxSmem = 227 * 1024;
 
 int sm_count() {
     static int n = 0;
@@ -848,20 +847,29 @@ int sm_count() {
     return n;
 }
 
-template <int D>
-int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
+template <int D, int NST>
+int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
-    const size_t smem = smem_bytes<D>(P, p.num_seqs);
-    cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = smem_bytes<D, NST>(P, p.num_seqs);
+    cudaError_t e =
+        cudaFuncSetAttribute(prefill_fwd_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     const long long items_bound = (long long)p.num_seqs * p.n_head * P;
     const long long items = items_bound * (p.nsplit > 0 ? p.nsplit : 1);
     const int grid_s = (int)(items < sm_count() ? items : sm_count());
-    prefill_fwd_kernel<D><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache, p, P);
+    prefill_fwd_kernel<D, NST><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache,
+                                                                                  p, P);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
     combine_splits_kernel<D><<<(unsigned)p.total, 32 * kCombineWarps, 0, (cudaStream_t)stream>>>(p);
     return (int)cudaGetLastError();
+}
+
+template <int D>
+int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
+    const int P = cdiv(p.max_q, 2 * BM);
+    if (smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem) return launch_nst<D, 5>(maps, p, stream);
+    return launch_nst<D, 4>(maps, p, stream);
 }
 
 }  // namespace
@@ -870,8 +878,8 @@ int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
 bool fwd_pipelined_supported(const FwdParams &p, int head_dim) {
     const int P = cdiv(p.max_q, 2 * BM);
     if (P > 2048 || p.num_seqs > 4096) return false;
-    const size_t smem = head_dim == 64 ? smem_bytes<64>(P, p.num_seqs) : smem_bytes<128>(P, p.num_seqs);
-    return smem <= 227 * 1024;
+    const size_t smem = head_dim == 64 ? smem_bytes<64, 4>(P, p.num_seqs) : smem_bytes<128, 4>(P, p.num_seqs);
+    return smem <= kMaxSmem;
 }
 
 int fwd_choose_splits(const FwdParams &p) {
