@@ -45,6 +45,8 @@ constexpr uint32_t CHUNK = 128 * 128;  // 128 rows x 64 bf16, 128B-swizzled
 // Threshold (log2 units) before the running max is moved and O rescaled;
 // between moves P can reach 2^8, well inside fp32 / bf16 range.
 constexpr float kRescaleLog2 = 8.0f;
+// P (bf16 pairs) occupies the first 64 columns of its S region.
+constexpr uint32_t kPOff = 0;
 // Which of the 32 column pairs in each 64-column half of an unmasked block take
 // their exponentials on the FMA pipe (exp2_fma2) instead of MUFU (ex2).
 #ifndef PF_EXP2_EMU_MASK
@@ -122,7 +124,7 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
     {
         uint32_t pw[32];
         exp_half<0, kFull>(x, sl2, -m_ref * sl2, pw, sa0, sa1, sb0, sb1);
-        tmem_st32(tS, pw);
+        tmem_st32(tS + kPOff, pw);
     }
     float m_new = m_ref, alpha = first ? 0.f : 1.f;
     if (!first) {
@@ -137,7 +139,7 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
             {
                 uint32_t pw[32];
                 exp_half<0, kFull>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
-                tmem_st32(tS, pw);
+                tmem_st32(tS + kPOff, pw);
             }
 #pragma unroll 1
             for (int cc = 0; cc < D / 16; ++cc) {
@@ -155,7 +157,103 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
     if (lane == 0) mbar_arrive(b_pa);
     uint32_t pw[32];
     exp_half<1, kFull>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
-    tmem_st32(tS + 32, pw);
+    tmem_st32(tS + kPOff + 32, pw);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_pb);
+    l_run = l_run * alpha + ((sa0 + sa1) + (sb0 + sb1));
+    m_run = m_new;
+}
+
+// Exponentials of 64 scores held in y64 (same arithmetic as exp_half),
+// written to TMEM as bf16 pairs at taddr in two 16-column stores so that only
+// 16 packed words are live at a time.
+template <bool kEmu>
+__device__ __forceinline__ void exp64_store(const float (&y64)[64], float sl2, float nms, uint32_t taddr,
+                                            float &sa0, float &sa1, float &sb0, float &sb1) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pw[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+            const int c = hh * 16 + cc;
+            float y0, y1, p0, p1;
+            fma2(y0, y1, y64[2 * c], y64[2 * c + 1], sl2, sl2, nms, nms);
+            if (kEmu && ((kEmuMask >> c) & 1u)) {
+                exp2_fma2(y0, y1, p0, p1);
+            } else {
+                p0 = ex2(y0);
+                p1 = ex2(y1);
+            }
+            if (c & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
+            pw[cc] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(taddr + hh * 16, pw);
+    }
+}
+
+__device__ __forceinline__ float rowmax64x2(const float (&a)[64], const float (&b)[64]) {
+    float a0 = a[0], a1 = a[1], a2 = b[0], a3 = b[1];
+#pragma unroll
+    for (int c = 2; c < 64; c += 2) {
+        a0 = max3(a0, a[c], a[c + 1]);
+        a2 = max3(a2, b[c], b[c + 1]);
+    }
+    return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+}
+
+// Online softmax of a block that is not the first of its range: the running
+// max is already known, so the first 64 scores are exponentiated while the
+// second 64 are still being read from TMEM; the block max is checked once both
+// halves are in (half 0 is redone and O rescaled only if it moved past the
+// threshold).  P goes to TMEM in two halves, announced on b_pa / b_pb.
+template <int D, bool kFull>
+__device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lim, float sl2, float thr, float &m_run,
+                                                     float &l_run, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
+                                                     int lane) {
+    float x0[64], x1[64];
+    {
+        uint32_t r[64];
+        tmem_ld64_nowait(tS, r);
+        tmem_wait_ld_tie64(r);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x0[c] = __uint_as_float(r[c]);
+    }
+    uint32_t r1[64];
+    tmem_ld64_nowait(tS + 64, r1);  // second half in flight during half 0's exponentials
+    if (!kFull) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+            if (c >= lim) x0[c] = -CUDART_INF_F;
+    }
+    float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+    exp64_store<kFull>(x0, sl2, -m_run * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
+    tmem_wait_ld_tie64(r1);
+#pragma unroll
+    for (int c = 0; c < 64; ++c) x1[c] = (kFull || 64 + c < lim) ? __uint_as_float(r1[c]) : -CUDART_INF_F;
+    const float mt = rowmax64x2(x0, x1);
+    const bool need = mt > m_run + thr;
+    float m_new = m_run, alpha = 1.f;
+    if (__any_sync(0xffffffffu, need)) {
+        m_new = need ? mt : m_run;
+        alpha = ex2((m_run - m_new) * sl2);
+        sa0 = sa1 = sb0 = sb1 = 0.f;
+        exp64_store<kFull>(x0, sl2, -m_new * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t r[16];
+            tmem_ld16(tO + cc * 16, r);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+            tmem_st16(tO + cc * 16, r);
+        }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_pa);
+    exp64_store<kFull>(x1, sl2, -m_new * sl2, tS + kPOff + 32, sa0, sa1, sb0, sb1);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -395,23 +493,22 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (!wait_bar(b_sfull, ph_s, abort)) { ok = false; break; }
                 ph_s ^= 1;
                 tc_fence_after();
-                float x[BN];
-                {
-                    uint32_t r[BN];
-                    tmem_ld128(tS, r);
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(r[c]);
-                }
                 const KvBlock kb = kv_block(qb, j, it.ctx, it.n, BM, BN);
-                if (!kb.full) {
-                    const int lim = col_limit(kb, row, BN);
+                const int lim = kb.full ? BN : col_limit(kb, row, BN);
+                if (j != it.j_lo) {
+                    if (kb.full) softmax_block_stream<D, true>(tS, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
+                    else softmax_block_stream<D, false>(tS, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
+                } else {
+                    float x[BN];
+                    {
+                        uint32_t r[BN];
+                        tmem_ld128(tS, r);
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (c >= lim) x[c] = -CUDART_INF_F;
+                        for (int c = 0; c < BN; ++c) x[c] = (c < lim) ? __uint_as_float(r[c]) : -CUDART_INF_F;
+                    }
+                    if (kb.full) softmax_block<D, true>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
+                    else softmax_block<D, false>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
                 }
-                const bool first = j == it.j_lo;
-                if (kb.full) softmax_block<D, true>(x, first, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
-                else softmax_block<D, false>(x, first, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
             }
             if (!ok) break;
             // final O / l -> bf16 rows of out
