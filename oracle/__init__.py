@@ -45,7 +45,7 @@ def _configure(lib):
     P = ctypes.c_void_p
     I = ctypes.c_int
     D = ctypes.c_double
-    prob = [P, P, P, P, P, I, I, I, I, D, P, I, P, I, I]
+    prob = [P, P, P, P, P, I, I, I, I, D, P, I, P, I, I, I]
     lib.oracle_attention_rows.argtypes = prob + [P, P, I, P]
     lib.oracle_attention_all.argtypes = prob + [P]
     lib.oracle_softmax_weights.argtypes = prob + [I, I, P, P]
@@ -89,7 +89,9 @@ def _ptr(a: Optional[np.ndarray]):
 
 class _Problem:
     def __init__(self, q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale,
-                 context_lens=None, kv_cache=None, block_table=None, block_size=16):
+                 context_lens=None, kv_cache=None, block_table=None, block_size=16, window=0):
+        if window < 0:
+            raise ValueError("window must be >= 0 (0: no window)")
         self.q, self.k, self.v = _bits(q), _bits(k), _bits(v)
         self.cu = _i32(cu_seqlens)
         self.ctx = None if context_lens is None else _i32(context_lens)
@@ -99,7 +101,7 @@ class _Problem:
         self.mbps = 0 if block_table is None else int(self.bt.shape[1]) if self.bt.ndim == 2 else int(self.bt.shape[0])
         self.args = (_ptr(self.q), _ptr(self.k), _ptr(self.v), _ptr(self.cu), _ptr(self.ctx),
                      len(self.cu) - 1, n_head, n_kv_head, head_dim, float(scale),
-                     _ptr(self.cache), self.num_blocks, _ptr(self.bt), self.mbps, block_size)
+                     _ptr(self.cache), self.num_blocks, _ptr(self.bt), self.mbps, block_size, int(window))
         self.n_head, self.head_dim = n_head, head_dim
 
 
@@ -109,11 +111,12 @@ def _check(rc: int, what: str):
 
 
 def attention(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale, *,
-              context_lens=None, kv_cache=None, block_table=None, block_size=16) -> np.ndarray:
+              context_lens=None, kv_cache=None, block_table=None, block_size=16, window=0) -> np.ndarray:
     """Full output [T, n_head, head_dim] in fp64.  With ``context_lens`` the
-    prefix keys come from ``kv_cache`` (as it stands) through ``block_table``."""
+    prefix keys come from ``kv_cache`` (as it stands) through ``block_table``.
+    ``window`` W >= 1 limits row P to keys P-W+1 .. P (0: plain causal)."""
     p = _Problem(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale,
-                 context_lens, kv_cache, block_table, block_size)
+                 context_lens, kv_cache, block_table, block_size, window)
     T = int(p.cu[-1]) if len(p.cu) else 0
     out = np.zeros((T, n_head, head_dim), dtype=np.float64)
     _check(_load().oracle_attention_all(*p.args, _ptr(out)), "oracle_attention_all")
@@ -122,10 +125,10 @@ def attention(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale, *,
 
 def attention_rows(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale, rows: Sequence[int],
                    heads: Sequence[int], *, context_lens=None, kv_cache=None, block_table=None,
-                   block_size=16) -> np.ndarray:
+                   block_size=16, window=0) -> np.ndarray:
     """Output rows for selected (packed row, head) pairs: [n_sel, head_dim] fp64."""
     p = _Problem(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale,
-                 context_lens, kv_cache, block_table, block_size)
+                 context_lens, kv_cache, block_table, block_size, window)
     r = _i32(rows)
     h = _i32(heads)
     assert r.shape == h.shape
@@ -136,9 +139,11 @@ def attention_rows(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale, rows
 
 
 def softmax_weights(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale, row: int, head: int, *,
-                    context_lens=None, kv_cache=None, block_table=None, block_size=16) -> np.ndarray:
+                    context_lens=None, kv_cache=None, block_table=None, block_size=16,
+                    window=0) -> np.ndarray:
+    """Softmax weights of one (row, head) over keys 0 .. P (0 outside the window)."""
     p = _Problem(q, k, v, cu_seqlens, n_head, n_kv_head, head_dim, scale,
-                 context_lens, kv_cache, block_table, block_size)
+                 context_lens, kv_cache, block_table, block_size, window)
     mk = int(max((p.ctx[i] if p.ctx is not None else 0) + p.cu[i + 1] - p.cu[i]
                  for i in range(len(p.cu) - 1)))
     w = np.zeros(max(mk, 1), dtype=np.float64)
@@ -164,14 +169,14 @@ def kv_write(k, v, cu_seqlens, kv_cache: torch.Tensor, block_table, block_size, 
     return torch.from_numpy(cache.view(np.int16)).view(torch.bfloat16).reshape(kv_cache.shape)
 
 
-def prefill(w, *, kv_cache=None, context_lens=None, rows=None, heads=None):
+def prefill(w, *, kv_cache=None, context_lens=None, rows=None, heads=None, window=0):
     """Oracle for one call on a ``workloads.Workload``-shaped problem:
     attention first (prefix read from the cache as it stood), then the KV
     write.  Returns (out fp64, new cache)."""
     cache = w.empty_cache() if kv_cache is None else kv_cache
     kw = dict(context_lens=context_lens, kv_cache=cache if context_lens is not None else None,
               block_table=w.block_table if context_lens is not None else None,
-              block_size=w.block_size)
+              block_size=w.block_size, window=window)
     if rows is None:
         out = attention(w.q, w.k, w.v, w.cu_seqlens, w.n_head, w.n_kv_head, w.head_dim, w.scale, **kw)
     else:

@@ -9,6 +9,7 @@
  *   absolute position    P  = ctx_i + a                (ctx_i = 0 unless chunked)
  *   kv head              g  = h / (n_head / n_kv_head)  (contiguous GQA groups)
  *   visible keys         j = 0 .. P                     (causal: j <= P)
+ *                        j = P - W + 1 .. P (and >= 0)   (sliding window of W keys)
  *   key / value row j    = cache row (page block_table[i][j / bs], slot j % bs)
  *                          if j < ctx_i, else the input row j - ctx_i
  *   score                s_j = scale * sum_d q[d] * k_j[d]
@@ -32,13 +33,17 @@
  *   hncyxsy.com/news/227904 §2.1 -- chunked prefill: a chunk needs the K/V of
  *       all earlier tokens.
  *   lnwmold.com/news/496245 §1.1 -- attention_scores = Q K^T / sqrt(d_head).
+ *   lnwmold.com/news/496245 §4.1 -- sliding-window attention: each token
+ *       attends only to its W nearest predecessors, n*W work instead of n^2.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   the scale is the caller's float, widened to fp64; disallowed keys are
  *   left out of the sum (no -inf arithmetic); GQA groups are contiguous; a
  *   chunk is aligned bottom-right (row a sits at absolute position ctx + a);
  *   the cache page is [2][block_size][n_kv_head][head_dim]; the prefix is read
- *   from the cache as it stood before the call.
+ *   from the cache as it stood before the call; a window of W keys counts the
+ *   token itself (row P sees keys P-W+1 .. P, so n rows cost n*W pairs once
+ *   P >= W - 1), W = 0 meaning no window.
  *
  * Parity pins: every function here is checked against closed forms,
  * invariants, a brute-force loop and a library routine by the CPU tests.
@@ -70,6 +75,7 @@ typedef struct {
     int num_blocks;
     const int32_t *block_table;
     int max_blocks_per_seq, block_size;
+    int window; /* 0: plain causal; W >= 1: keys P-W+1 .. P only */
 } problem_t;
 
 /* Sequence holding packed row t (cu_seqlens is non-decreasing). */
@@ -99,7 +105,8 @@ static const uint16_t *kv_row(const problem_t *p, int i, int j, int g, int which
 }
 
 /* One output row: query row t (packed index), query head h.
- * w: scratch of at least (P + 1) doubles; on return w[j] = softmax weight. */
+ * w: scratch of at least (P + 1) doubles; on return w[j] = softmax weight
+ * (exactly 0 for keys outside the window). */
 static int attend_one(const problem_t *p, int t, int h, double *out, double *w, int *n_keys) {
     int i = seq_of_row(p, t);
     if (i < 0) return ORACLE_ERR_ARG;
@@ -113,10 +120,14 @@ static int attend_one(const problem_t *p, int t, int h, double *out, double *w, 
 
     double qd[512];
     for (int x = 0; x < d; ++x) qd[x] = bf16_bits_to_double(qrow[x]);
+    /* first visible key: 0, or the start of the window ending at P */
+    int j0 = 0;
+    if (p->window > 0 && P - p->window + 1 > 0) j0 = P - p->window + 1;
+    for (int j = 0; j < j0; ++j) w[j] = 0.0;
 
-    /* pass 1: scores and their maximum (keys 0..P; the rest are masked out) */
+    /* pass 1: scores and their maximum (keys j0..P; the rest are masked out) */
     double m = -INFINITY;
-    for (int j = 0; j <= P; ++j) {
+    for (int j = j0; j <= P; ++j) {
         const uint16_t *krow = kv_row(p, i, j, g, 0);
         if (!krow) return ORACLE_ERR_BLOCK_TABLE;
         double dot = 0.0;
@@ -127,14 +138,14 @@ static int attend_one(const problem_t *p, int t, int h, double *out, double *w, 
     }
     /* pass 2: exponentials and their sum */
     double l = 0.0;
-    for (int j = 0; j <= P; ++j) {
+    for (int j = j0; j <= P; ++j) {
         w[j] = exp(w[j] - m);
         l += w[j];
     }
-    for (int j = 0; j <= P; ++j) w[j] /= l;
+    for (int j = j0; j <= P; ++j) w[j] /= l;
     /* weighted sum with V */
     for (int x = 0; x < d; ++x) out[x] = 0.0;
-    for (int j = 0; j <= P; ++j) {
+    for (int j = j0; j <= P; ++j) {
         const uint16_t *vrow = kv_row(p, i, j, g, 1);
         if (!vrow) return ORACLE_ERR_BLOCK_TABLE;
         for (int x = 0; x < d; ++x) out[x] += w[j] * bf16_bits_to_double(vrow[x]);
@@ -149,6 +160,7 @@ static int check_problem(const problem_t *p) {
     if (p->n_head % p->n_kv_head) return ORACLE_ERR_ARG;
     if (p->head_dim < 1 || p->head_dim > 512) return ORACLE_ERR_ARG;
     if (p->context_lens && (!p->kv_cache || !p->block_table || p->block_size < 1)) return ORACLE_ERR_ARG;
+    if (p->window < 0) return ORACLE_ERR_ARG;
     return ORACLE_OK;
 }
 
@@ -166,12 +178,12 @@ static int max_keys(const problem_t *p) {
     const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *cu_seqlens,   \
     const int32_t *context_lens, int num_seqs, int n_head, int n_kv_head, int head_dim,  \
     double scale, const uint16_t *kv_cache, int num_blocks, const int32_t *block_table,   \
-    int max_blocks_per_seq, int block_size
+    int max_blocks_per_seq, int block_size, int window
 
 #define PROBLEM_INIT                                                                       \
     problem_t pr = {q, k, v, cu_seqlens, context_lens, num_seqs, n_head, n_kv_head,       \
                     head_dim, scale, kv_cache, num_blocks, block_table, max_blocks_per_seq, \
-                    block_size};                                                            \
+                    block_size, window};                                                    \
     int rc0 = check_problem(&pr);                                                          \
     if (rc0) return rc0;
 

@@ -29,9 +29,14 @@ MUTANTS = {
                          "size_t slot = (size_t)((j + 1) % p->block_size);"),
     "v_written_over_k": ("uint16_t *vd = kv_cache + (((size_t)page * 2 + 1)",
                          "uint16_t *vd = kv_cache + (((size_t)page * 2 + 0)"),
-    "no_normalisation": ("for (int j = 0; j <= P; ++j) w[j] /= l;", "for (int j = 0; j <= P; ++j) w[j] /= 1.0;"),
+    "no_normalisation": ("for (int j = j0; j <= P; ++j) w[j] /= l;", "for (int j = j0; j <= P; ++j) w[j] /= 1.0;"),
     "value_column_fixed": ("out[x] += w[j] * bf16_bits_to_double(vrow[x]);",
                            "out[x] += w[j] * bf16_bits_to_double(vrow[0]);"),
+    "window_excludes_self": ("j0 = P - p->window + 1;", "j0 = P - p->window + 2;"),
+    "window_one_key_too_wide": ("j0 = P - p->window + 1;", "j0 = P - p->window;"),
+    "window_ignored": ("if (p->window > 0 && P - p->window + 1 > 0)", "if (0)"),
+    "window_from_chunk_row": ("if (p->window > 0 && P - p->window + 1 > 0) j0 = P - p->window + 1;",
+                              "if (p->window > 0 && a - p->window + 1 > 0) j0 = a - p->window + 1;"),
 }
 
 # pins run against each mutant (the cheap ones; the byte-count pin is run separately)
@@ -47,6 +52,9 @@ PIN_CALLS = [
     lambda: pins.test_chunked_equals_unchunked(100, 16),
     lambda: pins.test_block_table_invariance_and_gather(),
     lambda: pins.test_chunk_prefix_read_through_table(),
+    lambda: pins.test_window_one_outputs_own_value_exactly(),
+    lambda: pins.test_window_matches_torch_sdpa_band_mask([300, 129, 2], 64),
+    lambda: pins.test_window_chunk_matches_torch_sdpa_band_mask(),
 ]
 
 

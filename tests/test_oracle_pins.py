@@ -296,3 +296,135 @@ def test_bad_block_table_is_reported():
     bt[0, 1] = w.num_blocks + 3
     with pytest.raises(RuntimeError):
         oracle.kv_write(w.k, w.v, w.cu_seqlens, w.empty_cache(), bt, 16)
+
+
+# ---------------------------------------------------------------- sliding window
+# A window of W keys (lnwmold.com/news/496245 §4.1): row P sees keys
+# max(0, P-W+1) .. P.  Pinned by closed forms (W = 1; identical keys), by
+# reduction to plain causal attention (a wide window; a truncated sequence),
+# by torch's fp64 SDPA with an explicit band mask, and by a brute-force loop.
+
+def test_window_one_outputs_own_value_exactly():
+    w = _tiny([9, 33, 1, 64], 8, 2, 64, seed=40)
+    out = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, 8, 2, 64, w.scale, window=1)
+    v = _f64(w.v)
+    for h in range(8):
+        assert np.array_equal(out[:, h], v[:, h // 4])
+
+
+def test_wide_window_equals_plain_causal():
+    w = _tiny([70, 5, 129], 4, 2, 32, seed=41)
+    plain = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, 4, 2, 32, w.scale)
+    for win in (129, 130, 10_000):
+        out = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, 4, 2, 32, w.scale, window=win)
+        assert np.array_equal(out, plain)
+    # one key too narrow changes the last row of the longest sequence
+    out = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, 4, 2, 32, w.scale, window=128)
+    assert not np.array_equal(out[-1], plain[-1])
+    assert np.array_equal(out[:-1], plain[:-1])
+
+
+def test_window_equals_causal_on_truncated_sequence():
+    """Row a under window W is the last row of plain causal attention over
+    tokens a-W+1 .. a alone (positions only enter through the mask)."""
+    H, G, d, s, win = 4, 2, 16, 90, 23
+    w = _tiny([s], H, G, d, seed=42)
+    out = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, H, G, d, w.scale, window=win)
+    for a in (0, 5, 21, 22, 23, 50, 89):
+        b0 = max(0, a - win + 1)
+        n = a + 1 - b0
+        o1 = oracle.attention(w.q[b0:a + 1], w.k[b0:a + 1], w.v[b0:a + 1], torch.tensor([0, n], dtype=torch.int32),
+                              H, G, d, w.scale)
+        assert np.max(np.abs(out[a] - o1[-1])) < 1e-13
+
+
+def _band_mask(q_pos, n_keys, win):
+    j = torch.arange(n_keys)[None, :]
+    P = q_pos[:, None]
+    return (j <= P) & (j > P - win)
+
+
+@pytest.mark.parametrize("seqlens,win", [([300, 129, 2], 64), ([200], 1), ([150], 149)])
+def test_window_matches_torch_sdpa_band_mask(seqlens, win):
+    H, G, d = 8, 2, 32
+    w = _tiny(seqlens, H, G, d, seed=43)
+    out = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, H, G, d, w.scale, window=win)
+    for i in range(w.num_seqs):
+        a, b = int(w.cu_seqlens[i]), int(w.cu_seqlens[i + 1])
+        q = w.q[a:b].to(torch.float64).transpose(0, 1)
+        k = w.k[a:b].to(torch.float64).repeat_interleave(H // G, 1).transpose(0, 1)
+        v = w.v[a:b].to(torch.float64).repeat_interleave(H // G, 1).transpose(0, 1)
+        mask = _band_mask(torch.arange(b - a), b - a, win)
+        ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=w.scale)
+        assert np.max(np.abs(out[a:b] - ref.transpose(0, 1).numpy())) < 1e-10
+
+
+def test_window_chunk_matches_torch_sdpa_band_mask():
+    """Chunked mode: the window is counted in absolute positions, so it
+    reaches back into the cached prefix."""
+    H, G, d, ctx, L, win = 4, 2, 32, 70, 45, 50
+    w = _tiny([ctx + L], H, G, d, seed=44, bs=16)
+    cache = oracle.kv_write(w.k[:ctx], w.v[:ctx], torch.tensor([0, ctx], dtype=torch.int32),
+                            w.empty_cache(), w.block_table, 16)
+    out = oracle.attention(w.q[ctx:], w.k[ctx:], w.v[ctx:], torch.tensor([0, L], dtype=torch.int32),
+                           H, G, d, w.scale, context_lens=[ctx], kv_cache=cache,
+                           block_table=w.block_table, block_size=16, window=win)
+    q = w.q[ctx:].to(torch.float64).transpose(0, 1)
+    k = w.k.to(torch.float64).repeat_interleave(H // G, 1).transpose(0, 1)
+    v = w.v.to(torch.float64).repeat_interleave(H // G, 1).transpose(0, 1)
+    mask = _band_mask(ctx + torch.arange(L), ctx + L, win)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=w.scale)
+    assert np.max(np.abs(out - ref.transpose(0, 1).numpy())) < 1e-10
+
+
+def test_window_brute_force_tiny():
+    H, G, d, win = 4, 2, 3, 3
+    w = _tiny([9, 4], H, G, d, seed=45, scale=0.41)
+    q = (w.q.float() * 0.5).to(torch.bfloat16)
+    out = oracle.attention(q, w.k, w.v, w.cu_seqlens, H, G, d, 0.41, window=win)
+    qq, kk, vv = _f64(q), _f64(w.k), _f64(w.v)
+    for i in range(w.num_seqs):
+        a0, a1 = int(w.cu_seqlens[i]), int(w.cu_seqlens[i + 1])
+        for h in range(H):
+            g = h * G // H
+            for a in range(a0, a1):
+                num, den = np.zeros(d), 0.0
+                for b in range(a0, a + 1):
+                    if a - b >= win:
+                        continue
+                    e = math.exp(0.41 * sum(qq[a, h, x] * kk[b, g, x] for x in range(d)))
+                    den += e
+                    num += e * vv[b, g]
+                assert np.max(np.abs(out[a, h] - num / den)) < 1e-12
+
+
+def test_window_weights_and_identical_keys():
+    H, G, d, win = 4, 4, 32, 7
+    w = _tiny([50], H, G, d, seed=46)
+    for row in (0, 3, 6, 7, 49):
+        p = oracle.softmax_weights(w.q, w.k, w.v, w.cu_seqlens, H, G, d, w.scale, row, 2, window=win)
+        assert len(p) == row + 1
+        assert abs(p.sum() - 1.0) < 1e-12
+        assert np.count_nonzero(p) == min(row + 1, win)
+        assert (p[: max(0, row - win + 1)] == 0).all()
+    k = w.k.clone()
+    k[:] = k[0:1]
+    out = oracle.attention(w.q, k, w.v, w.cu_seqlens, H, G, d, w.scale, window=win)
+    v = _f64(w.v)
+    for a in range(50):
+        b0 = max(0, a - win + 1)
+        assert np.max(np.abs(out[a] - v[b0:a + 1].mean(axis=0))) < 1e-12
+
+
+def test_window_chunked_equals_unchunked():
+    H, G, d, s, bs, win = 4, 2, 32, 260, 16, 75
+    w = _tiny([s], H, G, d, seed=47, bs=bs)
+    full_out, full_cache = oracle.prefill(w, window=win)
+    cache = w.empty_cache()
+    outs = []
+    for q, k, v, cu, ctx, bt in W.chunk_views(w, 64):
+        outs.append(oracle.attention(q, k, v, cu, H, G, d, w.scale, context_lens=ctx, kv_cache=cache,
+                                     block_table=bt, block_size=bs, window=win))
+        cache = oracle.kv_write(k, v, cu, cache, bt, bs, context_lens=ctx)
+    assert np.max(np.abs(np.concatenate(outs, axis=0) - full_out)) < 1e-12
+    assert torch.equal(cache.view(torch.int16), full_cache.view(torch.int16))
