@@ -168,6 +168,25 @@ class ChunkedRunner:
             raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
 
 
+class WindowRunner(PlainRunner):
+    """prefill_attn_sliding_window over one workload; FLOPs counted over the
+    visible pairs only (4*d*H per pair, min(a + 1, window) keys for row a)."""
+
+    def __init__(self, w: W.Workload, window: int, stream):
+        super().__init__(w, stream)
+        self.window = window
+        self.flops = w.window_flops(window)
+
+    def step(self):
+        _lib.prefill_attn_sliding_window(self.q, self.k, self.v, self.cu, None, self.w.max_seqlen, 0, self.w.scale,
+                                         self.window, self.out, self.cache, self.bt, status=self.status,
+                                         stream=self.stream)
+
+
+# secondary line: the headline prompt under a sliding window of this many keys
+WINDOW_LINE = ("swa4096_gqa_s8192_h32g8_d128", "gqa_s8192_h32g8_d128", 4096)
+
+
 def time_steps(runner, steps, warmup, stream, flush):
     for _ in range(warmup):
         runner.step()
@@ -336,6 +355,16 @@ def main():
                            "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches}
             del rx, wx
             torch.cuda.empty_cache()
+        name, base, win = WINDOW_LINE
+        wx = W.named_workload(base)
+        rx = WindowRunner(wx, win, stream)
+        dx = time_steps(rx, max(5, args.steps // 2), 3, stream, flush)
+        mx = statistics.median(dx)
+        extra[name] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
+                       "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches,
+                       "window": win}
+        del rx, wx
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1:

@@ -21,7 +21,8 @@ STATUS_NAMES = {
 }
 EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall",
-            "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes")
+            "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
+            "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window")
 
 _lib = None
 
@@ -56,6 +57,12 @@ def load() -> ctypes.CDLL:
         lib.prefill_attn_chunked_noalloc.restype = I
         lib.prefill_noalloc_scratch_bytes.argtypes = []
         lib.prefill_noalloc_scratch_bytes.restype = ctypes.c_size_t
+        lib.prefill_attn_sliding_window.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, F, I, P, P, I, P, I, I, P, P]
+        lib.prefill_attn_sliding_window.restype = I
+        lib.prefill_first_kv_block.argtypes = [I, I, I, I, I, I]
+        lib.prefill_first_kv_block.restype = I
+        lib.prefill_kv_block_rule_window.argtypes = [I, I, I, I, I, I, I, P, P, P]
+        lib.prefill_kv_block_rule_window.restype = I
         _lib = lib
     return _lib
 
@@ -152,6 +159,31 @@ def prefill_attn_chunked_noalloc(q, k, v, cu_seqlens_q, context_lens, max_q_len:
     return rc
 
 
+def prefill_attn_sliding_window(q, k, v, cu_seqlens_q, context_lens, max_q_len: int, max_context_len: int,
+                                scale: float, window: int, out, kv_cache, block_table,
+                                status: Optional[torch.Tensor] = None, stream=None,
+                                raise_on_error: bool = True) -> int:
+    """Causal prefill with a sliding window of ``window`` keys (C ABI
+    ``prefill_attn_sliding_window``): row P sees keys P-window+1 .. P.
+    ``context_lens`` None means plain prefill (``max_context_len`` 0)."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3)
+    _check_bf16("out", out, 3), _check_bf16("kv_cache", kv_cache, 5)
+    _check_i32("cu_seqlens_q", cu_seqlens_q), _check_i32("block_table", block_table)
+    if context_lens is not None:
+        _check_i32("context_lens", context_lens)
+    T, H, D = q.shape
+    G = k.shape[1]
+    rc = load().prefill_attn_sliding_window(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(cu_seqlens_q), _ptr(context_lens), cu_seqlens_q.numel() - 1,
+        int(max_q_len), int(max_context_len), H, G, D, float(scale), int(window), _ptr(out), _ptr(kv_cache),
+        kv_cache.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "prefill_attn_sliding_window")
+    return rc
+
+
 def inject_stall(enable: bool = True) -> None:
     """Test hook: the next pipelined launch withholds one Q tile so that a
     bounded device wait expires and the call reports PREFILL_ERR_TIMEOUT."""
@@ -168,3 +200,16 @@ def kv_block_rule(qb: int, j: int, ctx: int, n: int, bm: int = 128, bn: int = 12
     kb = ctypes.c_int32(0)
     kind = load().prefill_kv_block_rule(qb, j, ctx, n, bm, bn, lim, ctypes.byref(kb))
     return kind, list(lim), kb.value
+
+
+def first_kv_block(qb: int, ctx: int, n: int, window: int, bm: int = 128, bn: int = 128) -> int:
+    return load().prefill_first_kv_block(qb, ctx, n, bm, bn, window)
+
+
+def kv_block_rule_window(qb: int, j: int, ctx: int, n: int, window: int, bm: int = 128, bn: int = 128):
+    """(kind, col_lo[bm], col_limit[bm], key_begin) under a sliding window."""
+    lo = (ctypes.c_int32 * bm)()
+    lim = (ctypes.c_int32 * bm)()
+    kb = ctypes.c_int32(0)
+    kind = load().prefill_kv_block_rule_window(qb, j, ctx, n, bm, bn, window, lo, lim, ctypes.byref(kb))
+    return kind, list(lo), list(lim), kb.value

@@ -102,13 +102,14 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
                 const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
                 int n_kv_head, int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *cache, int num_blocks,
                 const int32_t *bt, int mbps, int bs, int32_t *status, prefill_stream_t stream, void *scratch,
-                size_t scratch_bytes) {
+                size_t scratch_bytes, int window) {
     if (!q || !k || !v || !cu || !out || !cache || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
     if (total < 0 || num_seqs < 0 || max_q < 0 || max_ctx < 0) return PREFILL_ERR_SHAPE;
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
     if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
     if (bs != 16 && bs != 32 && bs != 64 && bs != 128) return PREFILL_ERR_UNSUPPORTED;
     if (!(std::isfinite(scale) && scale > 0.f)) return PREFILL_ERR_UNSUPPORTED;
+    if (window < 0) return PREFILL_ERR_SHAPE;
     if (num_blocks < 1 || mbps < 1) return PREFILL_ERR_BLOCK_TABLE;
     // each bound must fit the table; the exact per-sequence check (context +
     // chunk length) runs on the device, where the lengths are
@@ -165,6 +166,7 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     p.scale_log2 = scale * 1.4426950408889634f;
     p.test_stall = g_test_stall.exchange(0);
     p.max_ctx = (int)max_ctx;
+    p.window = window;
     p.nsplit = 1;
     p.part_o = nullptr;
     p.part_ml = nullptr;
@@ -215,6 +217,20 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
                            max_blocks_per_seq, block_size, status_dev, stream, nullptr, 0);
 }
 
+int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,
+                                const int32_t *cu_seqlens_q, const int32_t *context_lens, int num_seqs,
+                                int max_q_len, int max_context_len, int n_head, int n_kv_head, int head_dim,
+                                float scale, int window, prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks,
+                                const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                                int32_t *status_dev, prefill_stream_t stream) {
+    if (window < 1) return PREFILL_ERR_SHAPE;
+    if (!context_lens && max_context_len != 0) return PREFILL_ERR_SHAPE;
+    return pf::run_prefill(q, k, v, total_q, cu_seqlens_q, context_lens, context_lens != nullptr, num_seqs,
+                           max_q_len, max_context_len, n_head, n_kv_head, head_dim, scale, out, kv_cache,
+                           num_blocks, block_table, max_blocks_per_seq, block_size, status_dev, stream, nullptr, 0,
+                           window);
+}
+
 void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }
 
 const char *prefill_status_string(int s) {
@@ -239,11 +255,25 @@ int prefill_num_kv_blocks(int qb, int ctx, int n, int bm, int bn) {
 }
 
 int prefill_kv_block_rule(int qb, int j, int ctx, int n, int bm, int bn, int32_t *col_limit, int32_t *key_begin) {
-    if (bm < 1 || bn < 1 || ctx < 0 || n < 0 || j < 0 || j >= prefill_num_kv_blocks(qb, ctx, n, bm, bn)) return -1;
-    const pf::KvBlock b = pf::kv_block(qb, j, ctx, n, bm, bn);
+    return prefill_kv_block_rule_window(qb, j, ctx, n, bm, bn, 0, nullptr, col_limit, key_begin);
+}
+
+int prefill_first_kv_block(int qb, int ctx, int n, int bm, int bn, int window) {
+    if (bm < 1 || bn < 1 || ctx < 0 || n < 0 || window < 0) return 0;
+    return pf::first_kv_block(qb, ctx, n, bm, bn, window);
+}
+
+int prefill_kv_block_rule_window(int qb, int j, int ctx, int n, int bm, int bn, int window, int32_t *col_lo,
+                                 int32_t *col_limit, int32_t *key_begin) {
+    if (bm < 1 || bn < 1 || ctx < 0 || n < 0 || window < 0) return -1;
+    if (j < prefill_first_kv_block(qb, ctx, n, bm, bn, window) || j >= prefill_num_kv_blocks(qb, ctx, n, bm, bn))
+        return -1;
+    const pf::KvBlock b = pf::kv_block(qb, j, ctx, n, bm, bn, window);
     if (key_begin) *key_begin = b.key_begin;
-    if (col_limit)
-        for (int r = 0; r < bm; ++r) col_limit[r] = b.full ? bn : pf::col_limit(b, r, bn);
+    for (int r = 0; r < bm; ++r) {
+        if (col_limit) col_limit[r] = b.full ? bn : pf::col_limit(b, r, bn);
+        if (col_lo) col_lo[r] = b.full ? 0 : pf::col_lo(b, r, bn);
+    }
     return b.full ? 0 : 1;
 }
 

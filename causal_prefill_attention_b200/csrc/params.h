@@ -26,6 +26,7 @@ struct FwdParams {
     float scale_log2;             // scale * log2(e)
     int test_stall;               // test hook: withhold one Q tile (see prefill_test_inject_stall)
     int max_ctx;                  // bound on every context length (chunked prefill; 0 otherwise)
+    int window;                   // sliding window: row P sees keys P-window+1 .. P (<= 0: none)
     // split-KV: kv ranges split into up to nsplit parts; the partial results go to
     // part_o [nsplit][total][n_head][D] (fp32, unnormalised) and part_ml
     // [nsplit][total][n_head][2] (running max in log2 units, exp-sum)
@@ -54,10 +55,11 @@ int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void
 // Host path shared by the C entry points (api.cu).  scratch / scratch_bytes:
 // caller-supplied split-KV scratch (nullptr: the library's own workspace);
 // a split that needs more than scratch_bytes returns PREFILL_ERR_SCRATCH_LIMIT.
+// window: sliding window of that many keys (0: plain causal).
 int run_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int total, const int32_t *cu,
                 const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
                 int n_kv_head, int head_dim, float scale, uint16_t *out, uint16_t *cache, int num_blocks,
                 const int32_t *bt, int mbps, int bs, int32_t *status, struct CUstream_st *stream, void *scratch,
-                size_t scratch_bytes);
+                size_t scratch_bytes, int window = 0);
 
 }  // namespace pf

@@ -47,6 +47,8 @@ constexpr uint32_t CHUNK = 128 * 128;  // 128 rows x 64 bf16, 128B-swizzled
 constexpr float kRescaleLog2 = 8.0f;
 // P (bf16 pairs) occupies the first 64 columns of its S region.
 constexpr uint32_t kPOff = 0;
+// Running max of a row that has seen no visible key yet (finite, far below any score).
+constexpr float kNoKeyMax = -1e30f;
 // Which of the 32 column pairs in each 64-column half of an unmasked block take
 // their exponentials on the FMA pipe (exp2_fma2) instead of MUFU (ex2).
 #ifndef PF_EXP2_EMU_MASK
@@ -118,8 +120,10 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
                                               float &l_run, uint32_t tS, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
                                               int lane) {
     float mt = first ? rowmax128(x) : 0.f;
-    float m_ref = first ? mt : m_run;
-    if (m_ref == -CUDART_INF_F) m_ref = 0.f;  // nothing visible yet (cannot happen under causal masking)
+    // a row with nothing visible in its first block (a sliding window's edge)
+    // takes a finite floor as its max: its P is 0, and the first block that
+    // shows it a key moves the max and rescales the empty O and l by exactly 0
+    float m_ref = first ? fmaxf(mt, kNoKeyMax) : m_run;
     float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
     {
         uint32_t pw[32];
@@ -209,7 +213,7 @@ __device__ __forceinline__ float rowmax64x2(const float (&a)[64], const float (&
 // halves are in (half 0 is redone and O rescaled only if it moved past the
 // threshold).  P goes to TMEM in two halves, announced on b_pa / b_pb.
 template <int D, bool kFull>
-__device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lim, float sl2, float thr, float &m_run,
+__device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lo, int lim, float sl2, float thr, float &m_run,
                                                      float &l_run, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
                                                      int lane) {
     float x0[64], x1[64];
@@ -225,13 +229,14 @@ __device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lim, float
     if (!kFull) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-            if (c >= lim) x0[c] = -CUDART_INF_F;
+            if (c < lo || c >= lim) x0[c] = -CUDART_INF_F;
     }
     float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
     exp64_store<kFull>(x0, sl2, -m_run * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
     tmem_wait_ld_tie64(r1);
 #pragma unroll
-    for (int c = 0; c < 64; ++c) x1[c] = (kFull || 64 + c < lim) ? __uint_as_float(r1[c]) : -CUDART_INF_F;
+    for (int c = 0; c < 64; ++c)
+        x1[c] = (kFull || (64 + c >= lo && 64 + c < lim)) ? __uint_as_float(r1[c]) : -CUDART_INF_F;
     const float mt = rowmax64x2(x0, x1);
     const bool need = mt > m_run + thr;
     float m_new = m_run, alpha = 1.f;
@@ -265,20 +270,24 @@ __device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lim, float
 // ------------------------------------------------------------------ schedule
 struct Item {
     int i, h, g, qb0, c0, n, ctx;
-    int nk0, nk1;  // kv blocks visited by query block 0 / 1
+    int nk0, nk1;  // query block 0 / 1 visits kv blocks [jf0, nk0) / [jf1, nk1)
     int two;       // second query block present
     // split of the kv range (split-KV): this item covers kv blocks [j_lo, j_hi)
     int split, nsp, j_lo, j_hi;
+    int jb0, jb1;  // first kv block of query block 0 / 1 inside this split (j_lo without a window)
     bool skip;     // a split index beyond this pair's useful split count: no work
     __device__ __forceinline__ int nk(int s) const { return s ? nk1 : nk0; }
     __device__ __forceinline__ int nmax() const { return nk0 > nk1 ? nk0 : nk1; }
-    // end of query block s's blocks inside this split
+    // first / end of query block s's blocks inside this split
+    __device__ __forceinline__ int beg(int s) const { return s ? jb1 : jb0; }
     __device__ __forceinline__ int end(int s) const { return nk(s) < j_hi ? nk(s) : j_hi; }
 };
 
 // Useful number of splits of a pair whose kv range has nmax blocks: at most
 // nsplit, and every split keeps at least kMinSplitBlocks blocks (so query block
-// 0, which ends one block before query block 1, always has work in every split).
+// 0, which ends one block before query block 1, and query block 1, which
+// starts at most two blocks after query block 0 under a sliding window, always
+// have work in every split).
 constexpr int kMinSplitBlocks = 4;
 __host__ __device__ __forceinline__ int useful_splits(int nmax, int nsplit) {
     const int m = nmax / kMinSplitBlocks;
@@ -307,6 +316,9 @@ __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
 //   start[c] sequences with more than c pairs          (= first sorted slot of bucket c)
 //   B[c]     items of sequences with more than c pairs (= first item of bucket c)
 //   perm     sequence indices sorted by pair count, descending, stable
+// kWin: the kernel runs a sliding window (p.window keys); without it every
+// window term folds away at compile time.
+template <bool kWin>
 __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, const int *start, const uint16_t *perm,
                                             int P, int u_split) {
     const int u = u_split / p.nsplit;
@@ -334,11 +346,24 @@ __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, co
     it.nk0 = num_kv_blocks(it.qb0, it.ctx, it.n, BM, BN);
     it.nk1 = it.two ? num_kv_blocks(it.qb0 + 1, it.ctx, it.n, BM, BN) : 0;
     const int nmax = it.nmax();
-    it.nsp = useful_splits(nmax, p.nsplit);
     it.split = split;
-    it.skip = split >= it.nsp;
-    it.j_lo = (split * nmax) / it.nsp;
-    it.j_hi = ((split + 1) * nmax) / it.nsp;
+    if (!kWin) {
+        it.nsp = useful_splits(nmax, p.nsplit);
+        it.skip = split >= it.nsp;
+        it.j_lo = (split * nmax) / it.nsp;
+        it.j_hi = ((split + 1) * nmax) / it.nsp;
+        it.jb0 = it.jb1 = it.j_lo;
+    } else {
+        const int jf0 = first_kv_block(it.qb0, it.ctx, it.n, BM, BN, p.window);
+        const int jf1 = it.two ? first_kv_block(it.qb0 + 1, it.ctx, it.n, BM, BN, p.window) : jf0;
+        const int nrange = nmax - jf0;  // the pair's kv range [jf0, nmax)
+        it.nsp = useful_splits(nrange, p.nsplit);
+        it.skip = split >= it.nsp;
+        it.j_lo = jf0 + (split * nrange) / it.nsp;
+        it.j_hi = jf0 + ((split + 1) * nrange) / it.nsp;
+        it.jb0 = it.j_lo;  // jf0 <= j_lo
+        it.jb1 = jf1 > it.j_lo ? jf1 : it.j_lo;
+    }
     return it;
 }
 
@@ -359,7 +384,7 @@ __device__ __forceinline__ void setmaxnreg_softmax() { asm volatile("setmaxnreg.
 __device__ __forceinline__ void setmaxnreg_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
 
 // ------------------------------------------------------------------ kernel
-template <int D, int NST>
+template <int D, int NST, bool kWin>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_cache,
@@ -484,27 +509,31 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int k = 0; ok; ++k) {
             const int u = zigzag(k, cta, G);
             if (u >= total) break;
-            const Item it = decode_item(p, B, start, perm, P, u);
+            const Item it = decode_item<kWin>(p, B, start, perm, P, u);
             if (it.skip || (s == 1 && !it.two)) continue;
             const int qb = it.qb0 + s;
-            const int je = it.end(s);
+            const int jb = kWin ? it.beg(s) : it.j_lo, je = it.end(s);
             float m_run = -CUDART_INF_F, l_run = 0.f;
-            for (int j = it.j_lo; j < je; ++j) {
+            for (int j = jb; j < je; ++j) {
                 if (!wait_bar(b_sfull, ph_s, abort)) { ok = false; break; }
                 ph_s ^= 1;
                 tc_fence_after();
-                const KvBlock kb = kv_block(qb, j, it.ctx, it.n, BM, BN);
+                const KvBlock kb = kv_block(qb, j, it.ctx, it.n, BM, BN, kWin ? p.window : 0);
                 const int lim = kb.full ? BN : col_limit(kb, row, BN);
-                if (j != it.j_lo) {
-                    if (kb.full) softmax_block_stream<D, true>(tS, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
-                    else softmax_block_stream<D, false>(tS, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
+                const int lo = (kWin && !kb.full) ? col_lo(kb, row, BN) : 0;
+                if (j != jb) {
+                    if (kb.full)
+                        softmax_block_stream<D, true>(tS, lo, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
+                    else
+                        softmax_block_stream<D, false>(tS, lo, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
                 } else {
                     float x[BN];
                     {
                         uint32_t r[BN];
                         tmem_ld128(tS, r);
 #pragma unroll
-                        for (int c = 0; c < BN; ++c) x[c] = (c < lim) ? __uint_as_float(r[c]) : -CUDART_INF_F;
+                        for (int c = 0; c < BN; ++c)
+                            x[c] = (c >= lo && c < lim) ? __uint_as_float(r[c]) : -CUDART_INF_F;
                     }
                     if (kb.full) softmax_block<D, true>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
                     else softmax_block<D, false>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
@@ -573,7 +602,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item(p, B, start, perm, P, u);
+                const Item it = decode_item<kWin>(p, B, start, perm, P, u);
                 if (it.skip) continue;
                 const int ns = it.two ? 2 : 1;
                 for (int s = 0; s < ns; ++s) {
@@ -593,7 +622,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                 }
                 for (int j = it.j_lo; j < it.j_hi && ok; ++j) {
-                    const KvBlock kb = kv_block(it.qb0, j, it.ctx, it.n, BM, BN);
+                    const KvBlock kb = kv_block(it.qb0, j, it.ctx, it.n, BM, BN, 0);  // key range only
                     for (int t = 0; t < 2; ++t) {  // t = 0: K, t = 1: V
                         if (!wait_bar(bar(L::B_KVEMPTY + stage), phase ^ 1, abort)) { ok = false; break; }
                         const uint32_t dst = base + L::KV + stage * L::TILE;
@@ -695,7 +724,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item(p, B, start, perm, P, u);
+                const Item it = decode_item<kWin>(p, B, start, perm, P, u);
                 if (it.skip) continue;
                 const int ns = it.two ? 2 : 1;
                 const int j0 = it.j_lo, jend = it.j_hi;
@@ -711,6 +740,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (!wait_all(bar(L::B_KVFULL + kst), kph)) { ok = false; break; }
                 tc_fence_after();
                 for (int s = 0; s < ns; ++s) {
+                    if (kWin && it.beg(s) != j0) continue;  // a windowed query block 1 may start later
                     issue_s(s, kst);
                     tc_commit_elect(bar(L::B_SFULL + s));
                 }
@@ -729,19 +759,23 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (!wait_all(bar(L::B_KVFULL + vst), vph)) { ok = false; break; }
                     bool next_ready = false;
                     for (int s = 0; s < ns; ++s) {
-                        if (j >= it.end(s)) continue;
-                        if (!wait_all(bar(L::B_PA + s), (ph_pf >> s) & 1u)) { ok = false; break; }
-                        if (j == j0 && ((used >> s) & 1u)) {
-                            if (!wait_all(bar(L::B_OEMPTY + s), (ph_oe >> s) & 1u)) { ok = false; break; }
-                            ph_oe ^= 1u << s;
+                        // query block s visits [jb, je) of this split
+                        const int jb = kWin ? it.beg(s) : j0, je = it.end(s);
+                        const bool pv = (!kWin || j >= jb) && j < je;
+                        if (pv) {
+                            if (!wait_all(bar(L::B_PA + s), (ph_pf >> s) & 1u)) { ok = false; break; }
+                            if (j == jb && ((used >> s) & 1u)) {
+                                if (!wait_all(bar(L::B_OEMPTY + s), (ph_oe >> s) & 1u)) { ok = false; break; }
+                                ph_oe ^= 1u << s;
+                            }
+                            tc_fence_after();
+                            issue_pv(s, vst, j > jb, 0);
+                            if (!wait_all(bar(L::B_PB + s), (ph_pf >> s) & 1u)) { ok = false; break; }
+                            ph_pf ^= 1u << s;
+                            tc_fence_after();
+                            issue_pv(s, vst, j > jb, BN / 32);
                         }
-                        tc_fence_after();
-                        issue_pv(s, vst, j > j0, 0);
-                        if (!wait_all(bar(L::B_PB + s), (ph_pf >> s) & 1u)) { ok = false; break; }
-                        ph_pf ^= 1u << s;
-                        tc_fence_after();
-                        issue_pv(s, vst, j > j0, BN / 32);
-                        if (j + 1 < it.end(s)) {
+                        if ((!kWin || j + 1 >= jb) && j + 1 < je) {
                             if (!next_ready) {
                                 if (!wait_all(bar(L::B_KVFULL + nst), nph)) { ok = false; break; }
                                 tc_fence_after();
@@ -749,7 +783,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                             issue_s(s, nst);
                             tc_commit_elect(bar(L::B_SFULL + s));
-                        } else {
+                        } else if (pv) {
                             tc_commit_elect(bar(L::B_OFULL + s));
                             tc_commit_elect(bar(L::B_QEMPTY + s));
                         }
@@ -781,7 +815,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item(p, B, start, perm, P, u);
+                const Item it = decode_item<kWin>(p, B, start, perm, P, u);
                 if (it.skip) continue;
                 const int np = cdiv(it.ctx, BN);
                 const bool writes = (it.h % p.group) == 0;
@@ -873,7 +907,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(cons
                 const int qb0 = (a / (2 * BM)) * 2;
                 const bool two = (qb0 + 1) * BM < n;
                 const int nmax = two ? num_kv_blocks(qb0 + 1, ctx, n, BM, BN) : num_kv_blocks(qb0, ctx, n, BM, BN);
-                nsp = useful_splits(nmax, p.nsplit);
+                nsp = useful_splits(nmax - first_kv_block(qb0, ctx, n, BM, BN, p.window), p.nsplit);
             }
         }
         s_nsp = nsp;
@@ -944,18 +978,18 @@ int sm_count() {
     return n;
 }
 
-template <int D, int NST>
+template <int D, int NST, bool kWin>
 int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
     const size_t smem = smem_bytes<D, NST>(P, p.num_seqs);
-    cudaError_t e =
-        cudaFuncSetAttribute(prefill_fwd_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D, NST, kWin>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     const long long items_bound = (long long)p.num_seqs * p.n_head * P;
     const long long items = items_bound * (p.nsplit > 0 ? p.nsplit : 1);
     const int grid_s = (int)(items < sm_count() ? items : sm_count());
-    prefill_fwd_kernel<D, NST><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v, maps.cache,
-                                                                                  p, P);
+    prefill_fwd_kernel<D, NST, kWin><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v,
+                                                                                        maps.cache, p, P);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
     combine_splits_kernel<D><<<(unsigned)p.total, 32 * kCombineWarps, 0, (cudaStream_t)stream>>>(p);
@@ -965,8 +999,9 @@ int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
 template <int D>
 int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
-    if (smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem) return launch_nst<D, 5>(maps, p, stream);
-    return launch_nst<D, 4>(maps, p, stream);
+    const bool nst5 = smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem;
+    if (p.window > 0) return nst5 ? launch_nst<D, 5, true>(maps, p, stream) : launch_nst<D, 4, true>(maps, p, stream);
+    return nst5 ? launch_nst<D, 5, false>(maps, p, stream) : launch_nst<D, 4, false>(maps, p, stream);
 }
 
 }  // namespace
@@ -986,7 +1021,8 @@ int fwd_choose_splits(const FwdParams &p) {
     const long long items = (long long)p.num_seqs * p.n_head * cdiv(p.max_q, 2 * BM);
     const int sms = sm_count();
     if (items <= 0 || items >= sms) return 1;
-    const int nk = cdiv(p.max_ctx, BN) + cdiv(p.max_q, BN);
+    int nk = cdiv(p.max_ctx, BN) + cdiv(p.max_q, BN);
+    if (p.window > 0) nk = imin(nk, cdiv(p.window, BN) + 2);  // a windowed query block's range
     int best = 1;
     double best_cost = 1.0;  // waves per split at 1 split
     for (int sp = 2; sp <= 8; ++sp) {

@@ -98,11 +98,12 @@ prefill_fwd_v0_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     ph_load ^= 1;
 
     const int nkv = num_kv_blocks(qb, ctx, n, BM, BN);
+    const int j0 = first_kv_block(qb, ctx, n, BM, BN, p.window);  // 0 without a sliding window
     const int row = tid;  // query row of this thread inside the block (TMEM lane)
     float m_run = -CUDART_INF_F, l_run = 0.f;
 
-    for (int j = 0; j < nkv && ok; ++j) {
-        const KvBlock kb = kv_block(qb, j, ctx, n, BM, BN);
+    for (int j = j0; j < nkv && ok; ++j) {
+        const KvBlock kb = kv_block(qb, j, ctx, n, BM, BN, p.window);
         // ---- K, V block (prefix: gathered page by page from the cache)
         if (tid == 0) {
             if (kb.prefix) {
@@ -177,14 +178,16 @@ prefill_fwd_v0_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         }
         const int lim = kb.full ? BN : col_limit(kb, row, BN);
+        const int lo = kb.full ? 0 : col_lo(kb, row, BN);
         float mt = -CUDART_INF_F;
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
-            x[c] = (c < lim) ? x[c] * p.scale_log2 : -CUDART_INF_F;
+            x[c] = (c >= lo && c < lim) ? x[c] * p.scale_log2 : -CUDART_INF_F;
             mt = fmaxf(mt, x[c]);
         }
-        float m_new = fmaxf(m_run, mt);
-        if (m_new == -CUDART_INF_F) m_new = 0.f;  // a row with nothing visible yet
+        // a row with nothing visible yet (possible under a sliding window) keeps
+        // a finite floor, so that the first visible key rescales by exactly 0
+        const float m_new = fmaxf(fmaxf(m_run, mt), -1e30f);
         const float alpha = ex2(m_run - m_new);
         float sum = 0.f;
         {
@@ -203,7 +206,7 @@ prefill_fwd_v0_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         l_run = l_run * alpha + sum;
         m_run = m_new;
-        if (j > 0) {
+        if (j > j0) {
             uint32_t r[32];
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
@@ -223,7 +226,7 @@ prefill_fwd_v0_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
                 mma_ts(tO, tS + kk * 8, smem_desc_sw128(sV + kk * 2048, CHUNK_BYTES, 1024), IDESC_PV,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+                       (j > j0 || kk > 0) ? 1u : 0u);
             tc_commit(bar_mma);
         }
         ok = __syncthreads_and(mbar_wait(bar_mma, ph_mma));

@@ -77,6 +77,15 @@ class Workload:
         """2*s^2*head_dim*n_head per sequence: the causal half of 4*s^2*d*H."""
         return float(sum(2.0 * s * s * self.head_dim * self.n_head for s in self.seqlens))
 
+    def window_flops(self, window: int) -> float:
+        """4*head_dim*n_head per visible (query, key) pair under a sliding window
+        of ``window`` keys: row a of a sequence sees min(a + 1, window) keys."""
+        pairs = 0
+        for s in self.seqlens:
+            w = min(s, window)
+            pairs += w * (w + 1) // 2 + (s - w) * window
+        return 4.0 * self.head_dim * self.n_head * pairs
+
 
 def _bf16_randn(gen: torch.Generator, shape) -> torch.Tensor:
     return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)

@@ -151,6 +151,34 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
                          int32_t *status_dev, prefill_stream_t stream);
 
 /*
+ * prefill_attn_sliding_window -- causal prefill with a sliding window
+ * (lnwmold.com/news/496245 §4.1: each token attends only to its nearest W
+ * predecessors, so n rows cost n*W instead of n^2 key visits).  Row a of
+ * sequence i, at absolute position P = context_lens[i] + a, sees keys
+ * max(0, P - window + 1) .. P: the window counts the token itself, and
+ * window >= P + 1 for every row gives plain causal attention.  The KV write is
+ * the same as for prefill_attn: every token of the call lands in its slot,
+ * whether or not later rows still see it.
+ *
+ *   context_lens   device int32 [num_seqs] (chunked prefill: the window
+ *                  reaches back into the cached prefix, and prefix blocks
+ *                  wholly before it are not read), or NULL for plain prefill
+ *                  (then max_context_len must be 0)
+ *   window         keys per row, >= 1
+ *   the rest as for prefill_attn_chunked.
+ * Errors as for prefill_attn_chunked, plus PREFILL_ERR_SHAPE for window < 1 or
+ * a non-zero max_context_len without context_lens.
+ */
+int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                                int total_q, const int32_t *cu_seqlens_q, const int32_t *context_lens,
+                                int num_seqs, int max_q_len, int max_context_len,
+                                int n_head, int n_kv_head, int head_dim, float scale, int window,
+                                prefill_bf16 *out,
+                                prefill_bf16 *kv_cache, int num_blocks,
+                                const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                                int32_t *status_dev, prefill_stream_t stream);
+
+/*
  * prefill_attn_chunked_noalloc -- prefill_attn_chunked for callers that cannot
  * allocate device memory.  The pages have no counterpart: this is a deployment
  * variant of the chunked call, not a step of the method.
@@ -220,10 +248,19 @@ const char *prefill_status_string(int status);
  * masked block it writes, for each row r of the query block, the number of
  * leading visible key columns to col_limit[r] (bm entries; may be NULL).
  * Its key range starts at absolute position *key_begin (may be NULL).
+ *
+ * Under a sliding window of `window` keys (window 0: none) the visit starts
+ * at prefill_first_kv_block() instead of 0 (blocks wholly before the first
+ * row's window are not issued), and prefill_kv_block_rule_window also writes
+ * each row's first visible column to col_lo[r]: row r sees the columns
+ * [col_lo[r], col_limit[r]) of block j.  Both return values as above.
  */
 int prefill_num_kv_blocks(int qb, int ctx, int n, int bm, int bn);
 int prefill_kv_block_rule(int qb, int j, int ctx, int n, int bm, int bn,
                           int32_t *col_limit, int32_t *key_begin);
+int prefill_first_kv_block(int qb, int ctx, int n, int bm, int bn, int window);
+int prefill_kv_block_rule_window(int qb, int j, int ctx, int n, int bm, int bn, int window,
+                                 int32_t *col_lo, int32_t *col_limit, int32_t *key_begin);
 
 #ifdef __cplusplus
 }

@@ -123,3 +123,76 @@ def test_block_rule_matches_brute_force_mask(lib, bm, bn):
             assert _lib.kv_block_rule(qb, nkv, ctx, n, bm, bn)[0] == -1
         # every visible pair is covered by exactly one issued block; no invisible pair is
         assert np.array_equal(covered, vis.astype(np.int32)), (ctx, n)
+
+
+# ---------------------------------------------------------------- block rule under a sliding window
+def _brute_band(ctx, n, window):
+    """visible[a, p]: chunk row a (absolute position ctx + a) sees key p iff
+    ctx + a - window < p <= ctx + a."""
+    a = np.arange(n)[:, None]
+    p = np.arange(ctx + n)[None, :]
+    return (p <= ctx + a) & (p > ctx + a - window)
+
+
+@pytest.mark.parametrize("bm,bn", [(128, 128), (64, 64), (128, 64)])
+def test_window_block_rule_matches_brute_force_band(lib, bm, bn):
+    rng = np.random.default_rng(6)
+    cases = [(0, 300, w) for w in (1, 2, 63, 64, 65, 127, 128, 129, 200, 299, 300, 1000)]
+    cases += [(200, 300, w) for w in (1, 50, 128, 201, 260, 500)]
+    cases += [(int(c), int(n), int(w)) for c, n, w in
+              zip(rng.integers(0, 500, 40), rng.integers(1, 400, 40), rng.integers(1, 600, 40))]
+    for ctx, n, window in cases:
+        vis = _brute_band(ctx, n, window)
+        covered = np.zeros_like(vis, dtype=np.int32)
+        for qb in range(-(-n // bm)):
+            rows = np.arange(qb * bm, min(qb * bm + bm, n))
+            nkv = _lib.num_kv_blocks(qb, ctx, n, bm, bn)
+            first = _lib.first_kv_block(qb, ctx, n, window, bm, bn)
+            assert 0 <= first < nkv
+            for j in range(first, nkv):
+                kind, lo, lim, kb = _lib.kv_block_rule_window(qb, j, ctx, n, window, bm, bn)
+                assert kind in (0, 1)
+                any_visible = False
+                for a in rows:
+                    r = a - qb * bm
+                    cols = kb + np.arange(bn)
+                    in_range = cols < ctx + n
+                    want = np.zeros(bn, dtype=bool)
+                    want[in_range] = vis[a, cols[in_range]]
+                    if j < -(-ctx // bn):
+                        want &= cols < ctx
+                    got = (np.arange(bn) >= lo[r]) & (np.arange(bn) < lim[r])
+                    assert np.array_equal(got, want), (ctx, n, window, qb, j, a)
+                    if kind == 0:
+                        assert want.all()
+                    any_visible |= bool(want.any())
+                    covered[a, cols[got]] += 1
+                if j == first:
+                    assert any_visible, "the first issued block holds a visible pair"
+            assert _lib.kv_block_rule_window(qb, first - 1, ctx, n, window, bm, bn)[0] == -1 or first == 0
+            assert _lib.kv_block_rule_window(qb, nkv, ctx, n, window, bm, bn)[0] == -1
+        assert np.array_equal(covered, vis.astype(np.int32)), (ctx, n, window)
+
+
+def test_window_start_of_query_block_pair(lib):
+    """Query block 1 of a pair starts at most two kv blocks after query block 0
+    (the split-KV schedule relies on it)."""
+    for ctx in range(0, 700, 7):
+        for n in (129, 256, 300, 700):
+            for window in (1, 5, 100, 128, 129, 333, 700):
+                for qb in range(0, -(-n // 128) - 1):
+                    f0 = _lib.first_kv_block(qb, ctx, n, window)
+                    f1 = _lib.first_kv_block(qb + 1, ctx, n, window)
+                    assert f0 <= f1 <= f0 + 2, (ctx, n, window, qb)
+
+
+def test_window_validation(lib):
+    import ctypes
+    P = ctypes.c_void_p(16)
+    base = [P, P, P, 1, P, None, 1, 1, 0, 4, 4, 64, 0.125]
+    tail = [P, P, 8, P, 8, 16, None, None]
+    assert lib.prefill_attn_sliding_window(*base, 0, *tail) == 2     # window < 1
+    assert lib.prefill_attn_sliding_window(*base, -3, *tail) == 2
+    with_ctx = list(base)
+    with_ctx[8] = 5                                                     # max_context_len without context_lens
+    assert lib.prefill_attn_sliding_window(*with_ctx, 4, *tail) == 2
