@@ -316,9 +316,12 @@ __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
 //   start[c] sequences with more than c pairs          (= first sorted slot of bucket c)
 //   B[c]     items of sequences with more than c pairs (= first item of bucket c)
 //   perm     sequence indices sorted by pair count, descending, stable
-// kWin: the kernel runs a sliding window (p.window keys); without it every
-// window term folds away at compile time.
-template <bool kWin>
+// The kernel is compiled per mode: kWin runs a sliding window (p.window
+// keys), kChunk reads a cached prefix (p.context_lens).  Without them every
+// window term, and every prefix branch (the context is the constant 0), folds
+// away at compile time.
+constexpr int kModeWindow = 1, kModeChunk = 2;
+template <bool kWin, bool kChunk>
 __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, const int *start, const uint16_t *perm,
                                             int P, int u_split) {
     const int u = u_split / p.nsplit;
@@ -341,7 +344,7 @@ __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, co
     it.qb0 = 2 * (c - 1 - pw);
     it.c0 = p.cu_seqlens[it.i];
     it.n = p.cu_seqlens[it.i + 1] - it.c0;
-    it.ctx = p.context_lens ? p.context_lens[it.i] : 0;
+    it.ctx = kChunk ? p.context_lens[it.i] : 0;
     it.two = (it.qb0 + 1) * BM < it.n;
     it.nk0 = num_kv_blocks(it.qb0, it.ctx, it.n, BM, BN);
     it.nk1 = it.two ? num_kv_blocks(it.qb0 + 1, it.ctx, it.n, BM, BN) : 0;
@@ -384,12 +387,13 @@ __device__ __forceinline__ void setmaxnreg_softmax() { asm volatile("setmaxnreg.
 __device__ __forceinline__ void setmaxnreg_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
 
 // ------------------------------------------------------------------ kernel
-template <int D, int NST, bool kWin>
+template <int D, int NST, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_cache,
                    const FwdParams p, const int P) {
     using L = Lay<D, NST>;
+    constexpr bool kWin = (MODE & kModeWindow) != 0, kChunk = (MODE & kModeChunk) != 0;
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
 
@@ -509,7 +513,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int k = 0; ok; ++k) {
             const int u = zigzag(k, cta, G);
             if (u >= total) break;
-            const Item it = decode_item<kWin>(p, B, start, perm, P, u);
+            const Item it = decode_item<kWin, kChunk>(p, B, start, perm, P, u);
             if (it.skip || (s == 1 && !it.two)) continue;
             const int qb = it.qb0 + s;
             const int jb = kWin ? it.beg(s) : it.j_lo, je = it.end(s);
@@ -602,7 +606,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item<kWin>(p, B, start, perm, P, u);
+                const Item it = decode_item<kWin, kChunk>(p, B, start, perm, P, u);
                 if (it.skip) continue;
                 const int ns = it.two ? 2 : 1;
                 for (int s = 0; s < ns; ++s) {
@@ -621,8 +625,25 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tma_load_4d(base + (s ? L::Q1 : L::Q0), &tm_q, b, 0, it.h, it.c0 + (it.qb0 + s) * BM, 0);
                     }
                 }
+                // Prefix blocks: lane x < (whole pages) * NCH issues the box of page
+                // x / NCH, chunk x % NCH (bs >= 16, so at most 16 boxes per block).
+                // Its page number is read one block ahead, so that the block-table
+                // load overlaps the previous block's copies, and serves both K and V.
+                auto lane_page = [&](int jj) -> int {
+                    const KvBlock kk = kv_block(it.qb0, jj, it.ctx, it.n, BM, BN, 0);
+                    if (!kk.prefix || lane >= (kk.lim_const / bs) * L::NCH) return 0;
+                    return __ldg(&p.block_table[(size_t)it.i * p.mbps + kk.key_begin / bs + lane / L::NCH]);
+                };
+                const int np = cdiv(it.ctx, BN);  // prefix blocks come first
+                int page_next = it.j_lo < np ? lane_page(it.j_lo) : 0;
                 for (int j = it.j_lo; j < it.j_hi && ok; ++j) {
                     const KvBlock kb = kv_block(it.qb0, j, it.ctx, it.n, BM, BN, 0);  // key range only
+                    int page_cur = page_next;
+                    if (j + 1 < it.j_hi && j + 1 < np) page_next = lane_page(j + 1);
+                    if (page_cur < 0 || page_cur >= p.num_blocks) {
+                        report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                        page_cur = p.num_blocks;  // outside the map: the box reads zeros
+                    }
                     for (int t = 0; t < 2; ++t) {  // t = 0: K, t = 1: V
                         if (!wait_bar(bar(L::B_KVEMPTY + stage), phase ^ 1, abort)) { ok = false; break; }
                         const uint32_t dst = base + L::KV + stage * L::TILE;
@@ -669,15 +690,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             // ~300 clocks per TMA issue, lanes issuing together overlap it
                             if (lane == 0) mbar_expect_tx(b, (uint32_t)(full_pages * bs * 128 * L::NCH));
                             __syncwarp();
-                            for (int x = lane; x < full_pages * L::NCH; x += 32) {
-                                const int pg = x / L::NCH, ch = x % L::NCH;
-                                int page = p.block_table[(size_t)it.i * p.mbps + kb.key_begin / bs + pg];
-                                if (page < 0 || page >= p.num_blocks) {
-                                    report(p.status, PREFILL_ERR_BLOCK_TABLE);
-                                    page = p.num_blocks;  // outside the map: zero fill
-                                }
+                            if (lane < full_pages * L::NCH) {
+                                const int pg = lane / L::NCH, ch = lane % L::NCH;
                                 tma_load_4d(dst + ch * CHUNK + pg * bs * 128, &tm_cache, b, ch * 64, it.g, 0,
-                                            page * 2 + t);
+                                            page_cur * 2 + t);
                             }
                         }
                         if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -724,7 +740,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item<kWin>(p, B, start, perm, P, u);
+                const Item it = decode_item<kWin, kChunk>(p, B, start, perm, P, u);
                 if (it.skip) continue;
                 const int ns = it.two ? 2 : 1;
                 const int j0 = it.j_lo, jend = it.j_hi;
@@ -815,7 +831,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int k = 0; ok; ++k) {
                 const int u = zigzag(k, cta, G);
                 if (u >= total) break;
-                const Item it = decode_item<kWin>(p, B, start, perm, P, u);
+                const Item it = decode_item<kWin, kChunk>(p, B, start, perm, P, u);
                 if (it.skip) continue;
                 const int np = cdiv(it.ctx, BN);
                 const bool writes = (it.h % p.group) == 0;
@@ -978,17 +994,17 @@ int sm_count() {
     return n;
 }
 
-template <int D, int NST, bool kWin>
+template <int D, int NST, int MODE>
 int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
     const size_t smem = smem_bytes<D, NST>(P, p.num_seqs);
-    cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D, NST, kWin>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D, NST, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     const long long items_bound = (long long)p.num_seqs * p.n_head * P;
     const long long items = items_bound * (p.nsplit > 0 ? p.nsplit : 1);
     const int grid_s = (int)(items < sm_count() ? items : sm_count());
-    prefill_fwd_kernel<D, NST, kWin><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v,
+    prefill_fwd_kernel<D, NST, MODE><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v,
                                                                                         maps.cache, p, P);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
@@ -1000,8 +1016,13 @@ template <int D>
 int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
     const bool nst5 = smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem;
-    if (p.window > 0) return nst5 ? launch_nst<D, 5, true>(maps, p, stream) : launch_nst<D, 4, true>(maps, p, stream);
-    return nst5 ? launch_nst<D, 5, false>(maps, p, stream) : launch_nst<D, 4, false>(maps, p, stream);
+    const int mode = (p.window > 0 ? kModeWindow : 0) | (p.context_lens ? kModeChunk : 0);
+    switch (mode) {
+        case 0: return nst5 ? launch_nst<D, 5, 0>(maps, p, stream) : launch_nst<D, 4, 0>(maps, p, stream);
+        case 1: return nst5 ? launch_nst<D, 5, 1>(maps, p, stream) : launch_nst<D, 4, 1>(maps, p, stream);
+        case 2: return nst5 ? launch_nst<D, 5, 2>(maps, p, stream) : launch_nst<D, 4, 2>(maps, p, stream);
+        default: return nst5 ? launch_nst<D, 5, 3>(maps, p, stream) : launch_nst<D, 4, 3>(maps, p, stream);
+    }
 }
 
 }  // namespace
