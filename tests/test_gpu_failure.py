@@ -45,3 +45,30 @@ def test_hook_resets_after_one_launch():
     _, _, st1 = U.run_prefill(w)
     _, _, st2 = U.run_prefill(w)
     assert st1 == 6 and st2 == 0
+
+
+def test_stalled_split_call_leaves_no_stale_merge_state():
+    """A chunked call whose kv ranges are split (merged in-kernel by the split
+    that finishes last) is stalled, so some splits never arrive at their merge
+    counters; the next identical call must still merge every row correctly."""
+    ctx, L, H, G, d, bs = 3000, 300, 8, 2, 128, 16
+    full = W.make_workload([ctx + L], H, G, d, block_size=bs, seed=63, extra_pages=2)
+    cache = oracle.kv_write(full.k[:ctx], full.v[:ctx], torch.tensor([0, ctx], dtype=torch.int32),
+                            full.empty_cache(), full.block_table, bs)
+    q, k, v = (x[ctx:].contiguous() for x in (full.q, full.k, full.v))
+    cu = torch.tensor([0, L], dtype=torch.int32)
+    ctxs = torch.tensor([ctx], dtype=torch.int32)
+    ref_out = oracle.attention(q, k, v, cu, H, G, d, full.scale, context_lens=ctxs, kv_cache=cache,
+                               block_table=full.block_table, block_size=bs)
+    dev = [x.cuda() for x in (q, k, v, cu, ctxs, full.block_table)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for stall in (True, False):
+        cache_d = cache.cuda()
+        out = torch.full(dev[0].shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+        status.zero_()
+        _lib.inject_stall(stall)
+        _lib.prefill_attn_chunked(dev[0], dev[1], dev[2], dev[3], dev[4], L, ctx, full.scale, out, cache_d, dev[5],
+                                  status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == (6 if stall else 0)
+    U.compare_out(out.cpu(), ref_out, "split call after a stalled split call")
