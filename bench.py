@@ -187,6 +187,50 @@ class WindowRunner(PlainRunner):
 WINDOW_LINE = ("swa4096_gqa_s8192_h32g8_d128", "gqa_s8192_h32g8_d128", 4096)
 
 
+class DecodeRunner:
+    """One decode step (paged_decode_attn) for the 64 sequences of the varlen
+    workload: their prompts are prefilled once by prefill_attn (which writes the
+    paged cache), then each sequence's next token attends to its prompt and
+    itself.  Bound by HBM: the algorithmic bytes are the cached K/V read once,
+    the new tokens' q/k/v, the output and the appended K/V."""
+
+    def __init__(self, base: W.Workload, seed: int, stream):
+        w = W.make_workload([n + 1 for n in base.seqlens], base.n_head, base.n_kv_head, base.head_dim,
+                            block_size=base.block_size, seed=seed)
+        pq, pk, pv, pcu, q, k, v, ctx = W.decode_views(w)
+        d = torch.device("cuda")
+        self.w, self.stream = w, stream
+        self.cache = w.empty_cache().to(d)
+        self.bt = w.block_table.to(d)
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+        pout = torch.empty(pq.shape, dtype=torch.bfloat16, device=d)
+        _lib.prefill_attn(pq.to(d), pk.to(d), pv.to(d), pcu.to(d), int(ctx.max()), w.scale, pout, self.cache, self.bt,
+                          status=self.status, stream=stream)
+        del pout
+        self.q, self.k, self.v, self.ctx = q.to(d), k.to(d), v.to(d), ctx.to(d)
+        self.max_ctx = int(ctx.max())
+        self.out = torch.empty_like(self.q)
+        B, H, G, D = len(w.seqlens), w.n_head, w.n_kv_head, w.head_dim
+        self.bytes = (int(ctx.sum()) * G * D * 2 * 2        # cached K and V, read once
+                      + B * H * D * 2 * 2                   # q in, out
+                      + B * G * D * 2 * 2 * 2)              # new k, v in and into the cache
+        self.launches = 2 if -(-(self.max_ctx + 1) // 512) > 1 else 1
+        self.tokens = B
+
+    def step(self):
+        _lib.paged_decode_attn(self.q, self.k, self.v, self.ctx, self.max_ctx, self.w.scale, self.out, self.cache,
+                               self.bt, status=self.status, stream=self.stream)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
+
+
+# secondary line: one decode step after the 64 prompts of the varlen workload
+DECODE_LINE = ("decode64_gqa_h32g8_d128", "varlen64_gqa_h32g8_d128", 2001)
+
+
 def time_steps(runner, steps, warmup, stream, flush):
     for _ in range(warmup):
         runner.step()
@@ -364,6 +408,16 @@ def main():
                        "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches,
                        "window": win}
         del rx, wx
+        torch.cuda.empty_cache()
+        name, base, seed = DECODE_LINE
+        rx = DecodeRunner(W.named_workload(base), seed, stream)
+        dx = time_steps(rx, max(10, args.steps), 3, stream, flush)
+        mx = statistics.median(dx)
+        extra[name] = {"ms": round(mx, 4), "gbs": round(rx.bytes / (mx * 1e-3) / 1e9, 1),
+                       "frac_of_hbm": round(rx.bytes / (mx * 1e-3) / 1e9 / pk["hbm"], 4),
+                       "bytes_per_step": rx.bytes, "tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
+                       "launches": rx.launches}
+        del rx
         torch.cuda.empty_cache()
 
     cpu = None

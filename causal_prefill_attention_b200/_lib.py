@@ -22,7 +22,8 @@ STATUS_NAMES = {
 EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall",
             "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
-            "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window")
+            "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window",
+            "paged_decode_attn")
 
 _lib = None
 
@@ -63,6 +64,8 @@ def load() -> ctypes.CDLL:
         lib.prefill_first_kv_block.restype = I
         lib.prefill_kv_block_rule_window.argtypes = [I, I, I, I, I, I, I, P, P, P]
         lib.prefill_kv_block_rule_window.restype = I
+        lib.paged_decode_attn.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, I, P, I, I, P, P]
+        lib.paged_decode_attn.restype = I
         _lib = lib
     return _lib
 
@@ -181,6 +184,26 @@ def prefill_attn_sliding_window(q, k, v, cu_seqlens_q, context_lens, max_q_len: 
         _ptr(status), _stream_ptr(stream))
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "prefill_attn_sliding_window")
+    return rc
+
+
+def paged_decode_attn(q, k, v, context_lens, max_context_len: int, scale: float, out, kv_cache, block_table,
+                      status: Optional[torch.Tensor] = None, stream=None, raise_on_error: bool = True) -> int:
+    """Decode step over the paged cache (C ABI ``paged_decode_attn``): the new
+    token of each sequence (q [B, n_head, d], k/v [B, n_kv_head, d]) attends to
+    its ``context_lens[i]`` cached tokens and itself; its K/V are appended."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3)
+    _check_bf16("out", out, 3), _check_bf16("kv_cache", kv_cache, 5)
+    _check_i32("context_lens", context_lens), _check_i32("block_table", block_table)
+    B, H, D = q.shape
+    G = k.shape[1]
+    rc = load().paged_decode_attn(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(context_lens), B, int(max_context_len), H, G, D, float(scale), _ptr(out),
+        _ptr(kv_cache), kv_cache.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "paged_decode_attn")
     return rc
 
 

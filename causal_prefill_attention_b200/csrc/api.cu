@@ -15,6 +15,7 @@
 
 #include "../../include/prefill.h"
 #include "block_rule.h"
+#include "decode.h"
 #include "params.h"
 
 namespace {
@@ -229,6 +230,59 @@ int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, co
                            max_q_len, max_context_len, n_head, n_kv_head, head_dim, scale, out, kv_cache,
                            num_blocks, block_table, max_blocks_per_seq, block_size, status_dev, stream, nullptr, 0,
                            window);
+}
+
+int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                      const int32_t *context_lens, int num_seqs, int max_context_len, int n_head, int n_kv_head,
+                      int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks,
+                      const int32_t *block_table, int max_blocks_per_seq, int block_size, int32_t *status_dev,
+                      prefill_stream_t stream) {
+    if (!q || !k || !v || !context_lens || !out || !kv_cache || !block_table) return PREFILL_ERR_NULL;
+    if (num_seqs < 0 || max_context_len < 0) return PREFILL_ERR_SHAPE;
+    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
+    if (n_head / n_kv_head > 8) return PREFILL_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (!(std::isfinite(scale) && scale > 0.f)) return PREFILL_ERR_UNSUPPORTED;
+    if (num_blocks < 1 || max_blocks_per_seq < 1) return PREFILL_ERR_BLOCK_TABLE;
+    if ((long long)max_context_len + 1 > (long long)max_blocks_per_seq * block_size) return PREFILL_ERR_BLOCK_TABLE;
+    if (num_seqs > 65535 || n_kv_head > 65535) return PREFILL_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * 2 * block_size * n_kv_head * head_dim > (1ll << 40)) return PREFILL_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kv_cache))
+        return PREFILL_ERR_ALIGNMENT;
+    if (num_seqs == 0) return PREFILL_OK;
+
+    pf::DecodeParams p;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.out = out;
+    p.cache = kv_cache;
+    p.context_lens = context_lens;
+    p.block_table = block_table;
+    p.status = status_dev;
+    p.num_seqs = num_seqs;
+    p.n_head = n_head;
+    p.n_kv_head = n_kv_head;
+    p.num_blocks = num_blocks;
+    p.mbps = max_blocks_per_seq;
+    p.block_size = block_size;
+    p.max_ctx = max_context_len;
+    p.keys_per_unit = pf::decode_keys_per_unit(max_context_len);
+    p.max_units = pf::cdiv(max_context_len + 1, p.keys_per_unit);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.part_o = nullptr;
+    p.part_ml = nullptr;
+    if (p.max_units > 1) {
+        // partials [max_units][num_seqs][n_head][head_dim + 2] fp32, in the same
+        // per-(device, stream) workspace as the prefill split-KV partials
+        const size_t rows = (size_t)p.max_units * num_seqs * n_head;
+        char *ws = static_cast<char *>(split_workspace(rows * ((size_t)head_dim + 2) * sizeof(float), stream));
+        if (!ws) return PREFILL_ERR_CUDA;
+        p.part_o = reinterpret_cast<float *>(ws);
+        p.part_ml = reinterpret_cast<float *>(ws + rows * head_dim * sizeof(float));
+    }
+    return pf::launch_decode(p, head_dim, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 
 void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }

@@ -1,0 +1,35 @@
+// decode.h -- launch parameters of the paged decode kernels (decode.cu).
+#pragma once
+#include <cstdint>
+
+namespace pf {
+
+// At most this many key splits (work units) per sequence; longer contexts get
+// longer units (decode_keys_per_unit).
+constexpr int kDecodeMaxUnits = 64;
+
+struct DecodeParams {
+    const uint16_t *q;            // [B][n_head][D]   the new token's queries
+    const uint16_t *k;            // [B][n_kv_head][D] its keys
+    const uint16_t *v;            // [B][n_kv_head][D] its values
+    uint16_t *out;                // [B][n_head][D]
+    uint16_t *cache;              // [NB][2][bs][n_kv_head][D]
+    const int32_t *context_lens;  // [B] cached tokens before the new one
+    const int32_t *block_table;   // [B][mbps]
+    int32_t *status;              // nullable
+    int num_seqs, n_head, n_kv_head;
+    int num_blocks, mbps, block_size;
+    int max_ctx;                  // bound on every context length (sizes the grid)
+    int keys_per_unit;            // keys per work unit (a multiple of the 64-key tile)
+    int max_units;                // cdiv(max_ctx + 1, keys_per_unit)
+    float scale_log2;             // scale * log2(e)
+    // units' partials when a sequence has more than one unit:
+    // part_o [max_units][B][n_head][D] (fp32, unnormalised), part_ml [..][2] (max in log2 units, sum)
+    float *part_o;
+    float *part_ml;
+};
+
+int decode_keys_per_unit(int max_ctx);
+int launch_decode(const DecodeParams &p, int head_dim, void *stream);
+
+}  // namespace pf

@@ -181,3 +181,26 @@ def chunk_views(w: Workload, chunk: int, seq: int = 0):
         sl = slice(start + c0, start + c0 + L)
         yield (w.q[sl].contiguous(), w.k[sl].contiguous(), w.v[sl].contiguous(),
                torch.tensor([0, L], dtype=torch.int32), torch.tensor([c0], dtype=torch.int32), bt)
+
+
+def decode_views(w: Workload):
+    """Split every sequence of ``w`` into its prompt (all tokens but the last)
+    and one decode token (the last).
+
+    Returns (prompt_q, prompt_k, prompt_v, prompt_cu_seqlens, new_q, new_k,
+    new_v, context_lens): the packed prompts, whose K/V a prefill call writes
+    into the cache, and for each sequence the last token's q [B, H, d] and
+    k, v [B, G, d] with its position (= its prompt length).  Every sequence
+    needs at least one token; ``w``'s block table then has a page for the
+    decode token's slot.
+    """
+    lens = [int(s) for s in w.seqlens]
+    assert all(n >= 1 for n in lens), "every sequence needs its decode token"
+    starts = w.cu_seqlens[:-1].tolist()
+    keep = torch.cat([torch.arange(s, s + n - 1) for s, n in zip(starts, lens)]) if lens else torch.zeros(0, dtype=torch.long)
+    last = torch.tensor([s + n - 1 for s, n in zip(starts, lens)], dtype=torch.long)
+    ctx = torch.tensor([n - 1 for n in lens], dtype=torch.int32)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(ctx.to(torch.int64), 0).to(torch.int32)
+    return (w.q[keep].contiguous(), w.k[keep].contiguous(), w.v[keep].contiguous(), cu,
+            w.q[last].contiguous(), w.k[last].contiguous(), w.v[last].contiguous(), ctx)

@@ -179,6 +179,39 @@ int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, co
                                 int32_t *status_dev, prefill_stream_t stream);
 
 /*
+ * paged_decode_attn -- decode attention over the paged cache (the next step
+ * after prefill: hncyxsy.com/news/270449 §1.1, decode feeds only the token
+ * generated last; hncyxsy.com/news/227904 §1, the step is then bound by
+ * memory bandwidth, reading the KV cache).  For each sequence i, the one new
+ * token at absolute position context_lens[i] attends to the context_lens[i]
+ * cached tokens (gathered through block_table) and to itself; its K/V are then
+ * written to their slot.  The result equals prefill_attn_chunked with one-row
+ * chunks.
+ *
+ *   q              device bf16 [num_seqs][n_head][head_dim]: the new tokens' queries
+ *   k, v           device bf16 [num_seqs][n_kv_head][head_dim]: their keys and values
+ *   context_lens   device int32 [num_seqs]: cached tokens before each new one
+ *   max_context_len  upper bound on every context length (host; sizes the grid)
+ *   out            device, written: [num_seqs][n_head][head_dim] bf16
+ *   kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
+ *   status_dev, stream   as for prefill_attn_chunked.
+ * n_head / n_kv_head must be at most 8 (PREFILL_ERR_UNSUPPORTED otherwise).
+ * Requires max_context_len + 1 <= max_blocks_per_seq * block_size.  A sequence
+ * whose context length is negative or above max_context_len is skipped and
+ * reported as PREFILL_ERR_SHAPE.  Long contexts are split into units of >= 512
+ * keys whose partial results a second kernel merges; their partials use the
+ * same per-(device, stream) workspace as the prefill split-KV partials
+ * (max units x num_seqs x n_head x (head_dim + 2) x 4 bytes).
+ */
+int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                      const int32_t *context_lens, int num_seqs, int max_context_len,
+                      int n_head, int n_kv_head, int head_dim, float scale,
+                      prefill_bf16 *out,
+                      prefill_bf16 *kv_cache, int num_blocks,
+                      const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                      int32_t *status_dev, prefill_stream_t stream);
+
+/*
  * prefill_attn_chunked_noalloc -- prefill_attn_chunked for callers that cannot
  * allocate device memory.  The pages have no counterpart: this is a deployment
  * variant of the chunked call, not a step of the method.

@@ -23,12 +23,13 @@ def lib():
 def _declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(prefill_[a-z_0-9]+)\s*\(", src, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged)_[a-z_0-9]+)\s*\(", src,
+                                 flags=re.M)))
 
 
 def test_every_declared_symbol_is_exported(lib):
     names = _declared_functions()
-    assert "prefill_attn" in names and "prefill_attn_chunked" in names
+    assert "prefill_attn" in names and "prefill_attn_chunked" in names and "paged_decode_attn" in names
     for name in names:
         assert hasattr(lib, name), name
     assert set(_lib.EXPORTED) <= set(names)
@@ -196,3 +197,25 @@ def test_window_validation(lib):
     with_ctx = list(base)
     with_ctx[8] = 5                                                     # max_context_len without context_lens
     assert lib.prefill_attn_sliding_window(*with_ctx, 4, *tail) == 2
+
+
+def test_decode_validation(lib):
+    P = ctypes.c_void_p(FAKE)
+    #        q  k  v  ctx B  maxc H  G  D    scale  out cache nb bt mbps bs  status stream
+    base = [P, P, P, P, 2, 100, 8, 2, 128, 0.088, P, P, 16, P, 8, 16, None, None]
+
+    def call(**over):
+        a = list(base)
+        names = ["q", "k", "v", "ctx", "B", "maxc", "H", "G", "D", "scale", "out", "cache", "nb", "bt", "mbps", "bs"]
+        for key, val in over.items():
+            a[names.index(key)] = val
+        return lib.paged_decode_attn(*a)
+
+    assert call(q=None) == 1 and call(ctx=None) == 1 and call(bt=None) == 1
+    assert call(H=9, G=2) == 2
+    assert call(H=18, G=2) == 3            # 9 query heads per kv head: above 8
+    assert call(D=96) == 3 and call(bs=24) == 3 and call(scale=0.0) == 3
+    assert call(maxc=128) == 4             # 129 keys do not fit 8 pages of 16
+    assert call(nb=0) == 4
+    assert call(q=ctypes.c_void_p(FAKE + 4)) == 7
+    assert call(B=0) == 0
