@@ -240,13 +240,13 @@ int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefil
     if (!q || !k || !v || !context_lens || !out || !kv_cache || !block_table) return PREFILL_ERR_NULL;
     if (num_seqs < 0 || max_context_len < 0) return PREFILL_ERR_SHAPE;
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
-    if (n_head / n_kv_head > 8) return PREFILL_ERR_UNSUPPORTED;
+    if (n_head / n_kv_head > 16) return PREFILL_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
     if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return PREFILL_ERR_UNSUPPORTED;
     if (!(std::isfinite(scale) && scale > 0.f)) return PREFILL_ERR_UNSUPPORTED;
     if (num_blocks < 1 || max_blocks_per_seq < 1) return PREFILL_ERR_BLOCK_TABLE;
     if ((long long)max_context_len + 1 > (long long)max_blocks_per_seq * block_size) return PREFILL_ERR_BLOCK_TABLE;
-    if (num_seqs > 65535 || n_kv_head > 65535) return PREFILL_ERR_UNSUPPORTED;
+    if (num_seqs > pf::kDecodeMaxSeqs || n_kv_head > 65535) return PREFILL_ERR_UNSUPPORTED;
     if ((long long)num_blocks * 2 * block_size * n_kv_head * head_dim > (1ll << 40)) return PREFILL_ERR_SHAPE;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kv_cache))
         return PREFILL_ERR_ALIGNMENT;

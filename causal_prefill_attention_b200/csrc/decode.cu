@@ -7,21 +7,31 @@
 // and the step is bound by memory bandwidth, i.e. by reading the KV cache.
 // The result equals a chunked prefill call with one-row chunks.
 //
-// Design (HBM-bound; CUDA cores, no tensor cores: a query block here has
-// n_head / n_kv_head rows):
-//  * work unit = (sequence, kv head, split of keys_per_unit keys); the r query
-//    heads of the kv head share every K/V byte read;
-//  * 64-key K and V tiles are gathered page by page with cp.async (16 bytes per
-//    copy, zero fill past the end) into a 3-stage ring, rows 128-byte
-//    swizzled so that both the key-parallel and the column-parallel reads
-//    below are free of bank conflicts; page numbers are read one tile ahead;
-//  * scores: thread = (key, quarter of head_dim), partial dots for the r heads,
-//    summed per key; online softmax: warp h owns head h (running max and sum);
-//    P.V: thread = (pair of columns, group of keys), r x 2 accumulators;
+// Design (HBM-bound):
+//  * work unit = (sequence, kv head, split of keys_per_unit keys); the r <= 16
+//    query heads of the kv head share every K/V byte read;
+//  * every warp is an independent persistent worker: it takes the call's units
+//    round robin (numbered densely through an exclusive scan of the units per
+//    sequence, so every warp gets the same number of keys within one unit) and
+//    streams them, 16 keys per step, through its own 3-stage ring
+//    (cp.async, 16 bytes per copy, zero fill past the end), across unit
+//    boundaries, so its loads never stop between units; a step lies in one
+//    cache page (pages hold a multiple of 16 tokens), so one page-table read
+//    per step, made one step ahead.  No CTA-wide barrier after the start;
+//  * Q K^T and P V on warp-level tensor-core MMAs (m16n8k16, bf16 in, fp32
+//    out): the query heads are the 16 rows of the A operand, the scores'
+//    accumulators are the A operand of P V without leaving registers, O stays
+//    in registers (16 rows x head_dim over the warp).  Rows >= r are zero
+//    queries and never written out.  The running max moves only when a block
+//    max exceeds it by 2^8 (as in the prefill kernel), so O is rarely rescaled;
 //  * a unit's partial (unnormalised O, max, sum) is merged by
 //    decode_combine_kernel when a sequence has more than one unit.
-// Every wait is a cp.async group wait on the thread's own copies, so nothing
-// can wait forever.
+// Earlier versions for the record: CUDA-core dot products (one FMA per
+// element) issued ~6.5k warp instructions per 64 keys and reached 19 % of the
+// DRAM bandwidth; a CTA-wide version with tensor-core MMAs and three barriers
+// per 64-key tile reached 33 %.
+// Every wait is a cp.async group wait on the warp's own copies, so nothing can
+// wait forever.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -36,26 +46,24 @@
 namespace pf {
 namespace {
 
-constexpr int DT = 64;          // keys per tile
-constexpr int DTHREADS = 256;   // 8 warps
-constexpr int DSTAGES = 3;
-constexpr int kParts = DTHREADS / DT;  // head_dim quarters in the score phase
+constexpr int KS = 16;            // keys per step
+constexpr int WARPS = 4;          // warps (workers) per CTA
+constexpr int DTHREADS = 32 * WARPS;
+constexpr int NSTAGE = 3;         // ring stages per warp
+// sequences per call (their context lengths and unit counts live in shared memory)
+constexpr int kCtasPerSm = 2;
+constexpr float kLazyLog2 = 8.0f; // the running max moves when exceeded by 2^8
 
-template <int D, int R>
+template <int D>
 struct DecLay {
-    static constexpr int NCH = D / 64;               // 64-column chunks of a row
-    static constexpr uint32_t CHUNK = DT * 128;      // 64 rows x 128 bytes
-    static constexpr uint32_t TILE = NCH * CHUNK;    // one K or V tile
-    static constexpr uint32_t STAGE = 2 * TILE;      // K then V
-    static constexpr uint32_t Q = DSTAGES * STAGE;   // fp32 [R][D]
-    static constexpr uint32_t SPART = Q + R * D * 4; // fp32 [kParts][DT][R]
-    static constexpr uint32_t P = SPART + kParts * DT * R * 4;  // fp32 [DT][8]
-    static constexpr uint32_t ALPHA = P + DT * 8 * 4;           // fp32 [8]
-    static constexpr uint32_t ML = ALPHA + 8 * 4;               // fp32 [8][2]
-    static constexpr uint32_t BYTES = ML + 8 * 2 * 4;
-    // the final reduction over key groups reuses the ring
-    static constexpr int KG = DTHREADS / (D / 2);               // key groups in P.V
-    static_assert((uint32_t)KG * R * D * 4 <= DSTAGES * STAGE, "reduction buffer must fit the ring");
+    static constexpr uint32_t CHUNK = KS * 128;          // 16 rows x 128 bytes (64 columns)
+    static constexpr uint32_t TILE = (D / 64) * CHUNK;   // one K or V step tile
+    static constexpr uint32_t STAGE = 2 * TILE;          // K then V
+    static constexpr uint32_t WARP_RING = NSTAGE * STAGE;
+    static constexpr uint32_t CTX = WARPS * WARP_RING;   // int32 [kDecodeMaxSeqs]: context lengths
+    static constexpr uint32_t CUM = CTX + kDecodeMaxSeqs * 4;  // int32 [kDecodeMaxSeqs + 1]: units before sequence i
+    static constexpr uint32_t BYTES = CUM + (kDecodeMaxSeqs + 1) * 4;
+    static_assert(kCtasPerSm * (BYTES + 1024) <= 228 * 1024, "the resident CTAs must fit the SM");
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
@@ -66,247 +74,350 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-
-// byte offset of 16-byte slot `s` (0 .. D/8-1) of row `r` inside a K or V tile
-template <int D>
-__device__ __forceinline__ uint32_t slot_off(int r, int s) {
-    return (uint32_t)(s >> 3) * (DT * 128) + (uint32_t)r * 128 + (uint32_t)(((s & 7) ^ (r & 7)) << 4);
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row-major fragment) x B (16x8 bf16, column fragment)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int D, int R>
-__global__ void __launch_bounds__(DTHREADS, 2) paged_decode_kernel(const DecodeParams p) {
-    using L = DecLay<D, R>;
+// byte offset of 16-byte slot `s` (0 .. D/8-1) of row `r` (0 .. 15) in a step tile:
+// 64-column chunks of 16 rows x 128 bytes, slots swizzled by row
+__device__ __forceinline__ uint32_t slot_off(int r, int s) {
+    return (uint32_t)(s >> 3) * (KS * 128) + (uint32_t)r * 128 + (uint32_t)(((s & 7) ^ (r & 7)) << 4);
+}
+
+// A work unit: keys [k0, k1) of sequence i for kv head g (split `split` of
+// the sequence's nunits).  Units are numbered densely, sequence by sequence
+// (then kv head, then split): unit u of the call.
+struct Unit {
+    int u, i, g, split, nunits, ctx, k0, k1, nsteps;
+};
+
+// Unit u (below `total`), found by binary search over the per-sequence
+// cumulative unit counts; false past the end.
+__device__ __forceinline__ bool get_unit(const DecodeParams &p, const int *sctx, const int *scum, int u, int total,
+                                         Unit &o) {
+    if (u >= total) return false;
+    int lo = 0, hi = p.num_seqs - 1;  // last sequence with scum[i] <= u
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (scum[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    const int i = lo, ctx = sctx[i];
+    const int nunits = cdiv(ctx + 1, p.keys_per_unit);  // the cached prefix and the new token
+    const int rem = u - scum[i];
+    o.u = u;
+    o.i = i;
+    o.g = rem / nunits;
+    o.split = rem - o.g * nunits;
+    o.nunits = nunits;
+    o.ctx = ctx;
+    o.k0 = o.split * p.keys_per_unit;
+    o.k1 = min(o.k0 + p.keys_per_unit, ctx + 1);
+    o.nsteps = cdiv(o.k1 - o.k0, KS);
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(const DecodeParams p) {
+    using L = DecLay<D>;
+    constexpr int KSTEPS = D / 16;  // 16-column steps of Q K^T
+    constexpr int NT = D / 8;       // 8-column output tiles
     extern __shared__ __align__(128) uint8_t smem[];
-    const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int split = blockIdx.x, g = blockIdx.y, i = blockIdx.z;
-
-    const int ctx = p.context_lens[i];
-    if (ctx < 0 || ctx > p.max_ctx || (long long)ctx + 1 > (long long)p.mbps * p.block_size) {
-        if (split == 0 && g == 0 && tid == 0) report(p.status, PREFILL_ERR_SHAPE);
-        return;
-    }
-    const int nkeys = ctx + 1;  // the cached prefix and the new token
-    const int nunits = cdiv(nkeys, p.keys_per_unit);
-    if (split >= nunits) return;
-    const int k0 = split * p.keys_per_unit;
-    const int k1 = min(k0 + p.keys_per_unit, nkeys);
-    const int ntiles = cdiv(k1 - k0, DT);
-    const int bs = p.block_size;
-    const int32_t *bt = p.block_table + (size_t)i * p.mbps;
+    const uint32_t ring = smem_u32(smem) + (uint32_t)warp * L::WARP_RING;
+    const int W = gridDim.x * WARPS, worker = blockIdx.x * WARPS + warp;
+    const int bs = p.block_size, r = p.n_head / p.n_kv_head;
     const size_t G = p.n_kv_head;
-    const uint16_t *knew = p.k + ((size_t)i * G + g) * D;
-    const uint16_t *vnew = p.v + ((size_t)i * G + g) * D;
 
-    // the new token's K/V go to its slot (position ctx) in the last unit; no
-    // unit of this call reads that slot from the cache (it reads the inputs)
-    if (split == nunits - 1 && tid < 2 * (D / 8)) {
-        const int page = bt[ctx / bs];
-        if (page >= 0 && page < p.num_blocks) {
-            const int t = tid / (D / 8), s = tid % (D / 8);
-            const uint4 val = reinterpret_cast<const uint4 *>(t ? vnew : knew)[s];
-            uint16_t *dst = p.cache + ((((size_t)page * 2 + t) * bs + ctx % bs) * G + g) * D;
-            reinterpret_cast<uint4 *>(dst)[s] = val;
-        } else {
-            report(p.status, PREFILL_ERR_BLOCK_TABLE);
-        }
-    }
-
-    // queries of the r heads of this kv head, fp32
-    float *sq = reinterpret_cast<float *>(smem + L::Q);
-    for (int x = tid; x < R * D; x += DTHREADS) {
-        const int h = x / D, d = x % D;
-        const uint16_t b = p.q[((size_t)i * p.n_head + (size_t)g * R + h) * D + d];
-        sq[x] = __uint_as_float((uint32_t)b << 16);
-    }
-
-    // ---- loads: thread -> row tid / 4 of the tile, D/32 slots of K and of V
-    constexpr int SPT = D / 32;  // slots per thread per tensor
-    const int lrow = tid >> 2, lq = tid & 3;
-    auto row_page = [&](int tile) -> int {  // page of this thread's row (or -1: not from the cache)
-        const int pos = k0 + tile * DT + lrow;
-        if (pos >= k1 || pos >= ctx) return -1;
-        return __ldg(&bt[pos / bs]);
-    };
-    auto issue = [&](int tile, int page) {
-        if (tile < ntiles) {
-            const int pos = k0 + tile * DT + lrow;
-            const uint32_t st = sbase + (uint32_t)(tile % DSTAGES) * L::STAGE;
-            const uint16_t *src[2] = {knew, vnew};
-            uint32_t bytes = 0;
-            if (pos < k1) {
-                if (pos == ctx) {
-                    bytes = 16;  // the new token: from the inputs
-                } else if (page >= 0 && page < p.num_blocks) {
-                    bytes = 16;
-                    src[0] = p.cache + ((((size_t)page * 2 + 0) * bs + pos % bs) * G + g) * D;
-                    src[1] = p.cache + ((((size_t)page * 2 + 1) * bs + pos % bs) * G + g) * D;
+    // context lengths and an exclusive scan of the units per sequence (n_kv_head
+    // per key split; none for a sequence whose context is out of range, which
+    // is skipped and reported)
+    int *sctx = reinterpret_cast<int *>(smem + L::CTX);
+    int *scum = reinterpret_cast<int *>(smem + L::CUM);
+    __shared__ int s_wsum[WARPS];
+    {
+        constexpr int PER = kDecodeMaxSeqs / DTHREADS;  // sequences per thread
+        int cnt[PER], run = 0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int i = tid * PER + e;
+            int c = 0;
+            if (i < p.num_seqs) {
+                const int ctx = __ldg(&p.context_lens[i]);
+                sctx[i] = ctx;
+                if (ctx < 0 || ctx > p.max_ctx || (long long)ctx + 1 > (long long)p.mbps * p.block_size) {
+                    if (blockIdx.x == 0) report(p.status, PREFILL_ERR_SHAPE);
                 } else {
-                    report(p.status, PREFILL_ERR_BLOCK_TABLE);  // zero fill
+                    c = cdiv(ctx + 1, p.keys_per_unit) * p.n_kv_head;
                 }
             }
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int j = 0; j < SPT; ++j) {
-                    const int s = lq * SPT + j;
-                    cp_async16(st + t * L::TILE + slot_off<D>(lrow, s), src[t] + s * 8, bytes);
-                }
+            cnt[e] = run;
+            run += c;
         }
-        cp_async_commit();  // one group per tile slot, empty past the end
-    };
-    int pg_next = row_page(0);
-    for (int tile = 0; tile < DSTAGES - 1; ++tile) {
-        const int pg = pg_next;
-        pg_next = row_page(tile + 1);
-        issue(tile, pg);
-    }
-
-    const float sl2 = p.scale_log2;
-    float m_run = -CUDART_INF_F, l_run = 0.f;  // head `warp` (warps < R)
-    // P.V accumulators: columns 2*cp, 2*cp+1 for keys kg*KPG .. of each tile
-    constexpr int CP = D / 2, KPG = DT / L::KG;
-    const int cp = tid % CP, kg = tid / CP;
-    float acc[R][2];
+        int incl = run;  // inclusive scan of the per-thread totals over the warp
 #pragma unroll
-    for (int h = 0; h < R; ++h) acc[h][0] = acc[h][1] = 0.f;
-    float *spart = reinterpret_cast<float *>(smem + L::SPART);
-    float *sp = reinterpret_cast<float *>(smem + L::P);
-    float *salpha = reinterpret_cast<float *>(smem + L::ALPHA);
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int base = incl - run;
+        for (int w2 = 0; w2 < warp; ++w2) base += s_wsum[w2];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int i = tid * PER + e;
+            if (i <= p.num_seqs) scum[i] = base + cnt[e];  // scum[num_seqs] = total
+        }
+        if (tid == DTHREADS - 1 && p.num_seqs == kDecodeMaxSeqs) scum[kDecodeMaxSeqs] = base + run;
+    }
+    __syncthreads();  // the last CTA-wide barrier
+    const int total = scum[p.num_seqs];
+
+    // ---- load side of this warp: step (ui, si); in each copy instruction the
+    // lanes fetch consecutive 16-byte slots of the step's rows
+    Unit ui;
+    bool has_i = get_unit(p, sctx, scum, worker, total, ui);
+    int si = 0, issued = 0;
+    auto step_page = [&]() -> int {  // the page holding step (ui, si) (the whole step lies in it)
+        if (!has_i) return -1;
+        const int pos = ui.k0 + si * KS;
+        return pos < ui.ctx ? __ldg(&p.block_table[(size_t)ui.i * p.mbps + pos / bs]) : -1;
+    };
+    int pg_next = step_page();
+    auto issue_next = [&]() {
+        if (has_i) {
+            const uint32_t st = ring + (uint32_t)(issued % NSTAGE) * L::STAGE;
+            constexpr int SPR = D / 8;      // 16-byte slots per row
+            constexpr int RPI = 32 / SPR;   // rows per copy instruction
+            const int lrow = lane / SPR, s = lane % SPR;
+            const int p0 = ui.k0 + si * KS;                  // first position of the step
+            const int ncache = min(ui.k1, ui.ctx) - p0;      // rows [0, ncache) come from the cache page
+            const bool page_ok = pg_next >= 0 && pg_next < p.num_blocks;
+            const size_t rstride = G * D;                    // elements between consecutive positions of a page
+            const uint16_t *knew = p.k + ((size_t)ui.i * G + ui.g) * D + s * 8;
+            const uint16_t *vnew = p.v + ((size_t)ui.i * G + ui.g) * D + s * 8;
+            // row 0 of the step in the page's K half (the V half is bs positions later)
+            const uint16_t *krow0 =
+                page_ok ? p.cache + (((size_t)pg_next * 2 * bs + p0 % bs) * G + ui.g) * D + s * 8 : knew;
+            const size_t vhalf = (size_t)bs * rstride;
+            if (page_ok && ncache >= KS) {  // the common step: all 16 rows from the page
+#pragma unroll
+                for (int j = 0; j < KS / RPI; ++j) {
+                    const int row = j * RPI + lrow;
+                    const uint16_t *sk = krow0 + (size_t)row * rstride;
+                    cp_async16(st + slot_off(row, s), sk, 16);
+                    cp_async16(st + L::TILE + slot_off(row, s), sk + vhalf, 16);
+                }
+            } else {  // the new token's step or a unit's tail: per-row sources, zero fill past the end
+#pragma unroll
+                for (int j = 0; j < KS / RPI; ++j) {
+                    const int row = j * RPI + lrow;
+                    const uint16_t *sk = knew, *sv = vnew;
+                    uint32_t bytes = 0;
+                    if (row < ncache) {
+                        if (page_ok) {
+                            sk = krow0 + (size_t)row * rstride;
+                            sv = sk + vhalf;
+                            bytes = 16;
+                        } else if (s == 0) {
+                            report(p.status, PREFILL_ERR_BLOCK_TABLE);  // zero fill
+                        }
+                    } else if (p0 + row == ui.ctx) {
+                        bytes = 16;  // the new token: from the inputs
+                    }
+                    cp_async16(st + slot_off(row, s), sk, bytes);
+                    cp_async16(st + L::TILE + slot_off(row, s), sv, bytes);
+                }
+            }
+            ++issued;
+            if (++si == ui.nsteps) {
+                has_i = get_unit(p, sctx, scum, ui.u + W, total, ui);
+                si = 0;
+            }
+            pg_next = step_page();  // read one step ahead of its use
+        }
+        cp_async_commit();  // one group per compute step, empty once the stream has ended
+    };
+
+    // ---- compute side: queries as A fragments in registers (rows = heads)
+    const int row0 = lane >> 2, row1 = row0 + 8, c2 = 2 * (lane & 3);
+    auto load_q = [&](const Unit &u, uint32_t (&qa)[KSTEPS][4]) {
+        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(p.q + ((size_t)u.i * p.n_head + (size_t)u.g * r) * D);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            const int c = kk * 16 + c2;
+            qa[kk][0] = row0 < r ? __ldg(q0 + (row0 * D + c) / 2) : 0u;
+            qa[kk][1] = row1 < r ? __ldg(q0 + (row1 * D + c) / 2) : 0u;
+            qa[kk][2] = row0 < r ? __ldg(q0 + (row0 * D + c + 8) / 2) : 0u;
+            qa[kk][3] = row1 < r ? __ldg(q0 + (row1 * D + c + 8) / 2) : 0u;
+        }
+    };
+    Unit uc;
+    bool has_c = get_unit(p, sctx, scum, worker, total, uc);
+    int sc = 0, computed = 0;
+    uint32_t qa[KSTEPS][4], qn[KSTEPS][4];
+    if (has_c) load_q(uc, qa);
+
+    const float sl2 = p.scale_log2, thr = kLazyLog2 / sl2;
+    float m_ref[2] = {-CUDART_INF_F, -CUDART_INF_F};  // rows row0, row1
+    float l_part[2] = {0.f, 0.f};                       // this lane's share of the row sums
+    float o[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+    for (int k = 0; k < NSTAGE - 1; ++k) issue_next();
 
 #pragma unroll 1
-    for (int tile = 0; tile < ntiles; ++tile) {
+    while (has_c) {
+        cp_async_wait<NSTAGE - 2>();  // this step's copies (the oldest group) are done ...
+        __syncwarp();                 // ... for every lane, and the previous step is finished
+        issue_next();                 // into the stage the previous step used
+        if (sc == 0 && uc.split == uc.nunits - 1 && lane < 2 * (D / 8)) {
+            // the new token's K/V to its slot (position ctx); no unit reads
+            // that slot from the cache (the new token comes from the inputs)
+            const int page = __ldg(&p.block_table[(size_t)uc.i * p.mbps + uc.ctx / bs]);
+            if (page >= 0 && page < p.num_blocks) {
+                const int t = lane / (D / 8), s = lane % (D / 8);
+                const uint4 val =
+                    __ldg(reinterpret_cast<const uint4 *>((t ? p.v : p.k) + ((size_t)uc.i * G + uc.g) * D) + s);
+                uint16_t *dst = p.cache + ((((size_t)page * 2 + t) * bs + uc.ctx % bs) * G + uc.g) * D;
+                reinterpret_cast<uint4 *>(dst)[s] = val;
+            } else {
+                report(p.status, PREFILL_ERR_BLOCK_TABLE);
+            }
+        }
+        if (sc == uc.nsteps - 1) {  // the unit's last step: fetch the next unit's queries
+            Unit un;
+            if (get_unit(p, sctx, scum, uc.u + W, total, un)) load_q(un, qn);
+        }
+        const uint32_t st = ring + (uint32_t)(computed % NSTAGE) * L::STAGE;
+
+        // ---- S = Q K^T for the step's 16 keys (two 8-key tiles)
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
         {
-            const int pg = pg_next;
-            pg_next = row_page(tile + DSTAGES);
-            issue(tile + DSTAGES - 1, pg);
+            const int m = lane >> 3;  // matrices: keys 0-7 / 8-15 x columns +0 / +8
+            const int kr = (m >> 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                uint32_t kb[4];
+                ldsm_x4(st + slot_off(kr, 2 * kk + (m & 1)), kb);
+                mma16816(s0, qa[kk], kb[0], kb[1]);
+                mma16816(s1, qa[kk], kb[2], kb[3]);
+            }
         }
-        cp_async_wait<DSTAGES - 1>();
-        __syncthreads();  // tile `tile` has landed for every thread
-        const uint8_t *st = smem + (uint32_t)(tile % DSTAGES) * L::STAGE;
+        // columns of this lane: keys c2, c2 + 1 (tile 0) and 8 + c2, 9 + c2 (tile 1)
+        const int nvalid = uc.k1 - (uc.k0 + sc * KS);
+        if (c2 >= nvalid) s0[0] = s0[2] = -CUDART_INF_F;
+        if (c2 + 1 >= nvalid) s0[1] = s0[3] = -CUDART_INF_F;
+        if (c2 + 8 >= nvalid) s1[0] = s1[2] = -CUDART_INF_F;
+        if (c2 + 9 >= nvalid) s1[1] = s1[3] = -CUDART_INF_F;
+        float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
+        float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        // lazy max: move it (and rescale O and the sums) only past the threshold;
+        // every step holds a valid key, so a row's first step always moves it
+        const bool mv0 = mx0 > m_ref[0] + thr, mv1 = mx1 > m_ref[1] + thr;
+        if (__any_sync(0xffffffffu, mv0 || mv1)) {
+            const float n0 = mv0 ? mx0 : m_ref[0], n1 = mv1 ? mx1 : m_ref[1];
+            const float a0 = ex2((m_ref[0] - n0) * sl2), a1 = ex2((m_ref[1] - n1) * sl2);
+            m_ref[0] = n0;
+            m_ref[1] = n1;
+            l_part[0] *= a0;
+            l_part[1] *= a1;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                o[nt][0] *= a0;
+                o[nt][1] *= a0;
+                o[nt][2] *= a1;
+                o[nt][3] *= a1;
+            }
+        }
+        const float nm0 = -m_ref[0] * sl2, nm1 = -m_ref[1] * sl2;
+        const float p00 = ex2(fmaf(s0[0], sl2, nm0)), p01 = ex2(fmaf(s0[1], sl2, nm0));
+        const float p02 = ex2(fmaf(s0[2], sl2, nm1)), p03 = ex2(fmaf(s0[3], sl2, nm1));
+        const float p10 = ex2(fmaf(s1[0], sl2, nm0)), p11 = ex2(fmaf(s1[1], sl2, nm0));
+        const float p12 = ex2(fmaf(s1[2], sl2, nm1)), p13 = ex2(fmaf(s1[3], sl2, nm1));
+        l_part[0] += (p00 + p01) + (p10 + p11);
+        l_part[1] += (p02 + p03) + (p12 + p13);
+        // the scores' accumulators are the A fragment of P V (16 rows x 16 keys)
+        const uint32_t pa[4] = {pack_bf16x2(p00, p01), pack_bf16x2(p02, p03), pack_bf16x2(p10, p11),
+                                pack_bf16x2(p12, p13)};
 
-        // ---- scores: key kr, head_dim part pt
+        // ---- O += P V over all output columns, two 8-column tiles per load
         {
-            const int kr = tid % DT, pt = tid / DT;
-            float dot[R];
+            const int m = lane >> 3;  // matrices: keys 0-7 / 8-15 x columns +0 / +8
+            const int vr = (m & 1) * 8 + (lane & 7);
 #pragma unroll
-            for (int h = 0; h < R; ++h) dot[h] = 0.f;
-#pragma unroll
-            for (int j = 0; j < D / 32; ++j) {
-                const int s = pt * (D / 32) + j;
-                const uint4 kv = *reinterpret_cast<const uint4 *>(st + slot_off<D>(kr, s));
-                const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-                float kf[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    kf[2 * e] = __uint_as_float(w[e] << 16);
-                    kf[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-                }
-#pragma unroll
-                for (int h = 0; h < R; ++h) {
-                    const float4 qa = *reinterpret_cast<const float4 *>(sq + h * D + s * 8);
-                    const float4 qb = *reinterpret_cast<const float4 *>(sq + h * D + s * 8 + 4);
-                    dot[h] += qa.x * kf[0] + qa.y * kf[1] + qa.z * kf[2] + qa.w * kf[3] + qb.x * kf[4] +
-                              qb.y * kf[5] + qb.z * kf[6] + qb.w * kf[7];
-                }
+            for (int c = 0; c < NT / 2; ++c) {
+                uint32_t vb[4];
+                ldsm_x4_t(st + L::TILE + slot_off(vr, 2 * c + (m >> 1)), vb);
+                mma16816(o[2 * c], pa, vb[0], vb[1]);
+                mma16816(o[2 * c + 1], pa, vb[2], vb[3]);
             }
-#pragma unroll
-            for (int h = 0; h < R; ++h) spart[(pt * DT + kr) * R + h] = dot[h];
         }
-        __syncthreads();
+        ++computed;
+        if (++sc < uc.nsteps) continue;
 
-        // ---- online softmax: warp h owns head h; lane covers keys lane, lane + 32
-        if (warp < R) {
-            const int h = warp;
-            const int nvalid = min(DT, k1 - (k0 + tile * DT));
-            float s2[2];
+        // ---- end of the unit: row sums over the 4 lanes of a row, then rows < r out
+        float l0 = l_part[0], l1 = l_part[1];
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+        const bool whole = uc.nunits == 1;
+        const size_t hrow = (size_t)uc.i * p.n_head + (size_t)uc.g * r;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int kr = lane + 32 * u;
-                float s = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = hh ? row1 : row0;
+            if (h >= r) continue;
+            const float lsum = hh ? l1 : l0;
+            const size_t row = hrow + h;
+            if (whole) {
+                const float inv = 1.f / lsum;
 #pragma unroll
-                for (int pt = 0; pt < kParts; ++pt) s += spart[(pt * DT + kr) * R + h];
-                s2[u] = kr < nvalid ? s : -CUDART_INF_F;
-            }
-            float mt = fmaxf(s2[0], s2[1]);
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<uint32_t *>(p.out + row * D + nt * 8 + c2) =
+                        pack_bf16x2(o[nt][2 * hh] * inv, o[nt][2 * hh + 1] * inv);
+            } else {
+                const size_t prow = (size_t)uc.split * p.num_seqs * p.n_head + row;  // [unit][seq][head]
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-            const float m_new = fmaxf(m_run, mt);  // finite: every tile holds a valid key
-            const float alpha = ex2((m_run - m_new) * sl2);
-            const float p0 = ex2((s2[0] - m_new) * sl2), p1 = ex2((s2[1] - m_new) * sl2);
-            float sum = p0 + p1;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            l_run = l_run * alpha + sum;
-            m_run = m_new;
-            sp[lane * 8 + h] = p0;
-            sp[(lane + 32) * 8 + h] = p1;
-            if (lane == 0) salpha[h] = alpha;
-        }
-        __syncthreads();
-
-        // ---- O = alpha O + P V over this thread's keys and column pair
-        {
-#pragma unroll
-            for (int h = 0; h < R; ++h) {
-                const float a = salpha[h];
-                acc[h][0] *= a;
-                acc[h][1] *= a;
-            }
-            const int d = 2 * cp;
-            const uint8_t *vt = st + L::TILE;
-#pragma unroll
-            for (int kk = 0; kk < KPG; ++kk) {
-                const int kr = kg * KPG + kk;
-                const uint32_t v2 =
-                    *reinterpret_cast<const uint32_t *>(vt + slot_off<D>(kr, d >> 3) + (d & 7) * 2);
-                const float vx = __uint_as_float(v2 << 16), vy = __uint_as_float(v2 & 0xffff0000u);
-                const float4 pa = *reinterpret_cast<const float4 *>(sp + kr * 8);
-                const float4 pb = *reinterpret_cast<const float4 *>(sp + kr * 8 + 4);
-                const float pk[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-#pragma unroll
-                for (int h = 0; h < R; ++h) {
-                    acc[h][0] += pk[h] * vx;
-                    acc[h][1] += pk[h] * vy;
-                }
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<float2 *>(p.part_o + prow * D + nt * 8 + c2) =
+                        make_float2(o[nt][2 * hh], o[nt][2 * hh + 1]);
+                if ((lane & 3) == 0)
+                    *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_ref[hh] * sl2, lsum);
             }
         }
-        __syncthreads();  // the stage and P are free for the next tile
-    }
-    cp_async_wait<0>();
-
-    // ---- reduce the key groups, then write the output or this unit's partial
-    float *red = reinterpret_cast<float *>(smem);  // [KG][R][D], over the drained ring
-    float *sml = reinterpret_cast<float *>(smem + L::ML);
 #pragma unroll
-    for (int h = 0; h < R; ++h) {
-        red[(kg * R + h) * D + 2 * cp] = acc[h][0];
-        red[(kg * R + h) * D + 2 * cp + 1] = acc[h][1];
-    }
-    if (warp < R && lane == 0) {
-        sml[2 * warp] = m_run * sl2;
-        sml[2 * warp + 1] = l_run;
-    }
-    __syncthreads();
-    const bool whole = nunits == 1;
-    for (int x = tid; x < R * D / 2; x += DTHREADS) {  // column pairs
-        const int h = x / (D / 2), d = 2 * (x % (D / 2));
-        float o0 = 0.f, o1 = 0.f;
+        for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+        m_ref[0] = m_ref[1] = -CUDART_INF_F;
+        l_part[0] = l_part[1] = 0.f;
+        has_c = get_unit(p, sctx, scum, uc.u + W, total, uc);
+        sc = 0;
 #pragma unroll
-        for (int q = 0; q < L::KG; ++q) {
-            o0 += red[(q * R + h) * D + d];
-            o1 += red[(q * R + h) * D + d + 1];
-        }
-        const size_t row = (size_t)i * p.n_head + (size_t)g * R + h;
-        if (whole) {
-            const float inv = 1.f / sml[2 * h + 1];
-            *reinterpret_cast<uint32_t *>(p.out + row * D + d) = pack_bf16x2(o0 * inv, o1 * inv);
-        } else {
-            const size_t prow = (size_t)split * p.num_seqs * p.n_head + row;  // [unit][seq][head]
-            *reinterpret_cast<float2 *>(p.part_o + prow * D + d) = make_float2(o0, o1);
-            if (d == 0) *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(sml[2 * h], sml[2 * h + 1]);
-        }
+        for (int kk = 0; kk < KSTEPS; ++kk)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) qa[kk][e] = qn[kk][e];
     }
+    cp_async_wait<0>();  // nothing in flight when the warp exits
 }
 
 // Merge of a sequence's units: one warp per (sequence, query head), the
@@ -343,15 +454,20 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
 }
 
-template <int D, int R>
-int launch_r(const DecodeParams &p, void *stream) {
-    using L = DecLay<D, R>;
+template <int D>
+int launch_d(const DecodeParams &p, void *stream) {
+    using L = DecLay<D>;
     const size_t smem = L::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(paged_decode_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(paged_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
-    dim3 grid((unsigned)p.max_units, (unsigned)p.n_kv_head, (unsigned)p.num_seqs);
-    paged_decode_kernel<D, R><<<grid, DTHREADS, smem, (cudaStream_t)stream>>>(p);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long units = (long long)p.max_units * p.n_kv_head * p.num_seqs;  // a bound on the call's units
+    const long long ctas_needed = (units + WARPS - 1) / WARPS;
+    const long long slots = (long long)kCtasPerSm * sms;
+    const int grid = (int)(ctas_needed < slots ? ctas_needed : slots);
+    paged_decode_kernel<D><<<grid, DTHREADS, smem, (cudaStream_t)stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.max_units <= 1) return (int)e;
     dim3 cgrid((unsigned)p.num_seqs, (unsigned)cdiv(p.n_head, 4));
@@ -359,25 +475,14 @@ int launch_r(const DecodeParams &p, void *stream) {
     return (int)cudaGetLastError();
 }
 
-template <int D>
-int launch_d(const DecodeParams &p, void *stream) {
-    switch (p.n_head / p.n_kv_head) {
-        case 1: return launch_r<D, 1>(p, stream);
-        case 2: return launch_r<D, 2>(p, stream);
-        case 3: return launch_r<D, 3>(p, stream);
-        case 4: return launch_r<D, 4>(p, stream);
-        case 5: return launch_r<D, 5>(p, stream);
-        case 6: return launch_r<D, 6>(p, stream);
-        case 7: return launch_r<D, 7>(p, stream);
-        default: return launch_r<D, 8>(p, stream);
-    }
-}
-
 }  // namespace
 
 int decode_keys_per_unit(int max_ctx) {
-    // units of 512 keys, fewer and longer for very long contexts (at most 64 per sequence)
-    int u = 512;
+    // units of 128 keys (per-warp work within ~3 % of the mean on 64 varlen
+    // sequences, where 256-key units leave an 18 % spread), longer for very
+    // long contexts (at most kDecodeMaxUnits per sequence); always a multiple
+    // of the 16-key step
+    int u = 128;
     while (cdiv(max_ctx + 1, u) > kDecodeMaxUnits) u *= 2;
     return u;
 }

@@ -7,6 +7,9 @@ namespace pf {
 // At most this many key splits (work units) per sequence; longer contexts get
 // longer units (decode_keys_per_unit).
 constexpr int kDecodeMaxUnits = 64;
+// Sequences per decode call (their context lengths and unit counts are kept in
+// shared memory by every CTA).
+constexpr int kDecodeMaxSeqs = 2048;
 
 struct DecodeParams {
     const uint16_t *q;            // [B][n_head][D]   the new token's queries

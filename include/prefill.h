@@ -195,10 +195,11 @@ int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, co
  *   out            device, written: [num_seqs][n_head][head_dim] bf16
  *   kv_cache, num_blocks, block_table, max_blocks_per_seq, block_size,
  *   status_dev, stream   as for prefill_attn_chunked.
- * n_head / n_kv_head must be at most 8 (PREFILL_ERR_UNSUPPORTED otherwise).
+ * n_head / n_kv_head must be at most 16 and num_seqs at most 2048
+ * (PREFILL_ERR_UNSUPPORTED otherwise).
  * Requires max_context_len + 1 <= max_blocks_per_seq * block_size.  A sequence
  * whose context length is negative or above max_context_len is skipped and
- * reported as PREFILL_ERR_SHAPE.  Long contexts are split into units of >= 512
+ * reported as PREFILL_ERR_SHAPE.  Contexts are split into units of >= 128
  * keys whose partial results a second kernel merges; their partials use the
  * same per-(device, stream) workspace as the prefill split-KV partials
  * (max units x num_seqs x n_head x (head_dim + 2) x 4 bytes).

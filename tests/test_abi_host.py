@@ -213,7 +213,7 @@ def test_decode_validation(lib):
 
     assert call(q=None) == 1 and call(ctx=None) == 1 and call(bt=None) == 1
     assert call(H=9, G=2) == 2
-    assert call(H=18, G=2) == 3            # 9 query heads per kv head: above 8
+    assert call(H=34, G=2) == 3            # 17 query heads per kv head: above 16
     assert call(D=96) == 3 and call(bs=24) == 3 and call(scale=0.0) == 3
     assert call(maxc=128) == 4             # 129 keys do not fit 8 pages of 16
     assert call(nb=0) == 4

@@ -60,7 +60,7 @@ def test_decode_head_dim_64(n):
     _check(_case([n], 8, 2, 64, seed=420 + n), f"d=64 len={n}")
 
 
-@pytest.mark.parametrize("H,G", [(4, 4), (8, 4), (6, 2), (8, 2), (8, 1), (16, 2)])
+@pytest.mark.parametrize("H,G", [(4, 4), (8, 4), (6, 2), (8, 2), (8, 1), (16, 2), (16, 1), (30, 2)])
 def test_decode_head_groupings(H, G):
     _check(_case([700, 37], H, G, 128, seed=430 + H * 10 + G), f"H={H} G={G}")
 
