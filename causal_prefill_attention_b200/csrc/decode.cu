@@ -310,14 +310,24 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
         // ---- S = Q K^T for the step's 16 keys (two 8-key tiles)
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
         {
+            // four independent accumulation chains (even / odd column steps)
+            float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
             const int m = lane >> 3;  // matrices: keys 0-7 / 8-15 x columns +0 / +8
             const int kr = (m >> 1) * 8 + (lane & 7);
 #pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk) {
-                uint32_t kb[4];
+            for (int kk = 0; kk < KSTEPS; kk += 2) {
+                uint32_t kb[4], kc[4];
                 ldsm_x4(st + slot_off(kr, 2 * kk + (m & 1)), kb);
+                ldsm_x4(st + slot_off(kr, 2 * kk + 2 + (m & 1)), kc);
                 mma16816(s0, qa[kk], kb[0], kb[1]);
                 mma16816(s1, qa[kk], kb[2], kb[3]);
+                mma16816(t0, qa[kk + 1], kc[0], kc[1]);
+                mma16816(t1, qa[kk + 1], kc[2], kc[3]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s0[e] += t0[e];
+                s1[e] += t1[e];
             }
         }
         // columns of this lane: keys c2, c2 + 1 (tile 0) and 8 + c2, 9 + c2 (tile 1)
@@ -421,7 +431,9 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
 }
 
 // Merge of a sequence's units: one warp per (sequence, query head), the
-// online-softmax merge rule over the units' (max, sum, O).
+// online-softmax merge rule over the units' (max, sum, O): lane s holds unit
+// s's max and sum (and s + 32's), so the weights 2^(m_s - M) come from one warp
+// max and one warp sum; the O rows are then summed with independent loads.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
     const int i = blockIdx.x;
@@ -430,23 +442,48 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     if (h >= p.n_head) return;
     const int ctx = p.context_lens[i];
     if (ctx < 0 || ctx > p.max_ctx || (long long)ctx + 1 > (long long)p.mbps * p.block_size) return;
-    const int nunits = cdiv(ctx + 1, p.keys_per_unit);
-    if (nunits <= 1) return;  // written by the unit itself
+    const int nunits = cdiv(ctx + 1, p.keys_per_unit);  // <= kDecodeMaxUnits = 64
+    if (nunits <= 1) return;                             // written by the unit itself
     constexpr int E = D / 32;
     const size_t row = (size_t)i * p.n_head + h;
     const size_t sstride = (size_t)p.num_seqs * p.n_head;
-    float M = -CUDART_INF_F, Lsum = 0.f, acc[E];
+    float m[2], l[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int sidx = lane + 32 * u;
+        m[u] = -CUDART_INF_F;
+        l[u] = 0.f;
+        if (sidx < nunits) {
+            const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (sidx * sstride + row) * 2);
+            m[u] = ml.x;
+            l[u] = ml.y;
+        }
+    }
+    float M = fmaxf(m[0], m[1]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float w0 = ex2(m[0] - M), w1 = ex2(m[1] - M);  // 0 for absent units
+    float Lsum = w0 * l[0] + w1 * l[1];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
+    float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll 4
     for (int s = 0; s < nunits; ++s) {
-        const size_t prow = s * sstride + row;
-        const float m = p.part_ml[prow * 2], l = p.part_ml[prow * 2 + 1];
-        const float Mn = fmaxf(M, m);
-        const float a = ex2(M - Mn), b = ex2(m - Mn);
-        Lsum = Lsum * a + l * b;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = acc[e] * a + b * p.part_o[prow * D + lane * E + e];
-        M = Mn;
+        const float wgt = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+        const float *src = p.part_o + (s * sstride + row) * D + lane * E;
+        if constexpr (E == 4) {
+            const float4 f = *reinterpret_cast<const float4 *>(src);
+            acc[0] += wgt * f.x;
+            acc[1] += wgt * f.y;
+            acc[2] += wgt * f.z;
+            acc[3] += wgt * f.w;
+        } else {
+            const float2 f = *reinterpret_cast<const float2 *>(src);
+            acc[0] += wgt * f.x;
+            acc[1] += wgt * f.y;
+        }
     }
     const float inv = 1.f / Lsum;
     uint16_t *dst = p.out + row * D + lane * E;
