@@ -189,3 +189,22 @@ def prefill(w, *, kv_cache=None, context_lens=None, rows=None, heads=None, windo
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int):
+    """The fused QKV projection (hncyxsy.com/news/270449 §4.1: one GEMM with the
+    W_q, W_k, W_v blocks concatenated, its (s, (H + 2G) d) output cut by
+    columns into Q, K, V; §2.2: each reshaped to (s, heads, head_dim)).
+
+    x: [T, hidden] bf16; w: [(n_head + 2 n_kv_head) head_dim, hidden] bf16, one
+    row per output feature (the Q block's rows first, then K's, then V's).
+    Returns (q [T, H, d], k [T, G, d], v [T, G, d]) in fp64: the plain product
+    y = x w^T in fp64 from the bf16 values, then the column split."""
+    xs = x.detach().cpu().to(torch.float64).numpy()
+    ws = w.detach().cpu().to(torch.float64).numpy()
+    y = xs @ ws.T
+    T = y.shape[0]
+    hq, hk = n_head * head_dim, n_kv_head * head_dim
+    assert y.shape[1] == hq + 2 * hk
+    return (y[:, :hq].reshape(T, n_head, head_dim), y[:, hq:hq + hk].reshape(T, n_kv_head, head_dim),
+            y[:, hq + hk:].reshape(T, n_kv_head, head_dim))

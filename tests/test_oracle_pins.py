@@ -428,3 +428,60 @@ def test_window_chunked_equals_unchunked():
         cache = oracle.kv_write(k, v, cu, cache, bt, bs, context_lens=ctx)
     assert np.max(np.abs(np.concatenate(outs, axis=0) - full_out)) < 1e-12
     assert torch.equal(cache.view(torch.int16), full_cache.view(torch.int16))
+
+
+# ---------------------------------------------------------------- fused QKV projection
+# hncyxsy.com/news/270449 §4.1 / §2.2: y = x W^T with W = [W_q; W_k; W_v] (one row
+# per output feature), cut by columns into Q, K, V, each reshaped head-dim last.
+
+def test_qkv_projection_brute_force_tiny():
+    g = torch.Generator().manual_seed(50)
+    T, hid, H, G, d = 3, 5, 2, 1, 2
+    x = torch.randn(T, hid, generator=g).to(torch.bfloat16)
+    w = torch.randn((H + 2 * G) * d, hid, generator=g).to(torch.bfloat16)
+    q, k, v = oracle.qkv_projection(x, w, H, G, d)
+    xs, ws = _f64(x), _f64(w)
+    for t in range(T):
+        for n in range((H + 2 * G) * d):
+            y = sum(xs[t, c] * ws[n, c] for c in range(hid))
+            if n < H * d:
+                got = q[t, n // d, n % d]
+            elif n < (H + G) * d:
+                got = k[t, (n - H * d) // d, (n - H * d) % d]
+            else:
+                got = v[t, (n - (H + G) * d) // d, (n - (H + G) * d) % d]
+            assert abs(got - y) < 1e-12
+
+
+def test_qkv_projection_one_hot_weights_select_features():
+    """W rows one-hot: output feature n copies input feature perm[n], so every
+    element of Q, K and V is a known input element (checks the column order
+    Q | K | V and the head-dim-last reshape)."""
+    g = torch.Generator().manual_seed(51)
+    T, H, G, d = 4, 4, 2, 8
+    N = (H + 2 * G) * d
+    hid = N
+    x = torch.randn(T, hid, generator=g).to(torch.bfloat16)
+    perm = torch.randperm(hid, generator=g)
+    w = torch.zeros(N, hid)
+    w[torch.arange(N), perm] = 1.0
+    q, k, v = oracle.qkv_projection(x, w.to(torch.bfloat16), H, G, d)
+    xs = _f64(x)
+    for h in range(H):
+        for e in range(d):
+            assert np.array_equal(q[:, h, e], xs[:, perm[h * d + e]])
+    for gg in range(G):
+        for e in range(d):
+            assert np.array_equal(k[:, gg, e], xs[:, perm[H * d + gg * d + e]])
+            assert np.array_equal(v[:, gg, e], xs[:, perm[(H + G) * d + gg * d + e]])
+
+
+def test_qkv_projection_matches_torch_linear_fp64():
+    g = torch.Generator().manual_seed(52)
+    T, hid, H, G, d = 37, 96, 4, 2, 16
+    x = torch.randn(T, hid, generator=g).to(torch.bfloat16)
+    w = torch.randn((H + 2 * G) * d, hid, generator=g).to(torch.bfloat16)
+    q, k, v = oracle.qkv_projection(x, w, H, G, d)
+    ref = torch.nn.functional.linear(x.to(torch.float64), w.to(torch.float64)).numpy()
+    got = np.concatenate([q.reshape(T, -1), k.reshape(T, -1), v.reshape(T, -1)], axis=1)
+    assert np.max(np.abs(got - ref)) < 1e-12
