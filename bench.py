@@ -227,6 +227,49 @@ class DecodeRunner:
             raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
 
 
+class QkvRunner:
+    """The fused QKV projection that produces the headline prompt's q/k/v:
+    x [8192, 4096] times the concatenated weight [6144, 4096]^T (2 M N K FLOP),
+    with cuBLAS (torch.matmul) on the same operands timed beside it."""
+
+    def __init__(self, tokens, hidden, H, G, d, seed, stream):
+        x, w = W.make_projection(tokens, hidden, H, G, d, seed)
+        dv = torch.device("cuda")
+        self.x, self.w = x.to(dv), w.to(dv)
+        self.q = torch.empty(tokens, H, d, dtype=torch.bfloat16, device=dv)
+        self.k = torch.empty(tokens, G, d, dtype=torch.bfloat16, device=dv)
+        self.v = torch.empty_like(self.k)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dv)
+        self.H, self.G, self.d, self.stream = H, G, d, stream
+        self.flops = 2.0 * tokens * hidden * (H + 2 * G) * d
+        self.launches = 1
+
+    def step(self):
+        _lib.qkv_projection(self.x, self.w, self.H, self.G, self.d, self.q, self.k, self.v, status=self.status,
+                            stream=self.stream)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
+
+
+class LibraryMatmul:
+    """torch.matmul (cuBLAS) on the same operands: context for the QKV line."""
+
+    def __init__(self, runner):
+        self.r = runner
+        self.launches = 1
+
+    def step(self):
+        torch.matmul(self.r.x, self.r.w.t())
+
+    def check_status(self):
+        pass
+
+
+QKV_LINE = ("qkv_proj_s8192_h4096_n6144", 8192, 4096, 32, 8, 128, 3001)
+
 # secondary line: one decode step after the 64 prompts of the varlen workload
 DECODE_LINE = ("decode64_gqa_h32g8_d128", "varlen64_gqa_h32g8_d128", 2001)
 
@@ -408,6 +451,16 @@ def main():
                        "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches,
                        "window": win}
         del rx, wx
+        torch.cuda.empty_cache()
+        name, T_, hid_, H_, G_, d_, seed_ = QKV_LINE
+        rx = QkvRunner(T_, hid_, H_, G_, d_, seed_, stream)
+        dx = time_steps(rx, max(10, args.steps), 3, stream, flush)
+        lx = time_steps(LibraryMatmul(rx), max(10, args.steps), 3, stream, flush)
+        mx, ml = statistics.median(dx), statistics.median(lx)
+        extra[name] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
+                       "frac_of_peak": round(rx.flops / (mx * 1e-3) / 1e12 / pk["bf16"], 4),
+                       "library_matmul_tflops": round(rx.flops / (ml * 1e-3) / 1e12, 2), "launches": rx.launches}
+        del rx
         torch.cuda.empty_cache()
         name, base, seed = DECODE_LINE
         rx = DecodeRunner(W.named_workload(base), seed, stream)

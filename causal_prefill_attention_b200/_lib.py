@@ -23,7 +23,7 @@ EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall",
             "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
             "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window",
-            "paged_decode_attn")
+            "paged_decode_attn", "qkv_projection")
 
 _lib = None
 
@@ -66,6 +66,8 @@ def load() -> ctypes.CDLL:
         lib.prefill_kv_block_rule_window.restype = I
         lib.paged_decode_attn.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, I, P, I, I, P, P]
         lib.paged_decode_attn.restype = I
+        lib.qkv_projection.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
+        lib.qkv_projection.restype = I
         _lib = lib
     return _lib
 
@@ -204,6 +206,21 @@ def paged_decode_attn(q, k, v, context_lens, max_context_len: int, scale: float,
         _ptr(status), _stream_ptr(stream))
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "paged_decode_attn")
+    return rc
+
+
+def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int, q, k, v,
+                   status: Optional[torch.Tensor] = None, stream=None, raise_on_error: bool = True) -> int:
+    """Fused QKV projection (C ABI ``qkv_projection``): y = x w^T on the tensor
+    cores, cut by columns into q [T, n_head, d], k and v [T, n_kv_head, d].
+    x [T, hidden] and w [(n_head + 2 n_kv_head) d, hidden] are bf16."""
+    _check_bf16("x", x, 2), _check_bf16("w", w, 2)
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3)
+    T, hid = x.shape
+    rc = load().qkv_projection(_ptr(x), _ptr(w), T, hid, int(n_head), int(n_kv_head), int(head_dim), _ptr(q),
+                               _ptr(k), _ptr(v), _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "qkv_projection")
     return rc
 
 

@@ -11,8 +11,8 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libprefill.so")
 ROOT = os.path.dirname(HERE)
 
-SOURCES = ["api.cu", "noalloc.cu", "prefill_fwd.cu", "prefill_fwd_v0.cu", "decode.cu"]
-HEADERS = ["block_rule.h", "params.h", "sm100.cuh", "decode.h"]
+SOURCES = ["api.cu", "noalloc.cu", "prefill_fwd.cu", "prefill_fwd_v0.cu", "decode.cu", "qkv_gemm.cu"]
+HEADERS = ["block_rule.h", "params.h", "sm100.cuh", "decode.h", "qkv_gemm.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

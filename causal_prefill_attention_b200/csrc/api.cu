@@ -17,6 +17,7 @@
 #include "block_rule.h"
 #include "decode.h"
 #include "params.h"
+#include "qkv_gemm.h"
 
 namespace {
 
@@ -283,6 +284,40 @@ int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefil
         p.part_ml = reinterpret_cast<float *>(ws + rows * head_dim * sizeof(float));
     }
     return pf::launch_decode(p, head_dim, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+}
+
+int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int hidden, int n_head, int n_kv_head,
+                   int head_dim, prefill_bf16 *q, prefill_bf16 *k, prefill_bf16 *v, int32_t *status_dev,
+                   prefill_stream_t stream) {
+    if (!x || !w || !q || !k || !v) return PREFILL_ERR_NULL;
+    if (tokens < 0 || hidden < 0 || n_head < 1 || n_kv_head < 1 || head_dim < 1) return PREFILL_ERR_SHAPE;
+    if (head_dim % 32 != 0 || hidden % 64 != 0 || hidden == 0) return PREFILL_ERR_UNSUPPORTED;
+    const long long N = (long long)(n_head + 2 * n_kv_head) * head_dim;
+    if (N % 256 != 0 || N > (1 << 30) || hidden > (1 << 30)) return PREFILL_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PREFILL_ERR_ALIGNMENT;
+    if (tokens == 0) return PREFILL_OK;
+    CUtensorMap tm_x, tm_w;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)tokens}, strides[1] = {(cuuint64_t)hidden * 2};
+        const cuuint32_t box[2] = {64, 128};
+        if (!encode(&tm_x, x, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)N}, strides[1] = {(cuuint64_t)hidden * 2};
+        const cuuint32_t box[2] = {64, 256};
+        if (!encode(&tm_w, w, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+    pf::QkvParams p;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.M = tokens;
+    p.N = (int)N;
+    p.K = hidden;
+    p.hq = n_head * head_dim;
+    p.hkv = n_kv_head * head_dim;
+    p.status = status_dev;
+    return pf::launch_qkv_gemm(tm_x, tm_w, p, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 
 void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }

@@ -1,0 +1,21 @@
+// qkv_gemm.h -- launch parameters of the fused QKV projection (qkv_gemm.cu).
+#pragma once
+#include <cstdint>
+#include <cstddef>
+#include <cuda.h>
+
+namespace pf {
+
+struct QkvParams {
+    uint16_t *q;        // [M][hq]  = [T][n_head][head_dim]
+    uint16_t *k;        // [M][hkv] = [T][n_kv_head][head_dim]
+    uint16_t *v;        // [M][hkv]
+    int M, N, K;        // tokens, (n_head + 2 n_kv_head) head_dim, hidden
+    int hq, hkv;        // n_head * head_dim, n_kv_head * head_dim
+    int32_t *status;    // nullable
+};
+
+size_t qkv_gemm_smem_bytes();
+int launch_qkv_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const QkvParams &p, void *stream);
+
+}  // namespace pf

@@ -204,3 +204,15 @@ def decode_views(w: Workload):
     cu[1:] = torch.cumsum(ctx.to(torch.int64), 0).to(torch.int32)
     return (w.q[keep].contiguous(), w.k[keep].contiguous(), w.v[keep].contiguous(), cu,
             w.q[last].contiguous(), w.k[last].contiguous(), w.v[last].contiguous(), ctx)
+
+
+def make_projection(tokens: int, hidden: int, n_head: int, n_kv_head: int, head_dim: int, seed: int):
+    """Inputs of the fused QKV projection: activations x [tokens, hidden] and the
+    concatenated weight w [(n_head + 2 n_kv_head) head_dim, hidden], bf16, drawn
+    x ~ N(0, 1) then w ~ N(0, 1 / hidden) so that outputs are O(1)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    x = _bf16_randn(gen, (tokens, hidden))
+    w = (torch.randn((n_head + 2 * n_kv_head) * head_dim, hidden, generator=gen, dtype=torch.float32)
+         / math.sqrt(hidden)).to(torch.bfloat16)
+    return x, w

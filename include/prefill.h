@@ -213,6 +213,30 @@ int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefil
                       int32_t *status_dev, prefill_stream_t stream);
 
 /*
+ * qkv_projection -- the fused QKV projection that feeds prefill_attn
+ * (hncyxsy.com/news/270449 §4.1: the W_q, W_k, W_v blocks concatenated into
+ * one GEMM that reads the activations once, its output cut by columns into
+ * Q, K and V; §2.2: each reshaped to (tokens, heads, head_dim)).
+ *
+ *   x        device bf16 [tokens][hidden], row-major
+ *   w        device bf16 [(n_head + 2 n_kv_head) head_dim][hidden]: one row per
+ *            output feature (the layout of a linear layer's weight), the
+ *            n_head head_dim rows of W_q first, then W_k's, then W_v's
+ *   q        device, written: bf16 [tokens][n_head][head_dim]
+ *   k, v     device, written: bf16 [tokens][n_kv_head][head_dim]
+ * y = x w^T with fp32 accumulation, each output rounded once to bf16 (round to
+ * nearest even).  Requires hidden a multiple of 64, head_dim a multiple of 32
+ * and (n_head + 2 n_kv_head) head_dim a multiple of 256
+ * (PREFILL_ERR_UNSUPPORTED otherwise); pointers 16-byte aligned.  Runs on the
+ * tensor cores (tcgen05) with 128 x 256 output tiles; a device wait that runs
+ * past its limit is reported as PREFILL_ERR_TIMEOUT in *status_dev.
+ */
+int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int hidden,
+                   int n_head, int n_kv_head, int head_dim,
+                   prefill_bf16 *q, prefill_bf16 *k, prefill_bf16 *v,
+                   int32_t *status_dev, prefill_stream_t stream);
+
+/*
  * prefill_attn_chunked_noalloc -- prefill_attn_chunked for callers that cannot
  * allocate device memory.  The pages have no counterpart: this is a deployment
  * variant of the chunked call, not a step of the method.

@@ -23,7 +23,7 @@ def lib():
 def _declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged)_[a-z_0-9]+)\s*\(", src,
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged|qkv)_[a-z_0-9]+)\s*\(", src,
                                  flags=re.M)))
 
 
@@ -219,3 +219,24 @@ def test_decode_validation(lib):
     assert call(nb=0) == 4
     assert call(q=ctypes.c_void_p(FAKE + 4)) == 7
     assert call(B=0) == 0
+
+
+def test_qkv_projection_validation(lib):
+    P = ctypes.c_void_p(FAKE)
+    #        x  w  T    hid  H  G  d    q  k  v  status stream
+    base = [P, P, 128, 512, 4, 2, 64, P, P, P, None, None]
+
+    def call(**over):
+        a = list(base)
+        names = ["x", "w", "T", "hid", "H", "G", "d", "q", "k", "v"]
+        for key, val in over.items():
+            a[names.index(key)] = val
+        return lib.qkv_projection(*a)
+
+    assert call(x=None) == 1 and call(v=None) == 1
+    assert call(T=-1) == 2 and call(H=0) == 2
+    assert call(hid=100) == 3              # hidden not a multiple of 64
+    assert call(d=48) == 3                 # head_dim not a multiple of 32
+    assert call(H=3, G=1, d=64) == 3       # (3 + 2) * 64 = 320 output features: not a multiple of 256
+    assert call(q=ctypes.c_void_p(FAKE + 2)) == 7
+    assert call(T=0) == 0
