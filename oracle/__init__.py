@@ -54,6 +54,15 @@ def _configure(lib):
               lib.oracle_softmax_weights, lib.oracle_kv_write):
         f.restype = I
     lib.oracle_num_threads.restype = I
+    F = ctypes.c_float
+    lib.oracle_e4m3_encode.argtypes = [F]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = D
+    lib.oracle_kv_write_fp8.argtypes = [P, P, P, P, I, I, I, P, P, P, I, P, I, I]
+    lib.oracle_kv_write_fp8.restype = I
+    lib.oracle_decode_fp8.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, I, I, P]
+    lib.oracle_decode_fp8.restype = I
     return lib
 
 
@@ -208,3 +217,57 @@ def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int):
     assert y.shape[1] == hq + 2 * hk
     return (y[:, :hq].reshape(T, n_head, head_dim), y[:, hq:hq + hk].reshape(T, n_kv_head, head_dim),
             y[:, hq + hk:].reshape(T, n_kv_head, head_dim))
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) KV cache
+def e4m3_encode(x: float) -> int:
+    """e4m3 code of a float32 value: round to nearest (ties to even), magnitudes
+    beyond 448 saturate to 448."""
+    return int(_load().oracle_e4m3_encode(float(x)))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(_load().oracle_e4m3_decode(int(code)))
+
+
+def _f32(a) -> np.ndarray:
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def kv_write_fp8(k, v, cu_seqlens, kv_cache: torch.Tensor, block_table, block_size, k_scale, v_scale, *,
+                 context_lens=None) -> torch.Tensor:
+    """Copy of the FP8 cache (uint8 codes [NB, 2, bs, G, d]) with every token's K
+    and V quantized into its slot: code = e4m3(fp32(x) / scale[g])."""
+    kb, vb = _bits(k), _bits(v)
+    cu = _i32(cu_seqlens)
+    ctx = None if context_lens is None else _i32(context_lens)
+    bt = _i32(block_table)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    cache = kv_cache.detach().cpu().contiguous().numpy().copy()
+    assert cache.dtype == np.uint8
+    G, d = int(k.shape[1]), int(k.shape[2])
+    rc = _load().oracle_kv_write_fp8(_ptr(kb), _ptr(vb), _ptr(cu), _ptr(ctx), len(cu) - 1, G, d, _ptr(ks), _ptr(vs),
+                                     _ptr(cache), int(kv_cache.shape[0]), _ptr(bt), int(bt.shape[1]), block_size)
+    _check(rc, "oracle_kv_write_fp8")
+    return torch.from_numpy(cache).reshape(kv_cache.shape)
+
+
+def decode_fp8(q, k, v, context_lens, n_head, n_kv_head, head_dim, scale, k_scale, v_scale, kv_cache, block_table,
+               block_size) -> np.ndarray:
+    """Decode over an FP8 cache: the new token of sequence i (q [B, H, d],
+    k/v [B, G, d]) attends to the dequantized cache entries 0 .. ctx_i - 1 and
+    to its own K/V quantized the same way.  Returns [B, H, d] fp64."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    ctx = _i32(context_lens)
+    bt = _i32(block_table)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    cache = kv_cache.detach().cpu().contiguous().numpy()
+    B = len(ctx)
+    out = np.zeros((B, n_head, head_dim), dtype=np.float64)
+    rc = _load().oracle_decode_fp8(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(ctx), B, n_head, n_kv_head, head_dim,
+                                   float(scale), _ptr(ks), _ptr(vs), _ptr(cache), int(kv_cache.shape[0]), _ptr(bt),
+                                   int(bt.shape[1]), block_size, _ptr(out))
+    _check(rc, "oracle_decode_fp8")
+    return out

@@ -49,6 +49,7 @@
  * invariants, a brute-force loop and a library routine by the CPU tests.
  */
 #include <math.h>
+#include <stddef.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -267,6 +268,151 @@ int oracle_kv_write(const uint16_t *k, const uint16_t *v, const int32_t *cu_seql
         }
     }
     return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ FP8 KV cache
+ * hncyxsy.com/news/227904 §2.3: the KV cache may be kept in FP8 while the
+ * softmax stays at higher precision; §3.3: FP8 / INT8 (1 byte per element).
+ * Readings: the format is e4m3 (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent field 0 holds the subnormals m * 2^-9; code 0x7F /
+ * 0xFF is NaN, so the largest finite value is 448).  Each kv head has one
+ * scale for K and one for V: the stored code is e4m3(x / scale) with the
+ * quotient formed in fp32 (x is the bf16 value, scale the caller's float) and
+ * rounded to the nearest code, ties to the even code, magnitudes beyond 448
+ * saturating to 448; the value the attention uses is code_value * scale.
+ */
+
+/* e4m3 code of a float32 value (round to nearest even, saturate to +-448). */
+uint8_t oracle_e4m3_encode(float x) {
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a != a) return (uint8_t)(sign | 0x7F);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {                 /* subnormal codes: m * 2^-9, m = 0 .. 8 */
+        double m = nearbyint(a * 512.0);      /* default rounding: to nearest, ties to even */
+        return (uint8_t)(sign | (uint8_t)m);  /* m = 8 is the smallest normal, code 0x08 */
+    }
+    int e;
+    double f = frexp(a, &e);                  /* a = f 2^e, f in [0.5, 1) */
+    int E = e - 1;                            /* a = 2^E (1 + frac) */
+    double m = nearbyint((2.0 * f - 1.0) * 8.0);
+    if (m == 8.0) {
+        m = 0.0;
+        E += 1;
+    }
+    return (uint8_t)(sign | (uint8_t)((E + 7) << 3) | (uint8_t)m);
+}
+
+/* Value of an e4m3 code (NaN codes give NaN). */
+double oracle_e4m3_decode(uint8_t c) {
+    int e = (c >> 3) & 0xF, m = c & 7;
+    double v;
+    if ((c & 0x7F) == 0x7F) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* Quantize n bf16 values with one scale: out[x] = e4m3(fp32(value) / scale). */
+void oracle_e4m3_quantize(const uint16_t *in, size_t n, float scale, uint8_t *out) {
+    for (size_t x = 0; x < n; ++x) {
+        float v = (float)bf16_bits_to_double(in[x]);
+        out[x] = oracle_e4m3_encode(v / scale);
+    }
+}
+
+/* Paged KV write into an FP8 cache [num_blocks][2][bs][G][d] of codes:
+ * token t of sequence i goes to position ctx_i + t, K with k_scale[g], V with
+ * v_scale[g].  Nothing else in the pool changes. */
+int oracle_kv_write_fp8(const uint16_t *k, const uint16_t *v, const int32_t *cu_seqlens,
+                        const int32_t *context_lens, int num_seqs, int n_kv_head, int head_dim,
+                        const float *k_scale, const float *v_scale, uint8_t *kv_cache, int num_blocks,
+                        const int32_t *block_table, int max_blocks_per_seq, int block_size) {
+    if (!k || !v || !cu_seqlens || !kv_cache || !block_table || !k_scale || !v_scale || block_size < 1)
+        return ORACLE_ERR_ARG;
+    size_t d = (size_t)head_dim, G = (size_t)n_kv_head;
+    for (int i = 0; i < num_seqs; ++i) {
+        int ctx = context_lens ? context_lens[i] : 0;
+        for (int t = cu_seqlens[i]; t < cu_seqlens[i + 1]; ++t) {
+            int P = ctx + (t - cu_seqlens[i]);
+            int lp = P / block_size;
+            if (lp >= max_blocks_per_seq) return ORACLE_ERR_BLOCK_TABLE;
+            int page = block_table[(size_t)i * max_blocks_per_seq + lp];
+            if (page < 0 || page >= num_blocks) return ORACLE_ERR_BLOCK_TABLE;
+            size_t slot = (size_t)(P % block_size);
+            for (size_t g = 0; g < G; ++g) {
+                uint8_t *kd = kv_cache + ((((size_t)page * 2 + 0) * (size_t)block_size + slot) * G + g) * d;
+                uint8_t *vd = kv_cache + ((((size_t)page * 2 + 1) * (size_t)block_size + slot) * G + g) * d;
+                oracle_e4m3_quantize(k + ((size_t)t * G + g) * d, d, k_scale[g], kd);
+                oracle_e4m3_quantize(v + ((size_t)t * G + g) * d, d, v_scale[g], vd);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Decode over an FP8 cache: the new token of sequence i (q row i, k/v row i)
+ * at position ctx_i attends to the dequantized cache entries 0 .. ctx_i - 1
+ * and to its own K/V quantized the same way (every key the attention sees is
+ * a dequantized cache value).  out[B][n_head][head_dim] in fp64. */
+int oracle_decode_fp8(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *context_lens,
+                      int num_seqs, int n_head, int n_kv_head, int head_dim, double scale, const float *k_scale,
+                      const float *v_scale, const uint8_t *kv_cache, int num_blocks, const int32_t *block_table,
+                      int max_blocks_per_seq, int block_size, double *out) {
+    if (!q || !k || !v || !context_lens || !kv_cache || !block_table || !k_scale || !v_scale || !out)
+        return ORACLE_ERR_ARG;
+    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head || head_dim < 1 || head_dim > 512) return ORACLE_ERR_ARG;
+    int r = n_head / n_kv_head, rc = ORACLE_OK;
+    size_t d = (size_t)head_dim, G = (size_t)n_kv_head;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < num_seqs * n_head; ++u) {
+        int i = u / n_head, h = u % n_head, g = h / r, ctx = context_lens[i];
+        int local = ORACLE_OK;
+        double qd[512], kq[512], vq[512], *w = NULL, *o = out + (size_t)u * d;
+        uint8_t knew[512], vnew[512];
+        for (size_t x = 0; x < d; ++x) qd[x] = bf16_bits_to_double(q[((size_t)i * (size_t)n_head + (size_t)h) * d + x]);
+        oracle_e4m3_quantize(k + ((size_t)i * G + (size_t)g) * d, d, k_scale[g], knew);
+        oracle_e4m3_quantize(v + ((size_t)i * G + (size_t)g) * d, d, v_scale[g], vnew);
+        w = (double *)malloc(sizeof(double) * (size_t)(ctx + 1));
+        if (!w) local = ORACLE_ERR_NOMEM;
+        /* pass 1: scores over keys 0 .. ctx (key ctx = the new token) */
+        double m = -INFINITY;
+        for (int j = 0; j <= ctx && local == ORACLE_OK; ++j) {
+            const uint8_t *kc = knew;
+            if (j < ctx) {
+                int lp = j / block_size, page = lp < max_blocks_per_seq ? block_table[(size_t)i * max_blocks_per_seq + lp] : -1;
+                if (page < 0 || page >= num_blocks) { local = ORACLE_ERR_BLOCK_TABLE; break; }
+                kc = kv_cache + ((((size_t)page * 2 + 0) * (size_t)block_size + (size_t)(j % block_size)) * G + (size_t)g) * d;
+            }
+            for (size_t x = 0; x < d; ++x) kq[x] = oracle_e4m3_decode(kc[x]) * (double)k_scale[g];
+            double dot = 0.0;
+            for (size_t x = 0; x < d; ++x) dot += qd[x] * kq[x];
+            w[j] = scale * dot;
+            if (w[j] > m) m = w[j];
+        }
+        /* pass 2: exponentials, their sum, and the weighted sum of dequantized values */
+        double l = 0.0;
+        for (size_t x = 0; x < d; ++x) o[x] = 0.0;
+        for (int j = 0; j <= ctx && local == ORACLE_OK; ++j) {
+            w[j] = exp(w[j] - m);
+            l += w[j];
+        }
+        for (int j = 0; j <= ctx && local == ORACLE_OK; ++j) {
+            const uint8_t *vc = vnew;
+            if (j < ctx) {
+                int page = block_table[(size_t)i * max_blocks_per_seq + j / block_size];
+                vc = kv_cache + ((((size_t)page * 2 + 1) * (size_t)block_size + (size_t)(j % block_size)) * G + (size_t)g) * d;
+            }
+            for (size_t x = 0; x < d; ++x) vq[x] = oracle_e4m3_decode(vc[x]) * (double)v_scale[g];
+            for (size_t x = 0; x < d; ++x) o[x] += (w[j] / l) * vq[x];
+        }
+        free(w);
+        if (local) {
+#pragma omp critical
+            if (!rc) rc = local;
+        }
+    }
+    return rc;
 }
 
 int oracle_num_threads(void) {

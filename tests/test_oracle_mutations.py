@@ -10,6 +10,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_fp8_pins as fp8pins
 from tests import test_oracle_pins as pins
 
 SRC = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
@@ -37,6 +38,14 @@ MUTANTS = {
     "window_ignored": ("if (p->window > 0 && P - p->window + 1 > 0)", "if (0)"),
     "window_from_chunk_row": ("if (p->window > 0 && P - p->window + 1 > 0) j0 = P - p->window + 1;",
                               "if (p->window > 0 && a - p->window + 1 > 0) j0 = a - p->window + 1;"),
+    "e4m3_bias_off": ("return (uint8_t)(sign | (uint8_t)((E + 7) << 3) | (uint8_t)m);",
+                      "return (uint8_t)(sign | (uint8_t)((E + 6) << 3) | (uint8_t)m);"),
+    "e4m3_ties_away": ("double m = nearbyint((2.0 * f - 1.0) * 8.0);", "double m = round((2.0 * f - 1.0) * 8.0);"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);",
+                           "if (a >= 1e30) return (uint8_t)(sign | 0x7E);"),
+    "fp8_scale_multiplied": ("out[x] = oracle_e4m3_encode(v / scale);", "out[x] = oracle_e4m3_encode(v * scale);"),
+    "fp8_v_scale_on_keys": ("kq[x] = oracle_e4m3_decode(kc[x]) * (double)k_scale[g];",
+                            "kq[x] = oracle_e4m3_decode(kc[x]) * (double)v_scale[g];"),
 }
 
 # pins run against each mutant (the cheap ones; the byte-count pin is run separately)
@@ -55,6 +64,14 @@ PIN_CALLS = [
     lambda: pins.test_window_one_outputs_own_value_exactly(),
     lambda: pins.test_window_matches_torch_sdpa_band_mask([300, 129, 2], 64),
     lambda: pins.test_window_chunk_matches_torch_sdpa_band_mask(),
+    lambda: fp8pins.test_code_table_values(),
+    lambda: fp8pins.test_every_finite_code_round_trips(),
+    lambda: fp8pins.test_midpoints_round_to_the_even_code(),
+    lambda: fp8pins.test_saturation(),
+    lambda: fp8pins.test_kv_write_fp8_bytes_and_untouched_slots(),
+    lambda: fp8pins.test_decode_fp8_empty_context_returns_dequantized_value(),
+    lambda: fp8pins.test_decode_fp8_close_to_bf16_attention(),
+    lambda: fp8pins.test_decode_fp8_equals_bf16_definition_when_values_are_exact(),
 ]
 
 
