@@ -270,8 +270,50 @@ class LibraryMatmul:
 
 QKV_LINE = ("qkv_proj_s8192_h4096_n6144", 8192, 4096, 32, 8, 128, 3001)
 
+class DecodeFp8Runner:
+    """The decode step of DecodeRunner over an FP8 (e4m3) cache: the prompts'
+    K/V quantized into the cache once by kv_cache_store_fp8 (per-kv-head scales
+    from each head's largest magnitude), then paged_decode_attn_fp8.  The
+    algorithmic bytes count one byte per cached element."""
+
+    def __init__(self, base: W.Workload, seed: int, stream):
+        w = W.make_workload([n + 1 for n in base.seqlens], base.n_head, base.n_kv_head, base.head_dim,
+                            block_size=base.block_size, seed=seed)
+        pq, pk, pv, pcu, q, k, v, ctx = W.decode_views(w)
+        d = torch.device("cuda")
+        self.w, self.stream = w, stream
+        self.ks = (torch.cat([pk, k]).float().abs().amax(dim=(0, 2)).clamp(min=1e-6) / 448.0).contiguous().to(d)
+        self.vs = (torch.cat([pv, v]).float().abs().amax(dim=(0, 2)).clamp(min=1e-6) / 448.0).contiguous().to(d)
+        self.cache = torch.zeros((w.num_blocks, 2, w.block_size, w.n_kv_head, w.head_dim), dtype=torch.uint8,
+                                 device=d)
+        self.bt = w.block_table.to(d)
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+        _lib.kv_cache_store_fp8(pk.to(d), pv.to(d), pcu.to(d), None, self.ks, self.vs, self.cache, self.bt,
+                                status=self.status, stream=stream)
+        self.q, self.k, self.v, self.ctx = q.to(d), k.to(d), v.to(d), ctx.to(d)
+        self.max_ctx = int(ctx.max())
+        self.out = torch.empty_like(self.q)
+        B, H, G, D = len(w.seqlens), w.n_head, w.n_kv_head, w.head_dim
+        self.bytes = (int(ctx.sum()) * G * D * 2          # cached K and V codes, read once
+                      + B * H * D * 2 * 2                 # q in, out
+                      + B * G * D * 2 * 2                 # new k, v in
+                      + B * G * D * 2)                    # their codes into the cache
+        self.launches = 2 if -(-(self.max_ctx + 1) // 128) > 1 else 1
+        self.tokens = B
+
+    def step(self):
+        _lib.paged_decode_attn_fp8(self.q, self.k, self.v, self.ctx, self.max_ctx, self.w.scale, self.ks, self.vs,
+                                   self.out, self.cache, self.bt, status=self.status, stream=self.stream)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
+
+
 # secondary line: one decode step after the 64 prompts of the varlen workload
 DECODE_LINE = ("decode64_gqa_h32g8_d128", "varlen64_gqa_h32g8_d128", 2001)
+DECODE_FP8_LINE = ("decode64_fp8_gqa_h32g8_d128", "varlen64_gqa_h32g8_d128", 2001)
 
 
 def time_steps(runner, steps, warmup, stream, flush):
@@ -470,6 +512,16 @@ def main():
                        "frac_of_hbm": round(rx.bytes / (mx * 1e-3) / 1e9 / pk["hbm"], 4),
                        "bytes_per_step": rx.bytes, "tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
                        "launches": rx.launches}
+        del rx
+        torch.cuda.empty_cache()
+        name, base, seed = DECODE_FP8_LINE
+        rx = DecodeFp8Runner(W.named_workload(base), seed, stream)
+        dx = time_steps(rx, max(10, args.steps), 3, stream, flush)
+        mx = statistics.median(dx)
+        extra[name] = {"ms": round(mx, 4), "gbs": round(rx.bytes / (mx * 1e-3) / 1e9, 1),
+                       "frac_of_hbm": round(rx.bytes / (mx * 1e-3) / 1e9 / pk["hbm"], 4),
+                       "bytes_per_step": rx.bytes, "tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
+                       "launches": rx.launches, "kv_format": "e4m3, per-kv-head scales"}
         del rx
         torch.cuda.empty_cache()
 

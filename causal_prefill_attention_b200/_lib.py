@@ -23,7 +23,7 @@ EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall",
             "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
             "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window",
-            "paged_decode_attn", "qkv_projection")
+            "paged_decode_attn", "qkv_projection", "kv_cache_store_fp8", "paged_decode_attn_fp8")
 
 _lib = None
 
@@ -68,6 +68,10 @@ def load() -> ctypes.CDLL:
         lib.paged_decode_attn.restype = I
         lib.qkv_projection.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
         lib.qkv_projection.restype = I
+        lib.kv_cache_store_fp8.argtypes = [P, P, I, P, P, I, I, I, P, P, P, I, P, I, I, P, P]
+        lib.kv_cache_store_fp8.restype = I
+        lib.paged_decode_attn_fp8.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
+        lib.paged_decode_attn_fp8.restype = I
         _lib = lib
     return _lib
 
@@ -221,6 +225,55 @@ def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int, q, k, v,
                                _ptr(k), _ptr(v), _ptr(status), _stream_ptr(stream))
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "qkv_projection")
+    return rc
+
+
+def _check_f32(name, t):
+    if t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous float32 tensor")
+
+
+def _check_u8_cache(t):
+    if t.dtype != torch.uint8 or t.dim() != 5 or not t.is_contiguous():
+        raise ValueError("kv_cache_fp8: expected a contiguous 5-d uint8 tensor")
+
+
+def kv_cache_store_fp8(k, v, cu_seqlens, context_lens, k_scale, v_scale, kv_cache_fp8, block_table,
+                       status: Optional[torch.Tensor] = None, stream=None, raise_on_error: bool = True) -> int:
+    """Quantize a call's K/V rows into their FP8 (e4m3) cache slots (C ABI
+    ``kv_cache_store_fp8``); ``context_lens`` None means every context is 0."""
+    _check_bf16("k", k, 3), _check_bf16("v", v, 3), _check_u8_cache(kv_cache_fp8)
+    _check_i32("cu_seqlens", cu_seqlens), _check_i32("block_table", block_table)
+    _check_f32("k_scale", k_scale), _check_f32("v_scale", v_scale)
+    if context_lens is not None:
+        _check_i32("context_lens", context_lens)
+    T, G, D = k.shape
+    rc = load().kv_cache_store_fp8(
+        _ptr(k), _ptr(v), T, _ptr(cu_seqlens), _ptr(context_lens), cu_seqlens.numel() - 1, G, D, _ptr(k_scale),
+        _ptr(v_scale), _ptr(kv_cache_fp8), kv_cache_fp8.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache_fp8.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "kv_cache_store_fp8")
+    return rc
+
+
+def paged_decode_attn_fp8(q, k, v, context_lens, max_context_len: int, scale: float, k_scale, v_scale, out,
+                          kv_cache_fp8, block_table, status: Optional[torch.Tensor] = None, stream=None,
+                          raise_on_error: bool = True) -> int:
+    """Decode step over an FP8 (e4m3) cache (C ABI ``paged_decode_attn_fp8``)."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3), _check_bf16("out", out, 3)
+    _check_u8_cache(kv_cache_fp8), _check_i32("context_lens", context_lens), _check_i32("block_table", block_table)
+    _check_f32("k_scale", k_scale), _check_f32("v_scale", v_scale)
+    B, H, D = q.shape
+    G = k.shape[1]
+    rc = load().paged_decode_attn_fp8(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(context_lens), B, int(max_context_len), H, G, D, float(scale),
+        _ptr(k_scale), _ptr(v_scale), _ptr(out), _ptr(kv_cache_fp8), kv_cache_fp8.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache_fp8.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "paged_decode_attn_fp8")
     return rc
 
 

@@ -233,12 +233,19 @@ int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, co
                            window);
 }
 
-int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
-                      const int32_t *context_lens, int num_seqs, int max_context_len, int n_head, int n_kv_head,
-                      int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks,
-                      const int32_t *block_table, int max_blocks_per_seq, int block_size, int32_t *status_dev,
-                      prefill_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of paged_decode_attn (bf16 cache) and paged_decode_attn_fp8
+// (e4m3 cache with per-kv-head scales).
+int run_decode(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, const int32_t *context_lens,
+               int num_seqs, int max_context_len, int n_head, int n_kv_head, int head_dim, float scale,
+               prefill_bf16 *out, void *kv_cache, bool fp8, const float *k_scale, const float *v_scale,
+               int num_blocks, const int32_t *block_table, int max_blocks_per_seq, int block_size,
+               int32_t *status_dev, prefill_stream_t stream) {
     if (!q || !k || !v || !context_lens || !out || !kv_cache || !block_table) return PREFILL_ERR_NULL;
+    if (fp8 && (!k_scale || !v_scale)) return PREFILL_ERR_NULL;
     if (num_seqs < 0 || max_context_len < 0) return PREFILL_ERR_SHAPE;
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
     if (n_head / n_kv_head > 16) return PREFILL_ERR_UNSUPPORTED;
@@ -258,7 +265,7 @@ int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefil
     p.k = k;
     p.v = v;
     p.out = out;
-    p.cache = kv_cache;
+    p.cache = fp8 ? nullptr : static_cast<prefill_bf16 *>(kv_cache);
     p.context_lens = context_lens;
     p.block_table = block_table;
     p.status = status_dev;
@@ -283,7 +290,64 @@ int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefil
         p.part_o = reinterpret_cast<float *>(ws);
         p.part_ml = reinterpret_cast<float *>(ws + rows * head_dim * sizeof(float));
     }
-    return pf::launch_decode(p, head_dim, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+    p.cache8 = fp8 ? static_cast<uint8_t *>(kv_cache) : nullptr;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    return pf::launch_decode(p, head_dim, fp8, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                      const int32_t *context_lens, int num_seqs, int max_context_len, int n_head, int n_kv_head,
+                      int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *kv_cache, int num_blocks,
+                      const int32_t *block_table, int max_blocks_per_seq, int block_size, int32_t *status_dev,
+                      prefill_stream_t stream) {
+    return run_decode(q, k, v, context_lens, num_seqs, max_context_len, n_head, n_kv_head, head_dim, scale, out,
+                      kv_cache, false, nullptr, nullptr, num_blocks, block_table, max_blocks_per_seq, block_size,
+                      status_dev, stream);
+}
+
+int paged_decode_attn_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                          const int32_t *context_lens, int num_seqs, int max_context_len, int n_head, int n_kv_head,
+                          int head_dim, float scale, const float *k_scale, const float *v_scale, prefill_bf16 *out,
+                          uint8_t *kv_cache_fp8, int num_blocks, const int32_t *block_table, int max_blocks_per_seq,
+                          int block_size, int32_t *status_dev, prefill_stream_t stream) {
+    return run_decode(q, k, v, context_lens, num_seqs, max_context_len, n_head, n_kv_head, head_dim, scale, out,
+                      kv_cache_fp8, true, k_scale, v_scale, num_blocks, block_table, max_blocks_per_seq, block_size,
+                      status_dev, stream);
+}
+
+int kv_cache_store_fp8(const prefill_bf16 *k, const prefill_bf16 *v, int total_tokens, const int32_t *cu_seqlens,
+                       const int32_t *context_lens, int num_seqs, int n_kv_head, int head_dim, const float *k_scale,
+                       const float *v_scale, uint8_t *kv_cache_fp8, int num_blocks, const int32_t *block_table,
+                       int max_blocks_per_seq, int block_size, int32_t *status_dev, prefill_stream_t stream) {
+    if (!k || !v || !cu_seqlens || !k_scale || !v_scale || !kv_cache_fp8 || !block_table) return PREFILL_ERR_NULL;
+    if (total_tokens < 0 || num_seqs < 0 || n_kv_head < 1) return PREFILL_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (num_blocks < 1 || max_blocks_per_seq < 1) return PREFILL_ERR_BLOCK_TABLE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(kv_cache_fp8)) return PREFILL_ERR_ALIGNMENT;
+    if (total_tokens == 0 || num_seqs == 0) return PREFILL_OK;
+    pf::Fp8StoreParams p;
+    p.k = k;
+    p.v = v;
+    p.cu_seqlens = cu_seqlens;
+    p.context_lens = context_lens;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.cache8 = kv_cache_fp8;
+    p.block_table = block_table;
+    p.status = status_dev;
+    p.total = total_tokens;
+    p.num_seqs = num_seqs;
+    p.n_kv_head = n_kv_head;
+    p.num_blocks = num_blocks;
+    p.mbps = max_blocks_per_seq;
+    p.block_size = block_size;
+    return pf::launch_kv_store_fp8(p, head_dim, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 
 int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int hidden, int n_head, int n_kv_head,

@@ -54,12 +54,17 @@ constexpr int NSTAGE = 3;         // ring stages per warp
 constexpr int kCtasPerSm = 2;
 constexpr float kLazyLog2 = 8.0f; // the running max moves when exceeded by 2^8
 
-template <int D>
+template <int D, bool kFp8>
 struct DecLay {
     static constexpr uint32_t CHUNK = KS * 128;          // 16 rows x 128 bytes (64 columns)
-    static constexpr uint32_t TILE = (D / 64) * CHUNK;   // one K or V step tile
+    static constexpr uint32_t TILE = (D / 64) * CHUNK;   // one K or V step tile (16-bit elements)
     static constexpr uint32_t STAGE = 2 * TILE;          // K then V
-    static constexpr uint32_t WARP_RING = NSTAGE * STAGE;
+    // FP8: the ring holds code rows (16 x D bytes per tensor, unswizzled); each
+    // step widens them into one 16-bit stage (the MMA operand) after the ring
+    static constexpr uint32_t F8TILE = KS * D;
+    static constexpr uint32_t RING_STAGE = kFp8 ? 2 * F8TILE : STAGE;
+    static constexpr uint32_t WIDE = NSTAGE * RING_STAGE;  // the 16-bit stage of the FP8 mode
+    static constexpr uint32_t WARP_RING = NSTAGE * RING_STAGE + (kFp8 ? STAGE : 0);
     static constexpr uint32_t CTX = WARPS * WARP_RING;   // int32 [kDecodeMaxSeqs]: context lengths
     static constexpr uint32_t CUM = CTX + kDecodeMaxSeqs * 4;  // int32 [kDecodeMaxSeqs + 1]: units before sequence i
     static constexpr uint32_t BYTES = CUM + (kDecodeMaxSeqs + 1) * 4;
@@ -84,13 +89,42 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
 }
-// D (16x8 fp32) += A (16x16 bf16, row-major fragment) x B (16x8 bf16, column fragment)
+// D (16x8 fp32) += A (16x16, row-major fragment) x B (16x8, column fragment):
+// bf16 operands, or f16 operands in the FP8 mode
+template <bool kF16>
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    if constexpr (kF16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// two e4m3 codes (low byte first) -> two f16 (exact: f16 holds every e4m3 value)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    uint32_t d;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(d) : "r"(two_codes));
+    return d;
+}
+// e4m3 codes of x0 / s, x1 / s (IEEE division, round to nearest even,
+// saturating at +-448), x0's code in the low byte
+__device__ __forceinline__ uint32_t quant_e4m3x2(float x0, float x1, float s) {
+    const float a = __fdiv_rn(x0, s), b = __fdiv_rn(x1, s);
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
+    return d;
 }
 
 // byte offset of 16-byte slot `s` (0 .. D/8-1) of row `r` (0 .. 15) in a step tile:
@@ -131,9 +165,9 @@ __device__ __forceinline__ bool get_unit(const DecodeParams &p, const int *sctx,
     return true;
 }
 
-template <int D>
+template <int D, bool kFp8>
 __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(const DecodeParams p) {
-    using L = DecLay<D>;
+    using L = DecLay<D, kFp8>;
     constexpr int KSTEPS = D / 16;  // 16-column steps of Q K^T
     constexpr int NT = D / 8;       // 8-column output tiles
     extern __shared__ __align__(128) uint8_t smem[];
@@ -201,7 +235,36 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
     int pg_next = step_page();
     auto issue_next = [&]() {
         if (has_i) {
-            const uint32_t st = ring + (uint32_t)(issued % NSTAGE) * L::STAGE;
+            const uint32_t st = ring + (uint32_t)(issued % NSTAGE) * L::RING_STAGE;
+            if constexpr (kFp8) {
+                // code rows: D / 16 pieces of 16 bytes per row; the new token's row
+                // is zero here and written (quantized) by the compute side
+                constexpr int PPR = D / 16, RPI8 = 32 / PPR;
+                const int lrow = lane / PPR, s16 = lane % PPR;
+                const int p0 = ui.k0 + si * KS;
+                const int ncache = min(ui.k1, ui.ctx) - p0;
+                const bool page_ok = pg_next >= 0 && pg_next < p.num_blocks;
+                const size_t rstride = G * D;  // bytes between consecutive positions of a page
+                const uint8_t *krow0 =
+                    page_ok ? p.cache8 + (((size_t)pg_next * 2 * bs + p0 % bs) * G + ui.g) * D + s16 * 16 : p.cache8;
+                const size_t vhalf = (size_t)bs * rstride;
+#pragma unroll
+                for (int j = 0; j < KS / RPI8; ++j) {
+                    const int row = j * RPI8 + lrow;
+                    const uint8_t *sk = p.cache8;
+                    uint32_t bytes = 0;
+                    if (row < ncache) {
+                        if (page_ok) {
+                            sk = krow0 + (size_t)row * rstride;
+                            bytes = 16;
+                        } else if (s16 == 0) {
+                            report(p.status, PREFILL_ERR_BLOCK_TABLE);  // zero fill
+                        }
+                    }
+                    cp_async16(st + (uint32_t)(row * D + s16 * 16), sk, bytes);
+                    cp_async16(st + L::F8TILE + (uint32_t)(row * D + s16 * 16), bytes ? sk + vhalf : sk, bytes);
+                }
+            } else {
             constexpr int SPR = D / 8;      // 16-byte slots per row
             constexpr int RPI = 32 / SPR;   // rows per copy instruction
             const int lrow = lane / SPR, s = lane % SPR;
@@ -244,6 +307,7 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
                     cp_async16(st + L::TILE + slot_off(row, s), sv, bytes);
                 }
             }
+            }
             ++issued;
             if (++si == ui.nsteps) {
                 has_i = get_unit(p, sctx, scum, ui.u + W, total, ui);
@@ -265,6 +329,11 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             qa[kk][1] = row1 < r ? __ldg(q0 + (row1 * D + c) / 2) : 0u;
             qa[kk][2] = row0 < r ? __ldg(q0 + (row0 * D + c + 8) / 2) : 0u;
             qa[kk][3] = row1 < r ? __ldg(q0 + (row1 * D + c + 8) / 2) : 0u;
+            if constexpr (kFp8) {  // bf16 pairs -> f16 pairs (exact for |q| in f16's normal range)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    qa[kk][e] = pack_f16x2(__uint_as_float(qa[kk][e] << 16), __uint_as_float(qa[kk][e] & 0xffff0000u));
+            }
         }
     };
     Unit uc;
@@ -273,7 +342,7 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
     uint32_t qa[KSTEPS][4], qn[KSTEPS][4];
     if (has_c) load_q(uc, qa);
 
-    const float sl2 = p.scale_log2, thr = kLazyLog2 / sl2;
+    const float sl2_base = p.scale_log2;
     float m_ref[2] = {-CUDART_INF_F, -CUDART_INF_F};  // rows row0, row1
     float l_part[2] = {0.f, 0.f};                       // this lane's share of the row sums
     float o[NT][4];
@@ -284,10 +353,63 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
 
 #pragma unroll 1
     while (has_c) {
+        // the FP8 codes' scales fold into the scores (K) and the output (V)
+        const float sl2 = kFp8 ? sl2_base * __ldg(&p.k_scale[uc.g]) : sl2_base, thr = kLazyLog2 / sl2;
         cp_async_wait<NSTAGE - 2>();  // this step's copies (the oldest group) are done ...
         __syncwarp();                 // ... for every lane, and the previous step is finished
         issue_next();                 // into the stage the previous step used
-        if (sc == 0 && uc.split == uc.nunits - 1 && lane < 2 * (D / 8)) {
+        uint32_t st;
+        if constexpr (kFp8) {
+            const uint32_t f8 = ring + (uint32_t)(computed % NSTAGE) * L::RING_STAGE;
+            uint8_t *f8p = smem + (f8 - smem_u32(smem));
+            const int p0 = uc.k0 + sc * KS;
+            if (uc.ctx >= p0 && uc.ctx < p0 + KS) {
+                // the new token: quantize its K/V into the step's row and into its cache slot
+                const int row = uc.ctx - p0;
+                const int page = __ldg(&p.block_table[(size_t)uc.i * p.mbps + uc.ctx / bs]);
+                const bool page_ok = page >= 0 && page < p.num_blocks;
+                if (!page_ok && lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint16_t *src = (t ? p.v : p.k) + ((size_t)uc.i * G + uc.g) * D;
+                    const float sc_t = __ldg(&(t ? p.v_scale : p.k_scale)[uc.g]);
+                    for (int e = lane * 4; e < D; e += 128) {  // 4 codes per lane
+                        const uint2 x = __ldg(reinterpret_cast<const uint2 *>(src + e));
+                        const uint32_t c01 = quant_e4m3x2(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u), sc_t);
+                        const uint32_t c23 = quant_e4m3x2(__uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u), sc_t);
+                        const uint32_t word = c01 | (c23 << 16);
+                        *reinterpret_cast<uint32_t *>(f8p + t * L::F8TILE + row * D + e) = word;
+                        if (page_ok)
+                            *reinterpret_cast<uint32_t *>(p.cache8 + ((((size_t)page * 2 + t) * bs + uc.ctx % bs) * G + uc.g) * D + e) = word;
+                    }
+                }
+                __syncwarp();
+            }
+            // widen the step's codes into the 16-bit stage (same swizzled layout as the bf16 mode)
+            st = ring + L::WIDE;
+            constexpr int PPR = D / 16;
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int j = 0; j < KS * PPR / 32; ++j) {
+                    const int x = j * 32 + lane, row = x / PPR, s16 = x % PPR;
+                    const uint4 c = *reinterpret_cast<const uint4 *>(f8p + t * L::F8TILE + row * D + s16 * 16);
+                    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+                    uint32_t h[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        h[2 * e] = e4m3x2_to_f16x2(cw[e] & 0xffffu);
+                        h[2 * e + 1] = e4m3x2_to_f16x2(cw[e] >> 16);
+                    }
+                    uint8_t *wide = smem + (st - smem_u32(smem)) + t * L::TILE;
+                    *reinterpret_cast<uint4 *>(wide + slot_off(row, 2 * s16)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4 *>(wide + slot_off(row, 2 * s16 + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
+                }
+            __syncwarp();
+        } else {
+            st = ring + (uint32_t)(computed % NSTAGE) * L::RING_STAGE;
+        }
+        if (!kFp8 && sc == 0 && uc.split == uc.nunits - 1 && lane < 2 * (D / 8)) {
             // the new token's K/V to its slot (position ctx); no unit reads
             // that slot from the cache (the new token comes from the inputs)
             const int page = __ldg(&p.block_table[(size_t)uc.i * p.mbps + uc.ctx / bs]);
@@ -305,7 +427,6 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             Unit un;
             if (get_unit(p, sctx, scum, uc.u + W, total, un)) load_q(un, qn);
         }
-        const uint32_t st = ring + (uint32_t)(computed % NSTAGE) * L::STAGE;
 
         // ---- S = Q K^T for the step's 16 keys (two 8-key tiles)
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -319,10 +440,10 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
                 uint32_t kb[4], kc[4];
                 ldsm_x4(st + slot_off(kr, 2 * kk + (m & 1)), kb);
                 ldsm_x4(st + slot_off(kr, 2 * kk + 2 + (m & 1)), kc);
-                mma16816(s0, qa[kk], kb[0], kb[1]);
-                mma16816(s1, qa[kk], kb[2], kb[3]);
-                mma16816(t0, qa[kk + 1], kc[0], kc[1]);
-                mma16816(t1, qa[kk + 1], kc[2], kc[3]);
+                mma16816<kFp8>(s0, qa[kk], kb[0], kb[1]);
+                mma16816<kFp8>(s1, qa[kk], kb[2], kb[3]);
+                mma16816<kFp8>(t0, qa[kk + 1], kc[0], kc[1]);
+                mma16816<kFp8>(t1, qa[kk + 1], kc[2], kc[3]);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -368,8 +489,18 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
         l_part[0] += (p00 + p01) + (p10 + p11);
         l_part[1] += (p02 + p03) + (p12 + p13);
         // the scores' accumulators are the A fragment of P V (16 rows x 16 keys)
-        const uint32_t pa[4] = {pack_bf16x2(p00, p01), pack_bf16x2(p02, p03), pack_bf16x2(p10, p11),
-                                pack_bf16x2(p12, p13)};
+        uint32_t pa[4];
+        if constexpr (kFp8) {
+            pa[0] = pack_f16x2(p00, p01);
+            pa[1] = pack_f16x2(p02, p03);
+            pa[2] = pack_f16x2(p10, p11);
+            pa[3] = pack_f16x2(p12, p13);
+        } else {
+            pa[0] = pack_bf16x2(p00, p01);
+            pa[1] = pack_bf16x2(p02, p03);
+            pa[2] = pack_bf16x2(p10, p11);
+            pa[3] = pack_bf16x2(p12, p13);
+        }
 
         // ---- O += P V over all output columns, two 8-column tiles per load
         {
@@ -379,8 +510,8 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             for (int c = 0; c < NT / 2; ++c) {
                 uint32_t vb[4];
                 ldsm_x4_t(st + L::TILE + slot_off(vr, 2 * c + (m >> 1)), vb);
-                mma16816(o[2 * c], pa, vb[0], vb[1]);
-                mma16816(o[2 * c + 1], pa, vb[2], vb[3]);
+                mma16816<kFp8>(o[2 * c], pa, vb[0], vb[1]);
+                mma16816<kFp8>(o[2 * c + 1], pa, vb[2], vb[3]);
             }
         }
         ++computed;
@@ -394,6 +525,7 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
         l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
         const bool whole = uc.nunits == 1;
         const size_t hrow = (size_t)uc.i * p.n_head + (size_t)uc.g * r;
+        const float vsc = kFp8 ? __ldg(&p.v_scale[uc.g]) : 1.f;  // the V codes' scale
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int h = hh ? row1 : row0;
@@ -401,7 +533,7 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             const float lsum = hh ? l1 : l0;
             const size_t row = hrow + h;
             if (whole) {
-                const float inv = 1.f / lsum;
+                const float inv = vsc / lsum;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
                     *reinterpret_cast<uint32_t *>(p.out + row * D + nt * 8 + c2) =
@@ -411,7 +543,7 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
                     *reinterpret_cast<float2 *>(p.part_o + prow * D + nt * 8 + c2) =
-                        make_float2(o[nt][2 * hh], o[nt][2 * hh + 1]);
+                        make_float2(o[nt][2 * hh] * vsc, o[nt][2 * hh + 1] * vsc);
                 if ((lane & 3) == 0)
                     *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_ref[hh] * sl2, lsum);
             }
@@ -491,12 +623,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
 }
 
-template <int D>
+template <int D, bool kFp8>
 int launch_d(const DecodeParams &p, void *stream) {
-    using L = DecLay<D>;
+    using L = DecLay<D, kFp8>;
     const size_t smem = L::BYTES;
     cudaError_t e =
-        cudaFuncSetAttribute(paged_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(paged_decode_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -504,7 +636,7 @@ int launch_d(const DecodeParams &p, void *stream) {
     const long long ctas_needed = (units + WARPS - 1) / WARPS;
     const long long slots = (long long)kCtasPerSm * sms;
     const int grid = (int)(ctas_needed < slots ? ctas_needed : slots);
-    paged_decode_kernel<D><<<grid, DTHREADS, smem, (cudaStream_t)stream>>>(p);
+    paged_decode_kernel<D, kFp8><<<grid, DTHREADS, smem, (cudaStream_t)stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.max_units <= 1) return (int)e;
     dim3 cgrid((unsigned)p.num_seqs, (unsigned)cdiv(p.n_head, 4));
@@ -524,9 +656,62 @@ int decode_keys_per_unit(int max_ctx) {
     return u;
 }
 
-int launch_decode(const DecodeParams &p, int head_dim, void *stream) {
-    if (head_dim == 64) return launch_d<64>(p, stream);
-    return launch_d<128>(p, stream);
+int launch_decode(const DecodeParams &p, int head_dim, bool fp8, void *stream) {
+    if (fp8) return head_dim == 64 ? launch_d<64, true>(p, stream) : launch_d<128, true>(p, stream);
+    return head_dim == 64 ? launch_d<64, false>(p, stream) : launch_d<128, false>(p, stream);
+}
+
+namespace {
+
+// One warp per (token, kv head): the K and V rows quantized to e4m3 codes
+// (x / scale, nearest even, saturating) into the token's cache slot.
+template <int D>
+__global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams p) {
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (w >= p.total * p.n_kv_head) return;
+    const int t = w / p.n_kv_head, g = w % p.n_kv_head;
+    int lo = 0, hi = p.num_seqs - 1;  // sequence holding row t: last i with cu_seqlens[i] <= t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(&p.cu_seqlens[mid]) <= t) lo = mid; else hi = mid - 1;
+    }
+    const int i = lo, c0 = __ldg(&p.cu_seqlens[i]);
+    if (t >= __ldg(&p.cu_seqlens[i + 1])) return;  // not a row of any sequence
+    const int pos = (p.context_lens ? __ldg(&p.context_lens[i]) : 0) + (t - c0);
+    const int bs = p.block_size;
+    if (pos < 0 || pos / bs >= p.mbps) {
+        if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+        return;
+    }
+    const int page = __ldg(&p.block_table[(size_t)i * p.mbps + pos / bs]);
+    if (page < 0 || page >= p.num_blocks) {
+        if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+        return;
+    }
+    const size_t G = p.n_kv_head;
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+        const uint16_t *src = (tt ? p.v : p.k) + ((size_t)t * G + g) * D;
+        const float s = __ldg(&(tt ? p.v_scale : p.k_scale)[g]);
+        uint8_t *dst = p.cache8 + ((((size_t)page * 2 + tt) * bs + pos % bs) * G + g) * D;
+        for (int e = lane * 4; e < D; e += 128) {
+            const uint2 x = __ldg(reinterpret_cast<const uint2 *>(src + e));
+            const uint32_t c01 = quant_e4m3x2(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u), s);
+            const uint32_t c23 = quant_e4m3x2(__uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u), s);
+            *reinterpret_cast<uint32_t *>(dst + e) = c01 | (c23 << 16);
+        }
+    }
+}
+
+}  // namespace
+
+int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream) {
+    const long long warps = (long long)p.total * p.n_kv_head;
+    if (warps == 0) return 0;
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (head_dim == 64) kv_store_fp8_kernel<64><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    else kv_store_fp8_kernel<128><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    return (int)cudaGetLastError();
 }
 
 }  // namespace pf

@@ -26,6 +26,10 @@ struct DecodeParams {
     int keys_per_unit;            // keys per work unit (a multiple of the 64-key tile)
     int max_units;                // cdiv(max_ctx + 1, keys_per_unit)
     float scale_log2;             // scale * log2(e)
+    // FP8 (e4m3) cache: codes [NB][2][bs][n_kv_head][D] in cache8 (cache unused);
+    // the value of a code is code_value * k_scale[g] (K) or * v_scale[g] (V)
+    uint8_t *cache8;
+    const float *k_scale, *v_scale;
     // units' partials when a sequence has more than one unit:
     // part_o [max_units][B][n_head][D] (fp32, unnormalised), part_ml [..][2] (max in log2 units, sum)
     float *part_o;
@@ -33,6 +37,19 @@ struct DecodeParams {
 };
 
 int decode_keys_per_unit(int max_ctx);
-int launch_decode(const DecodeParams &p, int head_dim, void *stream);
+int launch_decode(const DecodeParams &p, int head_dim, bool fp8, void *stream);
+
+// FP8 store of a call's K/V rows into their cache slots (decode.cu).
+struct Fp8StoreParams {
+    const uint16_t *k, *v;        // [T][n_kv_head][D]
+    const int32_t *cu_seqlens;    // [B + 1]
+    const int32_t *context_lens;  // [B] or nullptr
+    const float *k_scale, *v_scale;
+    uint8_t *cache8;              // [NB][2][bs][n_kv_head][D]
+    const int32_t *block_table;   // [B][mbps]
+    int32_t *status;
+    int total, num_seqs, n_kv_head, num_blocks, mbps, block_size;
+};
+int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream);
 
 }  // namespace pf

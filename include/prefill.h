@@ -213,6 +213,49 @@ int paged_decode_attn(const prefill_bf16 *q, const prefill_bf16 *k, const prefil
                       int32_t *status_dev, prefill_stream_t stream);
 
 /*
+ * FP8 KV cache (hncyxsy.com/news/227904 §2.3: the KV cache may stay in FP8
+ * while the softmax keeps higher precision; §3.3: 1 byte per element).
+ * Format e4m3 (bias 7, 3 mantissa bits, no infinities, largest finite 448).
+ * The cache has the bf16 cache's layout with one byte per element,
+ * uint8 [num_blocks][2][block_size][n_kv_head][head_dim], and each kv head g
+ * has a K scale and a V scale (device fp32 [n_kv_head], caller-chosen, > 0):
+ * an element x is stored as the code of x / scale (fp32 division, rounded to
+ * the nearest code, ties to even, magnitudes beyond 448 saturated) and read as
+ * code_value * scale.
+ *
+ * kv_cache_store_fp8 -- write a call's K/V rows (k, v [total_tokens][n_kv_head]
+ * [head_dim] bf16, sequences by cu_seqlens, row a of sequence i at position
+ * context_lens[i] + a, context_lens NULL meaning 0) into their FP8 cache slots.
+ * Nothing else in the pool changes.  Argument checks and status codes as for
+ * prefill_attn_chunked.
+ */
+int kv_cache_store_fp8(const prefill_bf16 *k, const prefill_bf16 *v, int total_tokens,
+                       const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                       int n_kv_head, int head_dim, const float *k_scale, const float *v_scale,
+                       uint8_t *kv_cache_fp8, int num_blocks,
+                       const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                       int32_t *status_dev, prefill_stream_t stream);
+
+/*
+ * paged_decode_attn_fp8 -- paged_decode_attn over an FP8 cache: the new token
+ * of sequence i attends to the dequantized codes of positions
+ * 0 .. context_lens[i] - 1 and to its own K/V quantized the same way (every key
+ * and value the attention sees is a dequantized cache value); its codes are
+ * written to its slot.  Softmax and accumulation in fp32; the products run on
+ * f16 tensor-core operands (every e4m3 value is exact in f16; q is rounded to
+ * f16, exact for bf16 values of magnitude 2^-14 .. 65504).  Arguments as for
+ * paged_decode_attn, plus k_scale / v_scale (device fp32 [n_kv_head]).
+ */
+int paged_decode_attn_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                          const int32_t *context_lens, int num_seqs, int max_context_len,
+                          int n_head, int n_kv_head, int head_dim, float scale,
+                          const float *k_scale, const float *v_scale,
+                          prefill_bf16 *out,
+                          uint8_t *kv_cache_fp8, int num_blocks,
+                          const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                          int32_t *status_dev, prefill_stream_t stream);
+
+/*
  * qkv_projection -- the fused QKV projection that feeds prefill_attn
  * (hncyxsy.com/news/270449 §4.1: the W_q, W_k, W_v blocks concatenated into
  * one GEMM that reads the activations once, its output cut by columns into

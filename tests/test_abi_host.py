@@ -23,7 +23,7 @@ def lib():
 def _declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged|qkv)_[a-z_0-9]+)\s*\(", src,
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged|qkv|kv)_[a-z_0-9]+)\s*\(", src,
                                  flags=re.M)))
 
 
@@ -240,3 +240,26 @@ def test_qkv_projection_validation(lib):
     assert call(H=3, G=1, d=64) == 3       # (3 + 2) * 64 = 320 output features: not a multiple of 256
     assert call(q=ctypes.c_void_p(FAKE + 2)) == 7
     assert call(T=0) == 0
+
+
+def test_fp8_entry_points_validation(lib):
+    P = ctypes.c_void_p(FAKE)
+    #       k  v  T   cu ctx B  G  D    ks vs cache nb bt mbps bs  status stream
+    store = [P, P, 10, P, None, 1, 2, 128, P, P, P, 4, P, 4, 16, None, None]
+    # only calls that the host rejects before any launch (the pointers are fake)
+    bad = list(store); bad[8] = None
+    assert lib.kv_cache_store_fp8(*bad) == 1             # no K scale
+    bad = list(store); bad[7] = 96
+    assert lib.kv_cache_store_fp8(*bad) == 3             # head_dim
+    bad = list(store); bad[14] = 24
+    assert lib.kv_cache_store_fp8(*bad) == 3             # block size
+    bad = list(store); bad[10] = ctypes.c_void_p(FAKE + 8)
+    assert lib.kv_cache_store_fp8(*bad) == 7             # cache alignment
+    #      q  k  v  ctx B  maxc H  G  D    scale  ks vs out cache nb bt mbps bs status stream
+    dec = [P, P, P, P, 2, 100, 8, 2, 128, 0.088, P, P, P, P, 16, P, 8, 16, None, None]
+    bad = list(dec); bad[11] = None
+    assert lib.paged_decode_attn_fp8(*bad) == 1          # no V scale
+    bad = list(dec); bad[5] = 128
+    assert lib.paged_decode_attn_fp8(*bad) == 4          # 129 keys do not fit 8 pages of 16
+    bad = list(dec); bad[4] = 0
+    assert lib.paged_decode_attn_fp8(*bad) == 0          # nothing to do
