@@ -59,12 +59,11 @@ struct DecLay {
     static constexpr uint32_t CHUNK = KS * 128;          // 16 rows x 128 bytes (64 columns)
     static constexpr uint32_t TILE = (D / 64) * CHUNK;   // one K or V step tile (16-bit elements)
     static constexpr uint32_t STAGE = 2 * TILE;          // K then V
-    // FP8: the ring holds code rows (16 x D bytes per tensor, unswizzled); each
-    // step widens them into one 16-bit stage (the MMA operand) after the ring
+    // FP8: the ring holds code rows (16 x D bytes per tensor, 16-byte segments
+    // swizzled by row, see f8_off); the MMA operands are widened from them in registers
     static constexpr uint32_t F8TILE = KS * D;
     static constexpr uint32_t RING_STAGE = kFp8 ? 2 * F8TILE : STAGE;
-    static constexpr uint32_t WIDE = NSTAGE * RING_STAGE;  // the 16-bit stage of the FP8 mode
-    static constexpr uint32_t WARP_RING = NSTAGE * RING_STAGE + (kFp8 ? STAGE : 0);
+    static constexpr uint32_t WARP_RING = NSTAGE * RING_STAGE;
     static constexpr uint32_t CTX = WARPS * WARP_RING;   // int32 [kDecodeMaxSeqs]: context lengths
     static constexpr uint32_t CUM = CTX + kDecodeMaxSeqs * 4;  // int32 [kDecodeMaxSeqs + 1]: units before sequence i
     static constexpr uint32_t BYTES = CUM + (kDecodeMaxSeqs + 1) * 4;
@@ -131,6 +130,14 @@ __device__ __forceinline__ uint32_t quant_e4m3x2(float x0, float x1, float s) {
 // 64-column chunks of 16 rows x 128 bytes, slots swizzled by row
 __device__ __forceinline__ uint32_t slot_off(int r, int s) {
     return (uint32_t)(s >> 3) * (KS * 128) + (uint32_t)r * 128 + (uint32_t)(((s & 7) ^ (r & 7)) << 4);
+}
+
+// byte offset of 16-byte segment `s` (0 .. D/16-1) of code row `r` in an FP8
+// step tile: rows of D bytes, segments swizzled by row so that the 8 rows an
+// ldmatrix reads at one segment fall in distinct banks
+template <int D>
+__device__ __forceinline__ uint32_t f8_off(int r, int s) {
+    return (uint32_t)(r * D) + (uint32_t)((s ^ (r & (D / 16 - 1))) << 4);
 }
 
 // A work unit: keys [k0, k1) of sequence i for kv head g (split `split` of
@@ -261,8 +268,8 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
                             report(p.status, PREFILL_ERR_BLOCK_TABLE);  // zero fill
                         }
                     }
-                    cp_async16(st + (uint32_t)(row * D + s16 * 16), sk, bytes);
-                    cp_async16(st + L::F8TILE + (uint32_t)(row * D + s16 * 16), bytes ? sk + vhalf : sk, bytes);
+                    cp_async16(st + f8_off<D>(row, s16), sk, bytes);
+                    cp_async16(st + L::F8TILE + f8_off<D>(row, s16), bytes ? sk + vhalf : sk, bytes);
                 }
             } else {
             constexpr int SPR = D / 8;      // 16-byte slots per row
@@ -324,11 +331,15 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
         const uint32_t *q0 = reinterpret_cast<const uint32_t *>(p.q + ((size_t)u.i * p.n_head + (size_t)u.g * r) * D);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
-            const int c = kk * 16 + c2;
+            // FP8 mode: the 16 columns of a step are permuted (MMA k slots 2j, 2j+1,
+            // 2j+8, 2j+9 <- columns 4j .. 4j+3) to match the K codes' order in the
+            // widened fragments; the dot product does not depend on the order
+            const int c = kFp8 ? kk * 16 + 2 * c2 : kk * 16 + c2;
+            const int c_hi = kFp8 ? c + 2 : c + 8;
             qa[kk][0] = row0 < r ? __ldg(q0 + (row0 * D + c) / 2) : 0u;
             qa[kk][1] = row1 < r ? __ldg(q0 + (row1 * D + c) / 2) : 0u;
-            qa[kk][2] = row0 < r ? __ldg(q0 + (row0 * D + c + 8) / 2) : 0u;
-            qa[kk][3] = row1 < r ? __ldg(q0 + (row1 * D + c + 8) / 2) : 0u;
+            qa[kk][2] = row0 < r ? __ldg(q0 + (row0 * D + c_hi) / 2) : 0u;
+            qa[kk][3] = row1 < r ? __ldg(q0 + (row1 * D + c_hi) / 2) : 0u;
             if constexpr (kFp8) {  // bf16 pairs -> f16 pairs (exact for |q| in f16's normal range)
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
@@ -378,34 +389,14 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
                         const uint32_t c01 = quant_e4m3x2(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u), sc_t);
                         const uint32_t c23 = quant_e4m3x2(__uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u), sc_t);
                         const uint32_t word = c01 | (c23 << 16);
-                        *reinterpret_cast<uint32_t *>(f8p + t * L::F8TILE + row * D + e) = word;
+                        *reinterpret_cast<uint32_t *>(f8p + t * L::F8TILE + f8_off<D>(row, e / 16) + e % 16) = word;
                         if (page_ok)
                             *reinterpret_cast<uint32_t *>(p.cache8 + ((((size_t)page * 2 + t) * bs + uc.ctx % bs) * G + uc.g) * D + e) = word;
                     }
                 }
                 __syncwarp();
             }
-            // widen the step's codes into the 16-bit stage (same swizzled layout as the bf16 mode)
-            st = ring + L::WIDE;
-            constexpr int PPR = D / 16;
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int j = 0; j < KS * PPR / 32; ++j) {
-                    const int x = j * 32 + lane, row = x / PPR, s16 = x % PPR;
-                    const uint4 c = *reinterpret_cast<const uint4 *>(f8p + t * L::F8TILE + row * D + s16 * 16);
-                    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-                    uint32_t h[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        h[2 * e] = e4m3x2_to_f16x2(cw[e] & 0xffffu);
-                        h[2 * e + 1] = e4m3x2_to_f16x2(cw[e] >> 16);
-                    }
-                    uint8_t *wide = smem + (st - smem_u32(smem)) + t * L::TILE;
-                    *reinterpret_cast<uint4 *>(wide + slot_off(row, 2 * s16)) = make_uint4(h[0], h[1], h[2], h[3]);
-                    *reinterpret_cast<uint4 *>(wide + slot_off(row, 2 * s16 + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
-                }
-            __syncwarp();
+            st = f8;
         } else {
             st = ring + (uint32_t)(computed % NSTAGE) * L::RING_STAGE;
         }
@@ -430,7 +421,28 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
 
         // ---- S = Q K^T for the step's 16 keys (two 8-key tiles)
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-        {
+        if constexpr (kFp8) {
+            // matrices: keys 0-7 / 8-15 x segments 2j, 2j+1 of the code rows; a lane
+            // receives 4 consecutive codes of one key: the k slot pairs (2j, 2j+1)
+            // and (2j+8, 2j+9) of the permuted order, one conversion each
+            float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+            const int m = lane >> 3;
+            const int kr = (m & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int j = 0; j < D / 32; ++j) {
+                uint32_t w[4];
+                ldsm_x4(st + f8_off<D>(kr, 2 * j + (m >> 1)), w);
+                mma16816<true>(s0, qa[2 * j], e4m3x2_to_f16x2(w[0] & 0xffffu), e4m3x2_to_f16x2(w[0] >> 16));
+                mma16816<true>(s1, qa[2 * j], e4m3x2_to_f16x2(w[1] & 0xffffu), e4m3x2_to_f16x2(w[1] >> 16));
+                mma16816<true>(t0, qa[2 * j + 1], e4m3x2_to_f16x2(w[2] & 0xffffu), e4m3x2_to_f16x2(w[2] >> 16));
+                mma16816<true>(t1, qa[2 * j + 1], e4m3x2_to_f16x2(w[3] & 0xffffu), e4m3x2_to_f16x2(w[3] >> 16));
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s0[e] += t0[e];
+                s1[e] += t1[e];
+            }
+        } else {
             // four independent accumulation chains (even / odd column steps)
             float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
             const int m = lane >> 3;  // matrices: keys 0-7 / 8-15 x columns +0 / +8
@@ -502,16 +514,36 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             pa[3] = pack_bf16x2(p12, p13);
         }
 
-        // ---- O += P V over all output columns, two 8-column tiles per load
-        {
+        // ---- O += P V over all output columns
+        if constexpr (kFp8) {
+            // transposed matrices: keys 0-7 / 8-15 x segments 2c, 2c+1; a lane receives,
+            // for keys 2j and 2j+1, the codes of columns 16 seg + 2 (lane / 4) and + 1:
+            // bytes 0 and 2 form the pair of the even-column tile, bytes 1 and 3 the
+            // odd one.  o[4c + 2 h + e] holds segment 2c + h, column parity e.
+            const int m = lane >> 3;
+            const int vr = (m & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t w[4];
+                ldsm_x4_t(st + L::F8TILE + f8_off<D>(vr, 2 * c + (m >> 1)), w);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t lo = w[2 * h], hi = w[2 * h + 1];  // keys 0-7, keys 8-15
+                    mma16816<true>(o[4 * c + 2 * h], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0020)),
+                                   e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0020)));
+                    mma16816<true>(o[4 * c + 2 * h + 1], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0031)),
+                                   e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0031)));
+                }
+            }
+        } else {
             const int m = lane >> 3;  // matrices: keys 0-7 / 8-15 x columns +0 / +8
             const int vr = (m & 1) * 8 + (lane & 7);
 #pragma unroll
             for (int c = 0; c < NT / 2; ++c) {
                 uint32_t vb[4];
                 ldsm_x4_t(st + L::TILE + slot_off(vr, 2 * c + (m >> 1)), vb);
-                mma16816<kFp8>(o[2 * c], pa, vb[0], vb[1]);
-                mma16816<kFp8>(o[2 * c + 1], pa, vb[2], vb[3]);
+                mma16816<false>(o[2 * c], pa, vb[0], vb[1]);
+                mma16816<false>(o[2 * c + 1], pa, vb[2], vb[3]);
             }
         }
         ++computed;
@@ -532,7 +564,24 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             if (h >= r) continue;
             const float lsum = hh ? l1 : l0;
             const size_t row = hrow + h;
-            if (whole) {
+            if constexpr (kFp8) {
+                // segment sg: this lane's columns 16 sg + 4 (lane % 4) + 0 .. 3 are the even
+                // tile's two values and the odd tile's two values, interleaved
+                const float f = whole ? vsc / lsum : vsc;
+                const size_t prow = (size_t)uc.split * p.num_seqs * p.n_head + row;  // [unit][seq][head]
+#pragma unroll
+                for (int sg = 0; sg < D / 16; ++sg) {
+                    const float *ev = o[4 * (sg >> 1) + 2 * (sg & 1)], *od = o[4 * (sg >> 1) + 2 * (sg & 1) + 1];
+                    const float v0 = ev[2 * hh] * f, v1 = od[2 * hh] * f, v2 = ev[2 * hh + 1] * f, v3 = od[2 * hh + 1] * f;
+                    const int col = 16 * sg + 2 * c2;
+                    if (whole)
+                        *reinterpret_cast<uint2 *>(p.out + row * D + col) = make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
+                    else
+                        *reinterpret_cast<float4 *>(p.part_o + prow * D + col) = make_float4(v0, v1, v2, v3);
+                }
+                if (!whole && (lane & 3) == 0)
+                    *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_ref[hh] * sl2, lsum);
+            } else if (whole) {
                 const float inv = vsc / lsum;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
