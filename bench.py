@@ -540,6 +540,9 @@ def main():
             "steps": args.steps,
             "warmup": args.warmup,
             "ms_per_step": round(ms, 5),
+            # this rank's per-step CUDA-event times (the value above uses their mean)
+            "step_ms": {"median": round(statistics.median(durs), 5), "min": round(min(durs), 5),
+                        "p90": round(sorted(durs)[min(len(durs) - 1, int(0.9 * len(durs)))], 5)},
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
