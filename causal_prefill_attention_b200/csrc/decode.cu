@@ -25,7 +25,11 @@
 //    queries and never written out.  The running max moves only when a block
 //    max exceeds it by 2^8 (as in the prefill kernel), so O is rarely rescaled;
 //  * a unit's partial (unnormalised O, max, sum) is merged by
-//    decode_combine_kernel when a sequence has more than one unit.
+//    decode_combine_kernel when a sequence has more than one unit;
+//  * FP8 mode (kFp8): the cache holds e4m3 codes with a scale per kv head;
+//    the ring holds code rows and the codes are widened to f16 inside the MMA
+//    fragments (see the Q K^T and P V steps), the scales folded into the
+//    scores and the output; kv_store_fp8_kernel quantizes rows into the cache.
 // Earlier versions for the record: CUDA-core dot products (one FMA per
 // element) issued ~6.5k warp instructions per 64 keys and reached 19 % of the
 // DRAM bandwidth; a CTA-wide version with tensor-core MMAs and three barriers
@@ -50,7 +54,6 @@ constexpr int KS = 16;            // keys per step
 constexpr int WARPS = 4;          // warps (workers) per CTA
 constexpr int DTHREADS = 32 * WARPS;
 constexpr int NSTAGE = 3;         // ring stages per warp
-// sequences per call (their context lengths and unit counts live in shared memory)
 constexpr int kCtasPerSm = 2;
 constexpr float kLazyLog2 = 8.0f; // the running max moves when exceeded by 2^8
 
