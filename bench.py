@@ -300,6 +300,25 @@ class DecodeFp8Runner:
                       + B * G * D * 2)                    # their codes into the cache
         self.launches = 2 if -(-(self.max_ctx + 1) // 128) > 1 else 1
         self.tokens = B
+        self.prompt = (pk.to(d), pv.to(d), pcu.to(d))
+        # bytes of one store of the prompts: bf16 K and V read, their codes written
+        self.store_bytes = int(pk.numel()) * 2 * 2 + int(pk.numel()) * 2
+
+    def time_store(self, reps: int = 5) -> float:
+        """Median ms of kv_cache_store_fp8 over the prompts (it rewrites the same codes)."""
+        pk, pv, pcu = self.prompt
+        ts = []
+        for r in range(reps + 2):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            _lib.kv_cache_store_fp8(pk, pv, pcu, None, self.ks, self.vs, self.cache, self.bt, status=self.status,
+                                    stream=self.stream)
+            b.record(self.stream)
+            torch.cuda.synchronize()
+            if r >= 2:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
 
     def step(self):
         _lib.paged_decode_attn_fp8(self.q, self.k, self.v, self.ctx, self.max_ctx, self.w.scale, self.ks, self.vs,
@@ -522,6 +541,9 @@ def main():
                        "frac_of_hbm": round(rx.bytes / (mx * 1e-3) / 1e9 / pk["hbm"], 4),
                        "bytes_per_step": rx.bytes, "tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
                        "launches": rx.launches, "kv_format": "e4m3, per-kv-head scales"}
+        st_ms = rx.time_store()
+        extra[name]["store_prompts_ms"] = round(st_ms, 4)
+        extra[name]["store_prompts_gbs"] = round(rx.store_bytes / (st_ms * 1e-3) / 1e9, 1)
         del rx
         torch.cuda.empty_cache()
 

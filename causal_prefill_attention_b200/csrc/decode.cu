@@ -715,13 +715,13 @@ int launch_decode(const DecodeParams &p, int head_dim, bool fp8, void *stream) {
 
 namespace {
 
-// One warp per (token, kv head): the K and V rows quantized to e4m3 codes
-// (x / scale, nearest even, saturating) into the token's cache slot.
+// One warp per token: its sequence is found once (binary search over
+// cu_seqlens), then the K and V rows of every kv head are quantized to e4m3
+// codes (x / scale, nearest even, saturating) into the token's cache slot.
 template <int D>
 __global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams p) {
-    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (w >= p.total * p.n_kv_head) return;
-    const int t = w / p.n_kv_head, g = w % p.n_kv_head;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= p.total) return;
     int lo = 0, hi = p.num_seqs - 1;  // sequence holding row t: last i with cu_seqlens[i] <= t
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -741,16 +741,20 @@ __global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams 
         return;
     }
     const size_t G = p.n_kv_head;
+    // the token's rows of all kv heads are contiguous (G * D elements), as are
+    // its slot's codes in the K half and in the V half of the page
+    constexpr int PER = 4;  // elements per lane per step
+    for (int x = lane * PER; x < (int)G * D; x += 32 * PER) {
+        const int g = x / D;
 #pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-        const uint16_t *src = (tt ? p.v : p.k) + ((size_t)t * G + g) * D;
-        const float s = __ldg(&(tt ? p.v_scale : p.k_scale)[g]);
-        uint8_t *dst = p.cache8 + ((((size_t)page * 2 + tt) * bs + pos % bs) * G + g) * D;
-        for (int e = lane * 4; e < D; e += 128) {
-            const uint2 x = __ldg(reinterpret_cast<const uint2 *>(src + e));
-            const uint32_t c01 = quant_e4m3x2(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u), s);
-            const uint32_t c23 = quant_e4m3x2(__uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u), s);
-            *reinterpret_cast<uint32_t *>(dst + e) = c01 | (c23 << 16);
+        for (int tt = 0; tt < 2; ++tt) {
+            const uint16_t *src = (tt ? p.v : p.k) + (size_t)t * G * D + x;
+            const float sc = __ldg(&(tt ? p.v_scale : p.k_scale)[g]);
+            const uint2 v2 = __ldg(reinterpret_cast<const uint2 *>(src));
+            const uint32_t c01 = quant_e4m3x2(__uint_as_float(v2.x << 16), __uint_as_float(v2.x & 0xffff0000u), sc);
+            const uint32_t c23 = quant_e4m3x2(__uint_as_float(v2.y << 16), __uint_as_float(v2.y & 0xffff0000u), sc);
+            uint8_t *dst = p.cache8 + (((size_t)page * 2 + tt) * bs + pos % bs) * G * D + x;
+            *reinterpret_cast<uint32_t *>(dst) = c01 | (c23 << 16);
         }
     }
 }
@@ -758,9 +762,8 @@ __global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams 
 }  // namespace
 
 int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream) {
-    const long long warps = (long long)p.total * p.n_kv_head;
-    if (warps == 0) return 0;
-    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (p.total == 0) return 0;
+    const unsigned grid = (unsigned)((p.total + 7) / 8);  // one warp per token
     if (head_dim == 64) kv_store_fp8_kernel<64><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
     else kv_store_fp8_kernel<128><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
     return (int)cudaGetLastError();
