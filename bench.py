@@ -270,6 +270,58 @@ class LibraryMatmul:
 
 QKV_LINE = ("qkv_proj_s8192_h4096_n6144", 8192, 4096, 32, 8, 128, 3001)
 
+
+class OutProjRunner:
+    """The output projection W_o after the headline attention: o [8192, 32, 128]
+    merged to [8192, 4096] times W_o [4096, 4096]^T (2 M N K FLOP), with cuBLAS
+    (torch.matmul) on the same operands timed beside it."""
+
+    def __init__(self, tokens, H, d, hidden, seed, stream):
+        gen = torch.Generator().manual_seed(seed)
+        dv = torch.device("cuda")
+        self.x = torch.randn(tokens, H, d, generator=gen).to(torch.bfloat16).to(dv)
+        self.w = (torch.randn(hidden, H * d, generator=gen) / math.sqrt(H * d)).to(torch.bfloat16).to(dv)
+        self.y = torch.empty(tokens, hidden, dtype=torch.bfloat16, device=dv)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dv)
+        self.stream = stream
+        self.flops = 2.0 * tokens * H * d * hidden
+        self.launches = 1
+
+    def step(self):
+        _lib.attn_out_projection(self.x, self.w, self.y, status=self.status, stream=self.stream)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
+
+
+class OutProjMatmul(LibraryMatmul):
+    def step(self):
+        torch.matmul(self.r.x.view(self.r.x.shape[0], -1), self.r.w.t())
+
+
+OUT_LINE = ("out_proj_s8192_h4096", 8192, 32, 128, 4096, 3002)
+
+
+class PlainFp8Runner(PlainRunner):
+    """prefill_attn_fp8_cache on a workload: the same attention, the K/V rows
+    written to an FP8 (e4m3) cache with per-kv-head scales (two launches)."""
+
+    def __init__(self, w: W.Workload, stream):
+        super().__init__(w, stream)
+        d = torch.device("cuda")
+        self.cache = torch.zeros(w.num_blocks, 2, w.block_size, w.n_kv_head, w.head_dim, dtype=torch.uint8, device=d)
+        self.k_scale = (w.k.float().abs().amax(dim=(0, 2)).clamp(min=1e-6) / 448.0).to(d)
+        self.v_scale = (w.v.float().abs().amax(dim=(0, 2)).clamp(min=1e-6) / 448.0).to(d)
+        self.launches = 2  # the attention kernel without its cache writer, then the FP8 store
+
+    def step(self):
+        _lib.prefill_attn_fp8_cache(self.q, self.k, self.v, self.cu, self.w.max_seqlen, self.w.scale, self.k_scale,
+                                    self.v_scale, self.out, self.cache, self.bt, status=self.status,
+                                    stream=self.stream)
+
+
 class DecodeFp8Runner:
     """The decode step of DecodeRunner over an FP8 (e4m3) cache: the prompts'
     K/V quantized into the cache once by kv_cache_store_fp8 (per-kv-head scales
@@ -522,6 +574,25 @@ def main():
                        "frac_of_peak": round(rx.flops / (mx * 1e-3) / 1e12 / pk["bf16"], 4),
                        "library_matmul_tflops": round(rx.flops / (ml * 1e-3) / 1e12, 2), "launches": rx.launches}
         del rx
+        torch.cuda.empty_cache()
+        name, T_, H_, d_, hid_, seed_ = OUT_LINE
+        rx = OutProjRunner(T_, H_, d_, hid_, seed_, stream)
+        dx = time_steps(rx, max(10, args.steps), 3, stream, flush)
+        lx = time_steps(OutProjMatmul(rx), max(10, args.steps), 3, stream, flush)
+        mx, ml = statistics.median(dx), statistics.median(lx)
+        extra[name] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
+                       "frac_of_peak": round(rx.flops / (mx * 1e-3) / 1e12 / pk["bf16"], 4),
+                       "library_matmul_tflops": round(rx.flops / (ml * 1e-3) / 1e12, 2), "launches": rx.launches}
+        del rx
+        torch.cuda.empty_cache()
+        wx = W.named_workload(HEADLINE)
+        rx = PlainFp8Runner(wx, stream)
+        dx = time_steps(rx, max(10, args.steps), 3, stream, flush)
+        mx = statistics.median(dx)
+        extra[HEADLINE + "_fp8kv"] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
+                                      "frac_of_peak": round(rx.flops / (mx * 1e-3) / 1e12 / pk["bf16"], 4),
+                                      "launches": rx.launches, "kv_format": "e4m3, per-kv-head scales"}
+        del rx, wx
         torch.cuda.empty_cache()
         name, base, seed = DECODE_LINE
         rx = DecodeRunner(W.named_workload(base), seed, stream)

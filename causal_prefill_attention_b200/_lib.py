@@ -23,7 +23,8 @@ EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_num_kv_blocks", "prefill_kv_block_rule", "prefill_test_inject_stall",
             "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
             "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window",
-            "paged_decode_attn", "qkv_projection", "kv_cache_store_fp8", "paged_decode_attn_fp8")
+            "paged_decode_attn", "qkv_projection", "kv_cache_store_fp8", "paged_decode_attn_fp8",
+            "attn_out_projection", "prefill_attn_fp8_cache")
 
 _lib = None
 
@@ -68,6 +69,10 @@ def load() -> ctypes.CDLL:
         lib.paged_decode_attn.restype = I
         lib.qkv_projection.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
         lib.qkv_projection.restype = I
+        lib.attn_out_projection.argtypes = [P, P, I, I, I, I, P, P, P]
+        lib.attn_out_projection.restype = I
+        lib.prefill_attn_fp8_cache.argtypes = [P, P, P, I, P, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
+        lib.prefill_attn_fp8_cache.restype = I
         lib.kv_cache_store_fp8.argtypes = [P, P, I, P, P, I, I, I, P, P, P, I, P, I, I, P, P]
         lib.kv_cache_store_fp8.restype = I
         lib.paged_decode_attn_fp8.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
@@ -228,6 +233,20 @@ def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int, q, k, v,
     return rc
 
 
+def attn_out_projection(o, w_o, y, status: Optional[torch.Tensor] = None, stream=None,
+                        raise_on_error: bool = True) -> int:
+    """Output projection W_o after the attention (C ABI ``attn_out_projection``):
+    o [T, n_head, d] read as [T, n_head d] (heads merged, head after head),
+    w_o [hidden, n_head d], y [T, hidden] = o w_o^T; bf16, on the tensor cores."""
+    _check_bf16("o", o, 3), _check_bf16("w_o", w_o, 2), _check_bf16("y", y, 2)
+    T, H, D = o.shape
+    rc = load().attn_out_projection(_ptr(o), _ptr(w_o), T, H, D, w_o.shape[0], _ptr(y), _ptr(status),
+                                    _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "attn_out_projection")
+    return rc
+
+
 def _check_f32(name, t):
     if t.dtype != torch.float32 or not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous float32 tensor")
@@ -255,6 +274,26 @@ def kv_cache_store_fp8(k, v, cu_seqlens, context_lens, k_scale, v_scale, kv_cach
         _ptr(status), _stream_ptr(stream))
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "kv_cache_store_fp8")
+    return rc
+
+
+def prefill_attn_fp8_cache(q, k, v, cu_seqlens, max_seqlen: int, scale: float, k_scale, v_scale, out,
+                           kv_cache_fp8, block_table, status: Optional[torch.Tensor] = None, stream=None,
+                           raise_on_error: bool = True) -> int:
+    """prefill_attn writing an FP8 (e4m3) cache (C ABI ``prefill_attn_fp8_cache``):
+    the same attention output, the K/V rows stored as per-kv-head scaled codes."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3), _check_bf16("out", out, 3)
+    _check_u8_cache(kv_cache_fp8), _check_i32("cu_seqlens", cu_seqlens), _check_i32("block_table", block_table)
+    _check_f32("k_scale", k_scale), _check_f32("v_scale", v_scale)
+    T, H, D = q.shape
+    G = k.shape[1]
+    rc = load().prefill_attn_fp8_cache(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1, int(max_seqlen), H, G, D,
+        float(scale), _ptr(k_scale), _ptr(v_scale), _ptr(out), _ptr(kv_cache_fp8), kv_cache_fp8.shape[0],
+        _ptr(block_table), block_table.shape[1] if block_table.dim() == 2 else block_table.numel(),
+        kv_cache_fp8.shape[2], _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "prefill_attn_fp8_cache")
     return rc
 
 

@@ -104,8 +104,10 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
                 const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
                 int n_kv_head, int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *cache, int num_blocks,
                 const int32_t *bt, int mbps, int bs, int32_t *status, prefill_stream_t stream, void *scratch,
-                size_t scratch_bytes, int window) {
-    if (!q || !k || !v || !cu || !out || !cache || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
+                size_t scratch_bytes, int window, uint8_t *cache8, const float *k_scale, const float *v_scale) {
+    if (!q || !k || !v || !cu || !out || !(cache || cache8) || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
+    if (cache8 && (!k_scale || !v_scale)) return PREFILL_ERR_NULL;
+    if (cache8 && (cache || chunked || window > 0)) return PREFILL_ERR_UNSUPPORTED;  // whole prompts only
     if (total < 0 || num_seqs < 0 || max_q < 0 || max_ctx < 0) return PREFILL_ERR_SHAPE;
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
     if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
@@ -118,7 +120,8 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     if (max_ctx > (long long)mbps * bs || max_q > (long long)mbps * bs) return PREFILL_ERR_BLOCK_TABLE;
     if (num_seqs > 65535 || n_head > 65535) return PREFILL_ERR_UNSUPPORTED;
     if ((long long)num_blocks * 2 * bs * n_kv_head * head_dim > (1ll << 40)) return PREFILL_ERR_SHAPE;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cache))
+    const void *pool = cache ? static_cast<const void *>(cache) : static_cast<const void *>(cache8);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pool))
         return PREFILL_ERR_ALIGNMENT;
     if (total == 0 || num_seqs == 0 || max_q == 0) return PREFILL_OK;
 
@@ -140,11 +143,13 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
         if (!encode(&maps.k, k, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
         if (!encode(&maps.v, v, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
-    {
+    if (cache) {
         const cuuint64_t dims[4] = {D, G, (cuuint64_t)bs, (cuuint64_t)num_blocks * 2};
         const cuuint64_t strides[3] = {D * 2, G * D * 2, (cuuint64_t)bs * G * D * 2};
         const cuuint32_t box[4] = {64, 1, (cuuint32_t)bs, 1};
         if (!encode(&maps.cache, cache, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
+    } else {
+        maps.cache = maps.k;  // a valid map the FP8 kernels never use
     }
 
     pf::FwdParams p;
@@ -174,7 +179,9 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     p.part_ml = nullptr;
 
     int e;
-    if (use_pipelined() && pf::fwd_pipelined_supported(p, head_dim)) {
+    const bool pipelined = use_pipelined() && pf::fwd_pipelined_supported(p, head_dim);
+    if (cache8 && !pipelined) return PREFILL_ERR_UNSUPPORTED;  // the FP8 write lives in the pipelined kernel
+    if (pipelined) {
         p.nsplit = pf::fwd_choose_splits(p);
         if (p.nsplit > 1) {
             const size_t o_bytes = (size_t)p.nsplit * p.total * p.n_head * head_dim * sizeof(float);
@@ -189,6 +196,28 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
             }
         }
         e = pf::launch_fwd(maps, p, head_dim, stream);
+        if (e == 0 && cache8) {
+            // FP8 cache: quantize this call's K/V rows into their slots.  A
+            // separate pass: quantizing inside the attention kernel (by its
+            // spare warps, from L2) measured slower than this launch.
+            pf::Fp8StoreParams sp;
+            sp.k = k;
+            sp.v = v;
+            sp.cu_seqlens = cu;
+            sp.context_lens = nullptr;
+            sp.k_scale = k_scale;
+            sp.v_scale = v_scale;
+            sp.cache8 = cache8;
+            sp.block_table = bt;
+            sp.status = status;
+            sp.total = total;
+            sp.num_seqs = num_seqs;
+            sp.n_kv_head = n_kv_head;
+            sp.num_blocks = num_blocks;
+            sp.mbps = mbps;
+            sp.block_size = bs;
+            e = pf::launch_kv_store_fp8(sp, head_dim, stream);
+        }
     } else {
         e = pf::launch_fwd_v0(maps, p, head_dim, stream);
     }
@@ -217,6 +246,17 @@ int prefill_attn_chunked(const prefill_bf16 *q, const prefill_bf16 *k, const pre
     return pf::run_prefill(q, k, v, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len,
                            n_head, n_kv_head, head_dim, scale, out, kv_cache, num_blocks, block_table,
                            max_blocks_per_seq, block_size, status_dev, stream, nullptr, 0);
+}
+
+int prefill_attn_fp8_cache(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_tokens,
+                           const int32_t *cu_seqlens, int num_seqs, int max_seqlen, int n_head, int n_kv_head,
+                           int head_dim, float scale, const float *k_scale, const float *v_scale, prefill_bf16 *out,
+                           uint8_t *kv_cache_fp8, int num_blocks, const int32_t *block_table,
+                           int max_blocks_per_seq, int block_size, int32_t *status_dev, prefill_stream_t stream) {
+    if (!kv_cache_fp8) return PREFILL_ERR_NULL;
+    return pf::run_prefill(q, k, v, total_tokens, cu_seqlens, nullptr, false, num_seqs, max_seqlen, 0, n_head,
+                           n_kv_head, head_dim, scale, out, nullptr, num_blocks, block_table, max_blocks_per_seq,
+                           block_size, status_dev, stream, nullptr, 0, 0, kv_cache_fp8, k_scale, v_scale);
 }
 
 int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,
@@ -350,6 +390,35 @@ int kv_cache_store_fp8(const prefill_bf16 *k, const prefill_bf16 *v, int total_t
     return pf::launch_kv_store_fp8(p, head_dim, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+// y = x w^T on the tcgen05 GEMM: x [M][K], w [N][K] (bf16, K-contiguous), the
+// output columns routed by p (Q | K | V ranges, or one plain output).
+int run_linear(const prefill_bf16 *x, const prefill_bf16 *w, int M, int K, int N, pf::QkvParams &p,
+               prefill_stream_t stream) {
+    CUtensorMap tm_x, tm_w;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M}, strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {64, 128};
+        if (!encode(&tm_x, x, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N}, strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {64, 256};
+        if (!encode(&tm_w, w, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
+    }
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    return pf::launch_qkv_gemm(tm_x, tm_w, p, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
 int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int hidden, int n_head, int n_kv_head,
                    int head_dim, prefill_bf16 *q, prefill_bf16 *k, prefill_bf16 *v, int32_t *status_dev,
                    prefill_stream_t stream) {
@@ -360,28 +429,32 @@ int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int
     if (N % 256 != 0 || N > (1 << 30) || hidden > (1 << 30)) return PREFILL_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PREFILL_ERR_ALIGNMENT;
     if (tokens == 0) return PREFILL_OK;
-    CUtensorMap tm_x, tm_w;
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)tokens}, strides[1] = {(cuuint64_t)hidden * 2};
-        const cuuint32_t box[2] = {64, 128};
-        if (!encode(&tm_x, x, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
-    }
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)N}, strides[1] = {(cuuint64_t)hidden * 2};
-        const cuuint32_t box[2] = {64, 256};
-        if (!encode(&tm_w, w, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
-    }
     pf::QkvParams p;
     p.q = q;
     p.k = k;
     p.v = v;
-    p.M = tokens;
-    p.N = (int)N;
-    p.K = hidden;
     p.hq = n_head * head_dim;
     p.hkv = n_kv_head * head_dim;
     p.status = status_dev;
-    return pf::launch_qkv_gemm(tm_x, tm_w, p, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+    return run_linear(x, w, tokens, hidden, (int)N, p, stream);
+}
+
+int attn_out_projection(const prefill_bf16 *o, const prefill_bf16 *w_o, int tokens, int n_head, int head_dim,
+                        int hidden, prefill_bf16 *y, int32_t *status_dev, prefill_stream_t stream) {
+    if (!o || !w_o || !y) return PREFILL_ERR_NULL;
+    if (tokens < 0 || n_head < 1 || head_dim < 1 || hidden < 1) return PREFILL_ERR_SHAPE;
+    const long long K = (long long)n_head * head_dim;
+    if (K % 64 != 0 || hidden % 256 != 0 || K > (1 << 30) || hidden > (1 << 30)) return PREFILL_ERR_UNSUPPORTED;
+    if (!aligned16(o) || !aligned16(w_o) || !aligned16(y)) return PREFILL_ERR_ALIGNMENT;
+    if (tokens == 0) return PREFILL_OK;
+    pf::QkvParams p;  // one output range: every column goes to y
+    p.q = y;
+    p.k = nullptr;
+    p.v = nullptr;
+    p.hq = hidden;
+    p.hkv = 0;
+    p.status = status_dev;
+    return run_linear(o, w_o, tokens, (int)K, hidden, p, stream);
 }
 
 void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }

@@ -120,14 +120,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
     asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(d) : "r"(two_codes));
     return d;
 }
-// e4m3 codes of x0 / s, x1 / s (IEEE division, round to nearest even,
-// saturating at +-448), x0's code in the low byte
-__device__ __forceinline__ uint32_t quant_e4m3x2(float x0, float x1, float s) {
-    const float a = __fdiv_rn(x0, s), b = __fdiv_rn(x1, s);
-    uint16_t d;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
-    return d;
-}
 
 // byte offset of 16-byte slot `s` (0 .. D/8-1) of row `r` (0 .. 15) in a step tile:
 // 64-column chunks of 16 rows x 128 bytes, slots swizzled by row

@@ -9,7 +9,7 @@ struct FwdParams {
     const uint16_t *k;            // [T][G][D] this call's keys (for the cache write)
     const uint16_t *v;            // [T][G][D]
     uint16_t *out;                // [T][H][D]
-    uint16_t *cache;              // [NB][2][bs][G][D]
+    uint16_t *cache;              // [NB][2][bs][G][D], or nullptr: no cache write (plain prefill only)
     const int32_t *cu_seqlens;    // [B+1]
     const int32_t *context_lens;  // [B] or nullptr (plain prefill)
     const int32_t *block_table;   // [B][mbps]
@@ -55,11 +55,15 @@ int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void
 // Host path shared by the C entry points (api.cu).  scratch / scratch_bytes:
 // caller-supplied split-KV scratch (nullptr: the library's own workspace);
 // a split that needs more than scratch_bytes returns PREFILL_ERR_SCRATCH_LIMIT.
-// window: sliding window of that many keys (0: plain causal).
+// window: sliding window of that many keys (0: plain causal).  cache8 (with
+// k_scale / v_scale): the K/V rows go to this FP8 cache instead of `cache`
+// (plain prefill only; cache is then nullptr): the attention kernel runs
+// without its cache writer and the FP8 store kernel follows on the stream.
 int run_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int total, const int32_t *cu,
                 const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
                 int n_kv_head, int head_dim, float scale, uint16_t *out, uint16_t *cache, int num_blocks,
                 const int32_t *bt, int mbps, int bs, int32_t *status, struct CUstream_st *stream, void *scratch,
-                size_t scratch_bytes, int window = 0);
+                size_t scratch_bytes, int window = 0, uint8_t *cache8 = nullptr, const float *k_scale = nullptr,
+                const float *v_scale = nullptr);
 
 }  // namespace pf

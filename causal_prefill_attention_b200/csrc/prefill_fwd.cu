@@ -17,7 +17,8 @@
 //     paged prefix gather).  Warp 9: tcgen05 MMA issuer.  Warp 10: paged KV
 //     writer, a second consumer of the K/V ring that stores each item's own
 //     K/V tiles from shared memory into their cache pages (TMA stores).
-//     Warp 11: idle.
+//     Warp 11: idle.  A call that writes an FP8 cache runs the kernel
+//     without the writer (kNoWrite) and quantizes K/V in a separate pass.
 //   * TMEM (512 columns): S0 | S1 | O0 | O1, 128 columns each; P (bf16) is
 //     written over the first 64 columns of its S and read by the P.V MMA
 //     directly from TMEM.
@@ -319,8 +320,9 @@ __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
 // The kernel is compiled per mode: kWin runs a sliding window (p.window
 // keys), kChunk reads a cached prefix (p.context_lens).  Without them every
 // window term, and every prefix branch (the context is the constant 0), folds
-// away at compile time.
-constexpr int kModeWindow = 1, kModeChunk = 2;
+// away at compile time.  kNoWrite leaves the cache alone (no writer warp; the
+// K/V ring is released by the MMA warp alone).
+constexpr int kModeWindow = 1, kModeChunk = 2, kModeNoWrite = 4;
 template <bool kWin, bool kChunk>
 __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, const int *start, const uint16_t *perm,
                                             int P, int u_split) {
@@ -394,6 +396,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const FwdParams p, const int P) {
     using L = Lay<D, NST>;
     constexpr bool kWin = (MODE & kModeWindow) != 0, kChunk = (MODE & kModeChunk) != 0;
+    constexpr bool kWrite = (MODE & kModeNoWrite) == 0;
+    static_assert(kWrite || !kChunk, "a chunk's prefix is read from the cache that it appends to");
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
 
@@ -415,7 +419,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        tma_prefetch_desc(&tm_cache);
+        if (kWrite || kChunk) tma_prefetch_desc(&tm_cache);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::B_QFULL + s), 1);
             mbar_init(bar(L::B_QEMPTY + s), 1);
@@ -427,7 +431,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int s = 0; s < NST; ++s) {
             mbar_init(bar(L::B_KVFULL + s), 1);
-            mbar_init(bar(L::B_KVEMPTY + s), 2);  // MMA commit + KV writer
+            mbar_init(bar(L::B_KVEMPTY + s), kWrite ? 2 : 1);  // MMA commit (+ KV writer)
         }
         *abort = 0;
         fence_mbar_init();
@@ -817,7 +821,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
             __syncwarp();
-        } else if (warp == WARP_WRITER) {
+        } else if (kWrite && warp == WARP_WRITER) {
             // ================= paged KV write, fused with the K/V staging: the writer
             // consumes every stage of the ring; the item's own (diagonal) K and V
             // tiles are stored from shared memory straight into their cache pages,
@@ -1016,12 +1020,17 @@ template <int D>
 int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
     const bool nst5 = smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem;
-    const int mode = (p.window > 0 ? kModeWindow : 0) | (p.context_lens ? kModeChunk : 0);
+    const int mode = (p.window > 0 ? kModeWindow : 0) | (p.context_lens ? kModeChunk : 0) |
+                     (p.cache ? 0 : kModeNoWrite);
     switch (mode) {
         case 0: return nst5 ? launch_nst<D, 5, 0>(maps, p, stream) : launch_nst<D, 4, 0>(maps, p, stream);
         case 1: return nst5 ? launch_nst<D, 5, 1>(maps, p, stream) : launch_nst<D, 4, 1>(maps, p, stream);
         case 2: return nst5 ? launch_nst<D, 5, 2>(maps, p, stream) : launch_nst<D, 4, 2>(maps, p, stream);
-        default: return nst5 ? launch_nst<D, 5, 3>(maps, p, stream) : launch_nst<D, 4, 3>(maps, p, stream);
+        case 3: return nst5 ? launch_nst<D, 5, 3>(maps, p, stream) : launch_nst<D, 4, 3>(maps, p, stream);
+        case kModeNoWrite:
+            return nst5 ? launch_nst<D, 5, kModeNoWrite>(maps, p, stream)
+                        : launch_nst<D, 4, kModeNoWrite>(maps, p, stream);
+        default: return (int)cudaErrorInvalidValue;  // no cache with a window or a prefix: not built
     }
 }
 

@@ -6,7 +6,10 @@
 // (s, heads, head_dim), head_dim last.  Here y = x W^T with W stored one row
 // per output feature ([N][hidden], the Q block's rows first), and the
 // epilogue writes the Q, K and V column ranges straight into the [T][H][d] /
-// [T][G][d] tensors the attention call reads.
+// [T][G][d] tensors the attention call reads.  The same kernel runs the
+// output projection W_o after the attention (§3.3: the heads' outputs merged
+// by flattening (s, n_head, head_dim), then one plain GEMM): there every
+// column goes to one output, q = y [T][hidden].
 //
 // Design (a dense contraction: tcgen05 tensor cores):
 //  * persistent grid, one CTA per SM; 128 x 256 output tiles, K in steps of 64;

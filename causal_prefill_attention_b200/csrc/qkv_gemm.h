@@ -1,4 +1,6 @@
-// qkv_gemm.h -- launch parameters of the fused QKV projection (qkv_gemm.cu).
+// qkv_gemm.h -- launch parameters of the projection GEMM (qkv_gemm.cu): the
+// fused QKV projection, and with hq = N, hkv = 0 a plain y = x w^T into q
+// (the attention's output projection W_o).
 #pragma once
 #include <cstdint>
 #include <cstddef>
@@ -10,7 +12,7 @@ struct QkvParams {
     uint16_t *q;        // [M][hq]  = [T][n_head][head_dim]
     uint16_t *k;        // [M][hkv] = [T][n_kv_head][head_dim]
     uint16_t *v;        // [M][hkv]
-    int M, N, K;        // tokens, (n_head + 2 n_kv_head) head_dim, hidden
+    int M, N, K;        // tokens, output features, input features
     int hq, hkv;        // n_head * head_dim, n_kv_head * head_dim
     int32_t *status;    // nullable
 };

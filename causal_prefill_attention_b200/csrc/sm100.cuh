@@ -361,4 +361,14 @@ __device__ __forceinline__ void report(int32_t *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// FP8 (e4m3) cache codes: the codes of x0 / s and x1 / s (IEEE fp32 division,
+// round to nearest even, magnitudes beyond 448 saturated), x0's code in the
+// low byte.
+__device__ __forceinline__ uint32_t quant_e4m3x2(float x0, float x1, float s) {
+    const float a = __fdiv_rn(x0, s), b = __fdiv_rn(x1, s);
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
+    return d;
+}
+
 }  // namespace pf

@@ -256,6 +256,29 @@ int paged_decode_attn_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const pr
                           int32_t *status_dev, prefill_stream_t stream);
 
 /*
+ * prefill_attn_fp8_cache -- prefill_attn writing an FP8 cache: the same
+ * attention over the bf16 inputs (out is what prefill_attn returns), with each
+ * token's K/V rows stored in kv_cache_fp8 as the codes kv_cache_store_fp8
+ * writes (the FP8 format above).  Two launches on `stream`: the attention
+ * kernel without its cache writer, then the FP8 store kernel.  (The pages put
+ * the cache write inside the attention kernel, hncyxsy.com/news/270449 §4.2;
+ * for the bf16 cache that is what prefill_attn does, but quantizing inside the
+ * softmax-bound kernel measured slower than the separate pass.)
+ * Arguments, limits and errors as for prefill_attn, with k_scale / v_scale
+ * (device fp32 [n_kv_head], > 0) and the uint8 pool in place of the bf16 one.
+ * PREFILL_ERR_UNSUPPORTED when the call is beyond the work schedule that the
+ * pipelined kernel keeps in shared memory (more than 4096 sequences, or a
+ * max_seqlen above 524,288), where prefill_attn would run its simple kernel.
+ */
+int prefill_attn_fp8_cache(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                           int total_tokens, const int32_t *cu_seqlens, int num_seqs, int max_seqlen,
+                           int n_head, int n_kv_head, int head_dim, float scale,
+                           const float *k_scale, const float *v_scale,
+                           prefill_bf16 *out, uint8_t *kv_cache_fp8, int num_blocks,
+                           const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                           int32_t *status_dev, prefill_stream_t stream);
+
+/*
  * qkv_projection -- the fused QKV projection that feeds prefill_attn
  * (hncyxsy.com/news/270449 §4.1: the W_q, W_k, W_v blocks concatenated into
  * one GEMM that reads the activations once, its output cut by columns into
@@ -278,6 +301,26 @@ int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int
                    int n_head, int n_kv_head, int head_dim,
                    prefill_bf16 *q, prefill_bf16 *k, prefill_bf16 *v,
                    int32_t *status_dev, prefill_stream_t stream);
+
+/*
+ * attn_out_projection -- the output projection W_o that follows prefill_attn
+ * (hncyxsy.com/news/270449 §3.3: the heads' outputs merged back to (s, h) by
+ * flattening (s, n_head, head_dim), head after head, so that W_o is a plain
+ * GEMM whose input features run in head order; §2.3: it maps the merged
+ * heads to the hidden size).
+ *
+ *   o        device bf16 [tokens][n_head][head_dim] (prefill_attn's out), read as
+ *            [tokens][n_head * head_dim]
+ *   w_o      device bf16 [hidden][n_head * head_dim]: one row per output feature
+ *   y        device, written: bf16 [tokens][hidden]
+ * y = o w_o^T with fp32 accumulation, each output rounded once to bf16 (round to
+ * nearest even).  Requires n_head * head_dim a multiple of 64 and hidden a
+ * multiple of 256 (PREFILL_ERR_UNSUPPORTED otherwise); pointers 16-byte
+ * aligned.  Same tensor-core kernel, limits and error reports as qkv_projection.
+ */
+int attn_out_projection(const prefill_bf16 *o, const prefill_bf16 *w_o, int tokens, int n_head,
+                        int head_dim, int hidden, prefill_bf16 *y,
+                        int32_t *status_dev, prefill_stream_t stream);
 
 /*
  * prefill_attn_chunked_noalloc -- prefill_attn_chunked for callers that cannot

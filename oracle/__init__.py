@@ -219,6 +219,22 @@ def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int):
             y[:, hq + hk:].reshape(T, n_kv_head, head_dim))
 
 
+def out_projection(o, w_o):
+    """The output projection after the attention (hncyxsy.com/news/270449 §3.3:
+    the heads' outputs (s, n_head, head_dim) flattened back to (s, h), head
+    after head, then one GEMM with W_o).
+
+    o: [T, H, d] (any float dtype); w_o: [hidden, H d] bf16, one row per output
+    feature.  Returns y [T, hidden] in fp64: the merge, then the plain product
+    y = o_merged w_o^T in fp64."""
+    os_ = o.detach().cpu().to(torch.float64).numpy() if isinstance(o, torch.Tensor) else np.asarray(o, np.float64)
+    T = os_.shape[0]
+    merged = os_.reshape(T, -1)
+    ws = w_o.detach().cpu().to(torch.float64).numpy()
+    assert ws.shape[1] == merged.shape[1]
+    return merged @ ws.T
+
+
 # ---------------------------------------------------------------- FP8 (e4m3) KV cache
 def e4m3_encode(x: float) -> int:
     """e4m3 code of a float32 value: round to nearest (ties to even), magnitudes

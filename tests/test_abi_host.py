@@ -23,7 +23,7 @@ def lib():
 def _declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged|qkv|kv)_[a-z_0-9]+)\s*\(", src,
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:prefill|paged|qkv|kv|attn)_[a-z_0-9]+)\s*\(", src,
                                  flags=re.M)))
 
 
@@ -242,8 +242,42 @@ def test_qkv_projection_validation(lib):
     assert call(T=0) == 0
 
 
+def test_attn_out_projection_validation(lib):
+    P = ctypes.c_void_p(FAKE)
+    #        o  w  T    H  d    hid  y  status stream
+    base = [P, P, 128, 4, 64, 512, P, None, None]
+
+    def call(**over):
+        a = list(base)
+        names = ["o", "w", "T", "H", "d", "hid", "y"]
+        for key, val in over.items():
+            a[names.index(key)] = val
+        return lib.attn_out_projection(*a)
+
+    assert call(o=None) == 1 and call(y=None) == 1
+    assert call(T=-1) == 2 and call(H=0) == 2 and call(hid=0) == 2
+    assert call(H=3, d=48) == 3            # 144 input features: not a multiple of 64
+    assert call(hid=320) == 3              # hidden not a multiple of 256
+    assert call(w=ctypes.c_void_p(FAKE + 2)) == 7
+    assert call(T=0) == 0
+
+
 def test_fp8_entry_points_validation(lib):
     P = ctypes.c_void_p(FAKE)
+    #      q  k  v  T    cu B  maxs H  G  D    scale  ks vs out cache nb bt mbps bs status stream
+    pre = [P, P, P, 128, P, 1, 128, 4, 2, 128, 0.088, P, P, P, P, 8, P, 8, 16, None, None]
+    bad = list(pre); bad[14] = None
+    assert lib.prefill_attn_fp8_cache(*bad) == 1         # no FP8 pool
+    bad = list(pre); bad[12] = None
+    assert lib.prefill_attn_fp8_cache(*bad) == 1         # no V scale
+    bad = list(pre); bad[9] = 96
+    assert lib.prefill_attn_fp8_cache(*bad) == 3         # head_dim
+    bad = list(pre); bad[18] = 24
+    assert lib.prefill_attn_fp8_cache(*bad) == 3         # block size
+    bad = list(pre); bad[14] = ctypes.c_void_p(FAKE + 4)
+    assert lib.prefill_attn_fp8_cache(*bad) == 7         # pool alignment
+    bad = list(pre); bad[3] = 0
+    assert lib.prefill_attn_fp8_cache(*bad) == 0         # no rows: nothing to do
     #       k  v  T   cu ctx B  G  D    ks vs cache nb bt mbps bs  status stream
     store = [P, P, 10, P, None, 1, 2, 128, P, P, P, 4, P, 4, 16, None, None]
     # only calls that the host rejects before any launch (the pointers are fake)

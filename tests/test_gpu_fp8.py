@@ -58,8 +58,10 @@ def test_store_fp8_matches_oracle_codes(lens, ctxs, G, d, bs):
     _assert_bytes_equal(cache.cpu(), ref, "fp8 pool")
 
 
-def _decode_case(lens, H, G, d, bs=16, seed=0, fill_on_gpu=False):
-    """lens: tokens per sequence including the decode token."""
+def _decode_case(lens, H, G, d, bs=16, seed=0, fill_on_gpu=False, fill_by_prefill=False):
+    """lens: tokens per sequence including the decode token.  The prompts'
+    codes come from the oracle, or from kv_cache_store_fp8 (fill_on_gpu), or
+    from prefill_attn_fp8_cache (fill_by_prefill), checked byte for byte."""
     w = W.make_workload(lens, H, G, d, block_size=bs, seed=seed, extra_pages=2)
     pq, pk, pv, pcu, q, k, v, ctx = W.decode_views(w)
     ks, vs = _scales(torch.cat([pk, k])), _scales(torch.cat([pv, v]))
@@ -75,6 +77,13 @@ def _decode_case(lens, H, G, d, bs=16, seed=0, fill_on_gpu=False):
         _lib.kv_cache_store_fp8(pk.cuda(), pv.cuda(), pcu.cuda(), None, ks_d, vs_d, cache, bt)
         torch.cuda.synchronize()
         _assert_bytes_equal(cache.cpu(), pool, "prompts stored on the GPU")
+    elif fill_by_prefill:
+        cache = _fp8_pool(w).cuda()
+        pout = torch.empty(pq.shape, dtype=torch.bfloat16, device="cuda")
+        _lib.prefill_attn_fp8_cache(pq.cuda(), pk.cuda(), pv.cuda(), pcu.cuda(), max(int(c) for c in ctx) or 1,
+                                    w.scale, ks_d, vs_d, pout, cache, bt)
+        torch.cuda.synchronize()
+        _assert_bytes_equal(cache.cpu(), pool, "prompts written by prefill_attn_fp8_cache")
     else:
         cache = pool.cuda()
     out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -105,3 +114,57 @@ def test_decode_fp8_block_sizes(bs):
 def test_decode_fp8_varlen64_prompts_stored_on_gpu():
     base = W.named_workload("varlen64_gqa_h32g8_d128")
     _decode_case([n + 1 for n in base.seqlens], 32, 8, 128, seed=660, fill_on_gpu=True)
+
+
+def test_decode_fp8_after_fp8_prefill():
+    _decode_case([1, 300, 129, 1000, 2], 8, 2, 128, seed=670, fill_by_prefill=True)
+
+
+# ---------------------------------------------------------------- prefill writing the FP8 cache
+def _prefill_fp8(w: W.Workload, ks, vs):
+    t = U.to_dev(w)
+    cache = _fp8_pool(w).cuda()
+    out = torch.full_like(t["q"], float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _lib.prefill_attn_fp8_cache(t["q"], t["k"], t["v"], t["cu"], w.max_seqlen, w.scale, ks.cuda(), vs.cuda(), out,
+                                cache, t["bt"], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return out.cpu(), cache.cpu()
+
+
+def _check_prefill_fp8(w: W.Workload, full_output: bool, what: str):
+    """The codes byte-exact against the oracle (whole pool, sentinel included),
+    the output against the oracle's attention, and bit-equal to prefill_attn's
+    (the FP8 write leaves the attention arithmetic alone)."""
+    ks, vs = _scales(w.k), _scales(w.v)
+    out, cache = _prefill_fp8(w, ks, vs)
+    ref_pool = oracle.kv_write_fp8(w.k, w.v, w.cu_seqlens, _fp8_pool(w), w.block_table, w.block_size, ks, vs)
+    _assert_bytes_equal(cache, ref_pool, f"{what}: fp8 pool")
+    if full_output:
+        ref = oracle.attention(w.q, w.k, w.v, w.cu_seqlens, w.n_head, w.n_kv_head, w.head_dim, w.scale)
+        U.compare_out(out, ref, what)
+    else:
+        rows, heads = U.sample_rows(w, 96, seed=7)
+        ref = oracle.attention_rows(w.q, w.k, w.v, w.cu_seqlens, w.n_head, w.n_kv_head, w.head_dim, w.scale, rows,
+                                    heads)
+        U.compare_out(out[rows, heads], ref, what)
+    bf16_out, _, st = U.run_prefill(w)
+    assert st == 0
+    assert torch.equal(out.view(torch.int16), bf16_out.view(torch.int16)), f"{what}: output differs from prefill_attn"
+
+
+@pytest.mark.parametrize("lens,H,G,d,bs", [
+    ([37, 5, 300], 4, 2, 128, 16),        # few work items: split-KV
+    ([1000], 8, 2, 64, 32),
+    ([129, 64, 0, 700], 8, 8, 128, 128),  # an empty sequence
+    ([768, 255, 1], 16, 4, 128, 64),
+])
+def test_prefill_fp8_cache_matches_oracle(lens, H, G, d, bs):
+    w = W.make_workload(lens, H, G, d, block_size=bs, seed=680 + sum(lens), extra_pages=3)
+    _check_prefill_fp8(w, True, f"fp8 prefill {lens}")
+
+
+@pytest.mark.parametrize("name", ["gqa_s8192_h32g8_d128", "varlen64_gqa_h32g8_d128"])
+def test_prefill_fp8_cache_full_size(name):
+    _check_prefill_fp8(W.named_workload(name), False, name)

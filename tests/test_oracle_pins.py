@@ -485,3 +485,33 @@ def test_qkv_projection_matches_torch_linear_fp64():
     ref = torch.nn.functional.linear(x.to(torch.float64), w.to(torch.float64)).numpy()
     got = np.concatenate([q.reshape(T, -1), k.reshape(T, -1), v.reshape(T, -1)], axis=1)
     assert np.max(np.abs(got - ref)) < 1e-12
+
+
+# ---------------------------------------------------------------- output projection
+# hncyxsy.com/news/270449 §3.3: the heads' outputs (s, n_head, head_dim) are
+# flattened back to (s, h) head after head, then one plain GEMM with W_o.
+
+def test_out_projection_brute_force_tiny():
+    g = torch.Generator().manual_seed(53)
+    T, H, d, hid = 3, 2, 3, 4
+    o = torch.randn(T, H, d, generator=g).to(torch.bfloat16)
+    w = torch.randn(hid, H * d, generator=g).to(torch.bfloat16)
+    y = oracle.out_projection(o, w)
+    os_, ws = _f64(o), _f64(w)
+    for t in range(T):
+        for n in range(hid):
+            ref = sum(os_[t, h, e] * ws[n, h * d + e] for h in range(H) for e in range(d))
+            assert abs(y[t, n] - ref) < 1e-12
+
+
+def test_out_projection_head_block_selects_that_head():
+    """W_o zero except an identity block under head h's input features: y is
+    head h's output exactly (checks that merged feature h*d + e is (h, e))."""
+    g = torch.Generator().manual_seed(54)
+    T, H, d = 5, 3, 4
+    o = torch.randn(T, H, d, generator=g).to(torch.bfloat16)
+    for h in range(H):
+        w = torch.zeros(d, H * d)
+        w[:, h * d:(h + 1) * d] = torch.eye(d)
+        y = oracle.out_projection(o, w.to(torch.bfloat16))
+        assert np.array_equal(y, _f64(o)[:, h, :])
