@@ -63,6 +63,8 @@ def _configure(lib):
     lib.oracle_kv_write_fp8.restype = I
     lib.oracle_decode_fp8.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, I, I, P]
     lib.oracle_decode_fp8.restype = I
+    lib.oracle_chunked_fp8.argtypes = [P, P, P, P, P, I, I, I, I, D, P, P, P, I, P, I, I, P, P, I, P]
+    lib.oracle_chunked_fp8.restype = I
     return lib
 
 
@@ -286,4 +288,34 @@ def decode_fp8(q, k, v, context_lens, n_head, n_kv_head, head_dim, scale, k_scal
                                    float(scale), _ptr(ks), _ptr(vs), _ptr(cache), int(kv_cache.shape[0]), _ptr(bt),
                                    int(bt.shape[1]), block_size, _ptr(out))
     _check(rc, "oracle_decode_fp8")
+    return out
+
+
+def chunked_fp8(q, k, v, cu_seqlens, context_lens, n_head, n_kv_head, head_dim, scale, k_scale, v_scale, kv_cache,
+                block_table, block_size, *, rows=None, heads=None) -> np.ndarray:
+    """Chunked prefill over an FP8 cache (hncyxsy.com/news/227904 §2.1 chunked
+    prefill, §2.3 an FP8 KV cache with the softmax in higher precision): chunk
+    row a of sequence i at position ctx_i + a attends to the dequantized cache
+    entries 0 .. ctx_i - 1 and to the chunk's rows 0 .. a quantized with the
+    same per-kv-head scales.  q [T, H, d], k/v [T, G, d] bf16; kv_cache uint8
+    [NB, 2, bs, G, d] as it stood before the call.  Returns [T, H, d] fp64, or
+    [n, d] for the selected (packed row, head) pairs."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    cu, ctx, bt = _i32(cu_seqlens), _i32(context_lens), _i32(block_table)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    cache = kv_cache.detach().cpu().contiguous().numpy()
+    T = int(cu[-1])
+    if rows is None:
+        sr = sh = None
+        n_sel = -1
+        out = np.zeros((T, n_head, head_dim), dtype=np.float64)
+    else:
+        sr, sh = _i32(rows), _i32(heads)
+        n_sel = len(sr)
+        out = np.zeros((n_sel, head_dim), dtype=np.float64)
+    rc = _load().oracle_chunked_fp8(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(cu), _ptr(ctx), len(cu) - 1, n_head,
+                                    n_kv_head, head_dim, float(scale), _ptr(ks), _ptr(vs), _ptr(cache),
+                                    int(kv_cache.shape[0]), _ptr(bt), int(bt.shape[1]), block_size, _ptr(sr),
+                                    _ptr(sh), n_sel, _ptr(out))
+    _check(rc, "oracle_chunked_fp8")
     return out

@@ -415,6 +415,108 @@ int oracle_decode_fp8(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
     return rc;
 }
 
+/* Chunked prefill over an FP8 cache: chunk row a of sequence i (packed row
+ * cu_seqlens[i] + a) sits at position ctx_i + a and attends to keys
+ * 0 .. ctx_i + a.  Key j < ctx_i is the dequantized cache entry; key
+ * j >= ctx_i is chunk row j - ctx_i quantized with the same per-kv-head scales
+ * and dequantized, as it is then stored (every key and value the attention
+ * sees is a dequantized cache value).  With one-row chunks this is
+ * oracle_decode_fp8.  The chunk's codes are computed once, before any score.
+ * Outputs for the selected (packed row, head) pairs, or for every pair when
+ * n_sel < 0 (out[T][n_head][head_dim]), in fp64. */
+int oracle_chunked_fp8(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *cu_seqlens,
+                       const int32_t *context_lens, int num_seqs, int n_head, int n_kv_head, int head_dim,
+                       double scale, const float *k_scale, const float *v_scale, const uint8_t *kv_cache,
+                       int num_blocks, const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                       const int32_t *sel_row, const int32_t *sel_head, int n_sel, double *out) {
+    if (!q || !k || !v || !cu_seqlens || !context_lens || !kv_cache || !block_table || !k_scale || !v_scale || !out)
+        return ORACLE_ERR_ARG;
+    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head || head_dim < 1 || head_dim > 512 || block_size < 1)
+        return ORACLE_ERR_ARG;
+    int r = n_head / n_kv_head, rc = ORACLE_OK, T = cu_seqlens[num_seqs];
+    size_t d = (size_t)head_dim, G = (size_t)n_kv_head;
+    /* the chunk's own codes, and the sequence of each packed row */
+    uint8_t *kc8 = (uint8_t *)malloc((size_t)T * G * d + 1), *vc8 = (uint8_t *)malloc((size_t)T * G * d + 1);
+    int *seq_of = (int *)malloc(sizeof(int) * ((size_t)T + 1));
+    if (!kc8 || !vc8 || !seq_of) {
+        free(kc8);
+        free(vc8);
+        free(seq_of);
+        return ORACLE_ERR_NOMEM;
+    }
+    for (int i = 0; i < num_seqs; ++i)
+        for (int t = cu_seqlens[i]; t < cu_seqlens[i + 1]; ++t) {
+            seq_of[t] = i;
+            for (size_t g = 0; g < G; ++g) {
+                oracle_e4m3_quantize(k + ((size_t)t * G + g) * d, d, k_scale[g], kc8 + ((size_t)t * G + g) * d);
+                oracle_e4m3_quantize(v + ((size_t)t * G + g) * d, d, v_scale[g], vc8 + ((size_t)t * G + g) * d);
+            }
+        }
+    int n_pairs = n_sel >= 0 ? n_sel : T * n_head;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < n_pairs; ++u) {
+        int t = n_sel >= 0 ? sel_row[u] : u / n_head, h = n_sel >= 0 ? sel_head[u] : u % n_head;
+        int local = ORACLE_OK;
+        double *o = out + (size_t)u * d;
+        if (t < 0 || t >= T || h < 0 || h >= n_head) {
+            local = ORACLE_ERR_ARG;
+        } else {
+            int i = seq_of[t], g = h / r, ctx = context_lens[i], c0 = cu_seqlens[i];
+            int P = ctx + (t - c0); /* absolute position of the row */
+            double qd[512], kq[512], vq[512], *w = (double *)malloc(sizeof(double) * (size_t)(P + 1));
+            if (!w) local = ORACLE_ERR_NOMEM;
+            for (size_t x = 0; x < d; ++x) qd[x] = bf16_bits_to_double(q[((size_t)t * (size_t)n_head + (size_t)h) * d + x]);
+            /* pass 1: scores over keys 0 .. P */
+            double m = -INFINITY;
+            for (int j = 0; j <= P && local == ORACLE_OK; ++j) {
+                const uint8_t *kc;
+                if (j < ctx) {
+                    int lp = j / block_size;
+                    int page = lp < max_blocks_per_seq ? block_table[(size_t)i * max_blocks_per_seq + lp] : -1;
+                    if (page < 0 || page >= num_blocks) { local = ORACLE_ERR_BLOCK_TABLE; break; }
+                    kc = kv_cache + ((((size_t)page * 2 + 0) * (size_t)block_size + (size_t)(j % block_size)) * G +
+                                     (size_t)g) * d;
+                } else {
+                    kc = kc8 + ((size_t)(c0 + j - ctx) * G + (size_t)g) * d;
+                }
+                for (size_t x = 0; x < d; ++x) kq[x] = oracle_e4m3_decode(kc[x]) * (double)k_scale[g];
+                double dot = 0.0;
+                for (size_t x = 0; x < d; ++x) dot += qd[x] * kq[x];
+                w[j] = scale * dot;
+                if (w[j] > m) m = w[j];
+            }
+            /* pass 2: exponentials, their sum, and the weighted sum of dequantized values */
+            double l = 0.0;
+            for (size_t x = 0; x < d; ++x) o[x] = 0.0;
+            for (int j = 0; j <= P && local == ORACLE_OK; ++j) {
+                w[j] = exp(w[j] - m);
+                l += w[j];
+            }
+            for (int j = 0; j <= P && local == ORACLE_OK; ++j) {
+                const uint8_t *vc;
+                if (j < ctx) {
+                    int page = block_table[(size_t)i * max_blocks_per_seq + j / block_size];
+                    vc = kv_cache + ((((size_t)page * 2 + 1) * (size_t)block_size + (size_t)(j % block_size)) * G +
+                                     (size_t)g) * d;
+                } else {
+                    vc = vc8 + ((size_t)(c0 + j - ctx) * G + (size_t)g) * d;
+                }
+                for (size_t x = 0; x < d; ++x) vq[x] = oracle_e4m3_decode(vc[x]) * (double)v_scale[g];
+                for (size_t x = 0; x < d; ++x) o[x] += (w[j] / l) * vq[x];
+            }
+            free(w);
+        }
+        if (local) {
+#pragma omp critical
+            if (!rc) rc = local;
+        }
+    }
+    free(kc8);
+    free(vc8);
+    free(seq_of);
+    return rc;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

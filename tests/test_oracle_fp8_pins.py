@@ -134,3 +134,97 @@ def test_decode_fp8_close_to_bf16_attention():
                            kv_cache=cache, block_table=w.block_table, block_size=16)
     err = np.abs(out8 - ref)
     assert err.max() < 0.15 and err.mean() < 0.02
+
+
+# ---------------------------------------------------------------- chunked prefill over an FP8 cache
+def _exact_kv(shape, seed):
+    """K with values e4m3 code x 0.125 and V = 2 K (codes x 0.25): quantization
+    with scales 0.125 / 0.25 is exact for them."""
+    gen = torch.Generator().manual_seed(seed)
+    codes = torch.randint(0, 0x7F, shape, generator=gen).reshape(-1).tolist()
+    k = (torch.tensor([oracle.e4m3_decode(int(c)) for c in codes], dtype=torch.float64).reshape(shape) * 0.125)
+    k = k.to(torch.bfloat16)
+    return k, (k.to(torch.float64) * 2.0).to(torch.bfloat16)
+
+
+def _fp8_chunk_case(lens, ctxs, H, G, d, seed, exact=False):
+    """Sequences of ctx + n tokens: the first ctx of each are already in the FP8
+    cache (the oracle's FP8 write), the last n are the call's chunk rows."""
+    w = W.make_workload([c + n for c, n in zip(ctxs, lens)], H, G, d, block_size=16, seed=seed, extra_pages=2)
+    k, v = w.k, w.v
+    if exact:
+        k, v = _exact_kv(tuple(w.k.shape), seed + 1)
+        ks, vs = torch.full((G,), 0.125), torch.full((G,), 0.25)
+    else:
+        ks, vs = torch.linspace(0.01, 0.03, G), torch.linspace(0.02, 0.05, G)
+    starts = w.cu_seqlens.tolist()
+    pre = torch.cat([torch.arange(s, s + c) for s, c in zip(starts, ctxs)]).long()
+    chk = torch.cat([torch.arange(s + c, s + c + n) for s, c, n in zip(starts, ctxs, lens)]).long()
+    pcu = torch.tensor(np.concatenate([[0], np.cumsum(ctxs)]), dtype=torch.int32)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    cache8 = oracle.kv_write_fp8(k[pre], v[pre], pcu, _fp8_cache(w), w.block_table, 16, ks, vs)
+    return dict(w=w, q=w.q[chk], k=k[chk], v=v[chk], cu=cu, ctx=torch.tensor(ctxs, dtype=torch.int32),
+                cache8=cache8, ks=ks, vs=vs, k_all=k, v_all=v, pre=pre, pcu=pcu)
+
+
+def _chunked(c, H, G, d, **kw):
+    return oracle.chunked_fp8(c["q"], c["k"], c["v"], c["cu"], c["ctx"], H, G, d, c["w"].scale, c["ks"], c["vs"],
+                              c["cache8"], c["w"].block_table, 16, **kw)
+
+
+def test_chunked_fp8_one_row_chunks_equal_decode():
+    H, G, d = 4, 2, 16
+    w, pq, pk, pv, pcu, q, k, v, ctx, ks, vs = _decode_inputs([40, 1, 17], H, G, d, seed=65, exact=False)
+    cache8 = oracle.kv_write_fp8(pk, pv, pcu, _fp8_cache(w), w.block_table, 16, ks, vs)
+    B = len(w.seqlens)
+    dec = oracle.decode_fp8(q, k, v, ctx, H, G, d, w.scale, ks, vs, cache8, w.block_table, 16)
+    chk = oracle.chunked_fp8(q, k, v, torch.arange(B + 1, dtype=torch.int32), ctx, H, G, d, w.scale, ks, vs, cache8,
+                             w.block_table, 16)
+    assert np.max(np.abs(dec - chk)) < 1e-12
+
+
+def test_chunked_fp8_exact_values_equal_bf16_definition():
+    """Values that quantize exactly: the chunked FP8 attention equals the bf16
+    chunked definition over a bf16 cache holding the same prefix."""
+    H, G, d = 4, 2, 16
+    c = _fp8_chunk_case([37, 50, 1], [40, 0, 17], H, G, d, seed=66, exact=True)
+    out8 = _chunked(c, H, G, d)
+    cache = oracle.kv_write(c["k_all"][c["pre"]], c["v_all"][c["pre"]], c["pcu"], c["w"].empty_cache(),
+                            c["w"].block_table, 16)
+    ref = oracle.attention(c["q"], c["k"], c["v"], c["cu"], H, G, d, c["w"].scale, context_lens=c["ctx"],
+                           kv_cache=cache, block_table=c["w"].block_table, block_size=16)
+    assert np.max(np.abs(out8 - ref)) < 1e-12
+
+
+def test_chunked_fp8_split_invariance():
+    """One chunk of a sequence, or two chunks with the first one's codes in the
+    cache: the same outputs (a chunk's own keys are quantized as they are stored)."""
+    H, G, d = 4, 2, 16
+    lens, cut = [300, 77], [170, 30]
+    w = W.make_workload(lens, H, G, d, block_size=16, seed=67, extra_pages=2)
+    ks, vs = torch.linspace(0.01, 0.03, G), torch.linspace(0.02, 0.05, G)
+    zero = torch.zeros(2, dtype=torch.int32)
+    whole = oracle.chunked_fp8(w.q, w.k, w.v, w.cu_seqlens, zero, H, G, d, w.scale, ks, vs, _fp8_cache(w),
+                               w.block_table, 16)
+    s = w.cu_seqlens.tolist()
+    first = torch.cat([torch.arange(s[i], s[i] + cut[i]) for i in range(2)]).long()
+    second = torch.cat([torch.arange(s[i] + cut[i], s[i + 1]) for i in range(2)]).long()
+    cu1 = torch.tensor([0, cut[0], sum(cut)], dtype=torch.int32)
+    cu2 = torch.tensor([0, lens[0] - cut[0], sum(lens) - sum(cut)], dtype=torch.int32)
+    out1 = oracle.chunked_fp8(w.q[first], w.k[first], w.v[first], cu1, zero, H, G, d, w.scale, ks, vs, _fp8_cache(w),
+                              w.block_table, 16)
+    cache8 = oracle.kv_write_fp8(w.k[first], w.v[first], cu1, _fp8_cache(w), w.block_table, 16, ks, vs)
+    out2 = oracle.chunked_fp8(w.q[second], w.k[second], w.v[second], cu2, torch.tensor(cut, dtype=torch.int32), H, G,
+                              d, w.scale, ks, vs, cache8, w.block_table, 16)
+    assert np.max(np.abs(out1 - whole[first.numpy()])) < 1e-12
+    assert np.max(np.abs(out2 - whole[second.numpy()])) < 1e-12
+
+
+def test_chunked_fp8_selected_rows_match_full():
+    H, G, d = 4, 2, 16
+    c = _fp8_chunk_case([37, 50], [40, 3], H, G, d, seed=68)
+    full = _chunked(c, H, G, d)
+    rows, heads = [0, 36, 37, 86, 5], [0, 3, 1, 2, 3]
+    sel = _chunked(c, H, G, d, rows=rows, heads=heads)
+    for n, (r, h) in enumerate(zip(rows, heads)):
+        assert np.array_equal(sel[n], full[r, h])

@@ -46,6 +46,14 @@ MUTANTS = {
     "fp8_scale_multiplied": ("out[x] = oracle_e4m3_encode(v / scale);", "out[x] = oracle_e4m3_encode(v * scale);"),
     "fp8_v_scale_on_keys": ("kq[x] = oracle_e4m3_decode(kc[x]) * (double)k_scale[g];",
                             "kq[x] = oracle_e4m3_decode(kc[x]) * (double)v_scale[g];"),
+    "chunk_fp8_top_left_aligned": ("int P = ctx + (t - c0); /* absolute position of the row */",
+                                   "int P = (t - c0); /* absolute position of the row */"),
+    "chunk_fp8_prefix_boundary_off_by_one": ("                if (j < ctx) {\n                    int lp = j / block_size;",
+                                             "                if (j <= ctx) {\n                    int lp = j / block_size;"),
+    "chunk_fp8_values_from_key_codes": ("vc = vc8 + ((size_t)(c0 + j - ctx) * G + (size_t)g) * d;",
+                                        "vc = kc8 + ((size_t)(c0 + j - ctx) * G + (size_t)g) * d;"),
+    "chunk_fp8_keys_quantized_with_v_scale": ("d, k_scale[g], kc8 + ((size_t)t * G + g) * d);",
+                                              "d, v_scale[g], kc8 + ((size_t)t * G + g) * d);"),
 }
 
 # pins run against each mutant (the cheap ones; the byte-count pin is run separately)
@@ -72,6 +80,9 @@ PIN_CALLS = [
     lambda: fp8pins.test_decode_fp8_empty_context_returns_dequantized_value(),
     lambda: fp8pins.test_decode_fp8_close_to_bf16_attention(),
     lambda: fp8pins.test_decode_fp8_equals_bf16_definition_when_values_are_exact(),
+    lambda: fp8pins.test_chunked_fp8_one_row_chunks_equal_decode(),
+    lambda: fp8pins.test_chunked_fp8_exact_values_equal_bf16_definition(),
+    lambda: fp8pins.test_chunked_fp8_split_invariance(),
 ]
 
 
