@@ -168,6 +168,24 @@ class ChunkedRunner:
             raise RuntimeError(f"device status {s}: {_lib.status_string(s)}")
 
 
+class ChunkedFp8Runner(ChunkedRunner):
+    """The chunked workload over an FP8 (e4m3) cache: one prefill_attn_chunked_fp8
+    call per 512-token chunk (FP8 store of the chunk, staging of the dequantized
+    prefix, the bf16 chunked kernel: 3 launches, 4 when the call splits)."""
+
+    def __init__(self, w: W.Workload, chunk: int, stream):
+        super().__init__(w, chunk, stream)
+        d = torch.device("cuda")
+        self.cache = torch.zeros(w.num_blocks, 2, w.block_size, w.n_kv_head, w.head_dim, dtype=torch.uint8, device=d)
+        self.k_scale = (w.k.float().abs().amax(dim=(0, 2)).clamp(min=1e-6) / 448.0).to(d)
+        self.v_scale = (w.v.float().abs().amax(dim=(0, 2)).clamp(min=1e-6) / 448.0).to(d)
+
+    def step(self):
+        for q, k, v, cu, ctx, L, c, out in self.parts:
+            _lib.prefill_attn_chunked_fp8(q, k, v, cu, ctx, L, c, self.w.scale, self.k_scale, self.v_scale, out,
+                                          self.cache, self.bt, status=self.status, stream=self.stream)
+
+
 class WindowRunner(PlainRunner):
     """prefill_attn_sliding_window over one workload; FLOPs counted over the
     visible pairs only (4*d*H per pair, min(a + 1, window) keys for row a)."""
@@ -584,6 +602,20 @@ def main():
                        "frac_of_peak": round(rx.flops / (mx * 1e-3) / 1e12 / pk["bf16"], 4),
                        "library_matmul_tflops": round(rx.flops / (ml * 1e-3) / 1e12, 2), "launches": rx.launches}
         del rx
+        torch.cuda.empty_cache()
+        wx = W.named_workload("chunked512_gqa_s8192_h32g8_d128")
+        try:  # a failure of this secondary line is recorded in it, not raised
+            rx = ChunkedFp8Runner(wx, wx.chunk, stream)
+            dx = time_steps(rx, max(5, args.steps // 2), 3, stream, flush)
+            mx = statistics.median(dx)
+            extra[wx.name + "_fp8kv"] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
+                                         "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
+                                         "calls": len(rx.parts), "launches_per_call": "3 (4 when split)",
+                                         "kv_format": "e4m3, per-kv-head scales"}
+            del rx
+        except Exception as e:
+            extra[wx.name + "_fp8kv"] = {"error": f"{type(e).__name__}: {e}"}
+        del wx
         torch.cuda.empty_cache()
         wx = W.named_workload(HEADLINE)
         rx = PlainFp8Runner(wx, stream)

@@ -24,7 +24,7 @@ EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
             "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window",
             "paged_decode_attn", "qkv_projection", "kv_cache_store_fp8", "paged_decode_attn_fp8",
-            "attn_out_projection", "prefill_attn_fp8_cache")
+            "attn_out_projection", "prefill_attn_fp8_cache", "prefill_attn_chunked_fp8")
 
 _lib = None
 
@@ -73,6 +73,8 @@ def load() -> ctypes.CDLL:
         lib.attn_out_projection.restype = I
         lib.prefill_attn_fp8_cache.argtypes = [P, P, P, I, P, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
         lib.prefill_attn_fp8_cache.restype = I
+        lib.prefill_attn_chunked_fp8.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
+        lib.prefill_attn_chunked_fp8.restype = I
         lib.kv_cache_store_fp8.argtypes = [P, P, I, P, P, I, I, I, P, P, P, I, P, I, I, P, P]
         lib.kv_cache_store_fp8.restype = I
         lib.paged_decode_attn_fp8.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
@@ -294,6 +296,28 @@ def prefill_attn_fp8_cache(q, k, v, cu_seqlens, max_seqlen: int, scale: float, k
         kv_cache_fp8.shape[2], _ptr(status), _stream_ptr(stream))
     if rc != 0 and raise_on_error:
         raise PrefillError(rc, "prefill_attn_fp8_cache")
+    return rc
+
+
+def prefill_attn_chunked_fp8(q, k, v, cu_seqlens_q, context_lens, max_q_len: int, max_context_len: int,
+                             scale: float, k_scale, v_scale, out, kv_cache_fp8, block_table,
+                             status: Optional[torch.Tensor] = None, stream=None, raise_on_error: bool = True) -> int:
+    """Chunked prefill over an FP8 (e4m3) cache (C ABI ``prefill_attn_chunked_fp8``):
+    each chunk attends to its dequantized cached prefix and to its own rows
+    quantized the same way, then its codes are appended."""
+    _check_bf16("q", q, 3), _check_bf16("k", k, 3), _check_bf16("v", v, 3), _check_bf16("out", out, 3)
+    _check_u8_cache(kv_cache_fp8), _check_i32("cu_seqlens_q", cu_seqlens_q), _check_i32("context_lens", context_lens)
+    _check_i32("block_table", block_table), _check_f32("k_scale", k_scale), _check_f32("v_scale", v_scale)
+    T, H, D = q.shape
+    G = k.shape[1]
+    rc = load().prefill_attn_chunked_fp8(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(cu_seqlens_q), _ptr(context_lens), cu_seqlens_q.numel() - 1,
+        int(max_q_len), int(max_context_len), H, G, D, float(scale), _ptr(k_scale), _ptr(v_scale), _ptr(out),
+        _ptr(kv_cache_fp8), kv_cache_fp8.shape[0], _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else block_table.numel(), kv_cache_fp8.shape[2],
+        _ptr(status), _stream_ptr(stream))
+    if rc != 0 and raise_on_error:
+        raise PrefillError(rc, "prefill_attn_chunked_fp8")
     return rc
 
 

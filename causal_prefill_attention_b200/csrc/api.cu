@@ -11,6 +11,7 @@
 #include <atomic>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "../../include/prefill.h"
@@ -62,21 +63,24 @@ bool use_pipelined() {
 
 std::atomic<int> g_test_stall{0};
 
-// Split-KV workspace: one device buffer per (device, stream), allocated on the
-// first call that splits and grown when a larger call needs more.  Kept for
+// Device workspaces: one buffer per (device, stream, kind), allocated on the
+// first call that needs it and grown when a larger call needs more.  Kept for
 // later calls; a separate buffer per stream keeps concurrent streams apart.
+// Kinds: the split-KV partials, and the staging of a chunked prefill over an
+// FP8 cache (which then also uses the split-KV partials).
+enum WorkspaceKind { kSplitPartials = 0, kFp8Staging = 1 };
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
 };
 std::mutex g_ws_mu;
-std::map<std::pair<int, void *>, Workspace> g_ws;
+std::map<std::tuple<int, void *, int>, Workspace> g_ws;
 
-void *split_workspace(size_t bytes, void *stream) {
+void *device_workspace(int kind, size_t bytes, void *stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
     std::lock_guard<std::mutex> lock(g_ws_mu);
-    Workspace &w = g_ws[{dev, stream}];
+    Workspace &w = g_ws[std::make_tuple(dev, stream, kind)];
     if (w.bytes < bytes) {
         if (w.ptr) {
             cudaStreamSynchronize(static_cast<cudaStream_t>(stream));  // earlier calls may still read it
@@ -93,6 +97,8 @@ void *split_workspace(size_t bytes, void *stream) {
     }
     return w.ptr;
 }
+
+void *split_workspace(size_t bytes, void *stream) { return device_workspace(kSplitPartials, bytes, stream); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -257,6 +263,94 @@ int prefill_attn_fp8_cache(const prefill_bf16 *q, const prefill_bf16 *k, const p
     return pf::run_prefill(q, k, v, total_tokens, cu_seqlens, nullptr, false, num_seqs, max_seqlen, 0, n_head,
                            n_kv_head, head_dim, scale, out, nullptr, num_blocks, block_table, max_blocks_per_seq,
                            block_size, status_dev, stream, nullptr, 0, 0, kv_cache_fp8, k_scale, v_scale);
+}
+
+int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,
+                             const int32_t *cu_seqlens_q, const int32_t *context_lens, int num_seqs, int max_q_len,
+                             int max_context_len, int n_head, int n_kv_head, int head_dim, float scale,
+                             const float *k_scale, const float *v_scale, prefill_bf16 *out, uint8_t *kv_cache_fp8,
+                             int num_blocks, const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                             int32_t *status_dev, prefill_stream_t stream) {
+    if (!q || !k || !v || !cu_seqlens_q || !context_lens || !k_scale || !v_scale || !out || !kv_cache_fp8 ||
+        !block_table)
+        return PREFILL_ERR_NULL;
+    if (total_q < 0 || num_seqs < 0 || max_q_len < 0 || max_context_len < 0) return PREFILL_ERR_SHAPE;
+    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return PREFILL_ERR_UNSUPPORTED;
+    if (!(std::isfinite(scale) && scale > 0.f)) return PREFILL_ERR_UNSUPPORTED;
+    if (num_blocks < 1 || max_blocks_per_seq < 1) return PREFILL_ERR_BLOCK_TABLE;
+    // each bound must fit the table (the exact per-sequence check, context +
+    // chunk length, runs on the device, where the lengths are)
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size ||
+        (long long)max_q_len > (long long)max_blocks_per_seq * block_size)
+        return PREFILL_ERR_BLOCK_TABLE;
+    const long long span = (long long)max_context_len + max_q_len;  // bound on every context + chunk length
+    if (num_seqs > 65535 || n_head > 65535 || span > (1 << 30)) return PREFILL_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * 2 * block_size * n_kv_head * head_dim > (1ll << 40)) return PREFILL_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kv_cache_fp8))
+        return PREFILL_ERR_ALIGNMENT;
+    if (total_q == 0 || num_seqs == 0 || max_q_len == 0) return PREFILL_OK;
+
+    // staging: the bf16 shadow pool (mbps2 pages per sequence), k2 / v2, the shadow table
+    const int mbps2 = (int)((span + block_size - 1) / block_size);
+    if ((long long)num_seqs * mbps2 >= (1ll << 30)) return PREFILL_ERR_UNSUPPORTED;
+    const size_t row = (size_t)n_kv_head * head_dim * 2;  // bytes of one token's K (or V) row in bf16
+    const size_t shadow_bytes = (size_t)num_seqs * mbps2 * 2 * block_size * row;
+    const size_t kv2_bytes = (size_t)total_q * row;
+    const size_t table_bytes = (size_t)num_seqs * mbps2 * sizeof(int32_t);
+    char *ws = static_cast<char *>(device_workspace(kFp8Staging, shadow_bytes + 2 * kv2_bytes + table_bytes, stream));
+    if (!ws) return PREFILL_ERR_CUDA;
+    prefill_bf16 *shadow = reinterpret_cast<prefill_bf16 *>(ws);
+    prefill_bf16 *k2 = reinterpret_cast<prefill_bf16 *>(ws + shadow_bytes);
+    prefill_bf16 *v2 = reinterpret_cast<prefill_bf16 *>(ws + shadow_bytes + kv2_bytes);
+    int32_t *table2 = reinterpret_cast<int32_t *>(ws + shadow_bytes + 2 * kv2_bytes);
+
+    // 1. the chunk's codes into the FP8 cache
+    pf::Fp8StoreParams sp;
+    sp.k = k;
+    sp.v = v;
+    sp.cu_seqlens = cu_seqlens_q;
+    sp.context_lens = context_lens;
+    sp.k_scale = k_scale;
+    sp.v_scale = v_scale;
+    sp.cache8 = kv_cache_fp8;
+    sp.block_table = block_table;
+    sp.status = status_dev;
+    sp.total = total_q;
+    sp.num_seqs = num_seqs;
+    sp.n_kv_head = n_kv_head;
+    sp.num_blocks = num_blocks;
+    sp.mbps = max_blocks_per_seq;
+    sp.block_size = block_size;
+    if (pf::launch_kv_store_fp8(sp, head_dim, stream) != 0) return PREFILL_ERR_CUDA;
+    // 2. every key and value the chunk attends to, dequantized from the cache
+    pf::Fp8StageParams gp;
+    gp.cache8 = kv_cache_fp8;
+    gp.block_table = block_table;
+    gp.cu_seqlens = cu_seqlens_q;
+    gp.context_lens = context_lens;
+    gp.k_scale = k_scale;
+    gp.v_scale = v_scale;
+    gp.shadow = shadow;
+    gp.shadow_table = table2;
+    gp.k2 = k2;
+    gp.v2 = v2;
+    gp.status = status_dev;
+    gp.total = total_q;
+    gp.num_seqs = num_seqs;
+    gp.n_kv_head = n_kv_head;
+    gp.num_blocks = num_blocks;
+    gp.mbps = max_blocks_per_seq;
+    gp.block_size = block_size;
+    gp.mbps2 = mbps2;
+    gp.max_span = (int)span;
+    if (pf::launch_fp8_stage(gp, head_dim, stream) != 0) return PREFILL_ERR_CUDA;
+    // 3. the bf16 chunked attention over the staged rows (it also writes k2 / v2
+    //    into the shadow pool, which is scratch)
+    return pf::run_prefill(q, k2, v2, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len,
+                           n_head, n_kv_head, head_dim, scale, out, shadow, num_seqs * mbps2, table2, mbps2,
+                           block_size, status_dev, stream, nullptr, 0);
 }
 
 int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,

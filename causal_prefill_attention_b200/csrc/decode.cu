@@ -751,7 +751,73 @@ __global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams 
     }
 }
 
+// the two f16 halves of a word as fp32 (exact), the low half first
+__device__ __forceinline__ void f16x2_to_f32(uint32_t h, float &lo, float &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h));
+}
+
+// One warp per (sequence, position): the K and V code rows of every kv head
+// (G * D bytes each, contiguous in the slot) are widened exactly to f16, scaled
+// in fp32 and rounded to bf16, 8 elements per lane step.
+template <int D>
+__global__ void __launch_bounds__(256) fp8_stage_kernel(const Fp8StageParams p) {
+    const int i = blockIdx.y, lane = threadIdx.x & 31;
+    const int pos = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (blockIdx.x == 0)
+        for (int x = threadIdx.x; x < p.mbps2; x += blockDim.x) p.shadow_table[(size_t)i * p.mbps2 + x] = i * p.mbps2 + x;
+    const int c0 = __ldg(&p.cu_seqlens[i]), n = __ldg(&p.cu_seqlens[i + 1]) - c0;
+    const int ctx = __ldg(&p.context_lens[i]);
+    const int bs = p.block_size;
+    if (pos >= p.max_span) return;
+    if (n < 0 || c0 < 0 || c0 + n > p.total || ctx < 0 || (long long)ctx + n > p.max_span) {
+        if (pos == 0 && lane == 0) report(p.status, PREFILL_ERR_SHAPE);
+        return;
+    }
+    if (pos >= ctx + n) return;
+    if (pos / bs >= p.mbps) {
+        if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+        return;
+    }
+    const int page = __ldg(&p.block_table[(size_t)i * p.mbps + pos / bs]);
+    if (page < 0 || page >= p.num_blocks) {
+        if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+        return;
+    }
+    const size_t G = p.n_kv_head, row = G * D;
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+        const uint8_t *src = p.cache8 + (((size_t)page * 2 + tt) * bs + pos % bs) * row;
+        uint16_t *dst = pos < ctx
+            ? p.shadow + ((((size_t)i * p.mbps2 + pos / bs) * 2 + tt) * bs + pos % bs) * row
+            : (tt ? p.v2 : p.k2) + (size_t)(c0 + pos - ctx) * row;
+        const float *sc = tt ? p.v_scale : p.k_scale;
+        for (int x = lane * 8; x < (int)row; x += 32 * 8) {
+            const float s = __ldg(&sc[x / D]);
+            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(src + x));
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t two = ((e < 2 ? c.x : c.y) >> (16 * (e & 1))) & 0xffffu;
+                float lo, hi;
+                f16x2_to_f32(e4m3x2_to_f16x2(two), lo, hi);
+                w[e] = pack_bf16x2(lo * s, hi * s);
+            }
+            *reinterpret_cast<uint4 *>(dst + x) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
 }  // namespace
+
+int launch_fp8_stage(const Fp8StageParams &p, int head_dim, void *stream) {
+    if (p.num_seqs == 0 || p.max_span == 0) return 0;
+    const dim3 grid((unsigned)((p.max_span + 7) / 8), (unsigned)p.num_seqs);
+    if (head_dim == 64) fp8_stage_kernel<64><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    else fp8_stage_kernel<128><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    return (int)cudaGetLastError();
+}
 
 int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream) {
     if (p.total == 0) return 0;

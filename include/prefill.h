@@ -279,6 +279,34 @@ int prefill_attn_fp8_cache(const prefill_bf16 *q, const prefill_bf16 *k, const p
                            int32_t *status_dev, prefill_stream_t stream);
 
 /*
+ * prefill_attn_chunked_fp8 -- prefill_attn_chunked over an FP8 cache
+ * (hncyxsy.com/news/227904 §2.1 chunked prefill; §2.3 the KV cache in FP8
+ * with the softmax at higher precision).  Chunk row a of sequence i sits at
+ * position context_lens[i] + a and attends to keys 0 .. context_lens[i] + a,
+ * every one of them a dequantized cache value: the cached prefix's codes, and
+ * the chunk's own K/V rows quantized with the same scales, as they are stored.
+ * The chunk's codes are appended to kv_cache_fp8 (as kv_cache_store_fp8 writes
+ * them).  Arguments, limits and errors as for prefill_attn_chunked, with
+ * k_scale / v_scale (device fp32 [n_kv_head], > 0) and the uint8 pool.
+ *
+ * Three launches on `stream`: the FP8 store of the chunk, a staging kernel that
+ * dequantizes (code value x scale, rounded to bf16) every position the chunk
+ * attends to into a bf16 workspace, and the bf16 chunked attention over it.
+ * The workspace -- num_seqs x ceil((max_context_len + max_q_len) / block_size)
+ * bf16 pages, plus 2 x total_q x n_kv_head x head_dim bf16 -- is allocated
+ * like the split-KV workspace (first call per device and stream, grown when
+ * needed, kept); PREFILL_ERR_CUDA if that allocation fails.
+ */
+int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
+                             int total_q, const int32_t *cu_seqlens_q, const int32_t *context_lens,
+                             int num_seqs, int max_q_len, int max_context_len,
+                             int n_head, int n_kv_head, int head_dim, float scale,
+                             const float *k_scale, const float *v_scale,
+                             prefill_bf16 *out, uint8_t *kv_cache_fp8, int num_blocks,
+                             const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                             int32_t *status_dev, prefill_stream_t stream);
+
+/*
  * qkv_projection -- the fused QKV projection that feeds prefill_attn
  * (hncyxsy.com/news/270449 §4.1: the W_q, W_k, W_v blocks concatenated into
  * one GEMM that reads the activations once, its output cut by columns into

@@ -278,6 +278,22 @@ def test_fp8_entry_points_validation(lib):
     assert lib.prefill_attn_fp8_cache(*bad) == 7         # pool alignment
     bad = list(pre); bad[3] = 0
     assert lib.prefill_attn_fp8_cache(*bad) == 0         # no rows: nothing to do
+    #      q  k  v  T   cu ctx B  maxq maxc H  G  D    scale  ks vs out cache nb bt mbps bs status stream
+    chk = [P, P, P, 64, P, P, 1, 64, 64, 4, 2, 128, 0.088, P, P, P, P, 8, P, 8, 16, None, None]
+    bad = list(chk); bad[5] = None
+    assert lib.prefill_attn_chunked_fp8(*bad) == 1       # no context lengths
+    bad = list(chk); bad[13] = None
+    assert lib.prefill_attn_chunked_fp8(*bad) == 1       # no K scale
+    bad = list(chk); bad[9] = 5
+    assert lib.prefill_attn_chunked_fp8(*bad) == 2       # 5 query heads over 2 kv heads
+    bad = list(chk); bad[11] = 96
+    assert lib.prefill_attn_chunked_fp8(*bad) == 3       # head_dim
+    bad = list(chk); bad[8] = 129
+    assert lib.prefill_attn_chunked_fp8(*bad) == 4       # a 129-token context does not fit 8 pages of 16
+    bad = list(chk); bad[16] = ctypes.c_void_p(FAKE + 8)
+    assert lib.prefill_attn_chunked_fp8(*bad) == 7       # pool alignment
+    bad = list(chk); bad[3] = 0
+    assert lib.prefill_attn_chunked_fp8(*bad) == 0       # no rows: nothing to do
     #       k  v  T   cu ctx B  G  D    ks vs cache nb bt mbps bs  status stream
     store = [P, P, 10, P, None, 1, 2, 128, P, P, P, 4, P, 4, 16, None, None]
     # only calls that the host rejects before any launch (the pointers are fake)

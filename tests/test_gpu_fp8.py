@@ -168,3 +168,4 @@ def test_prefill_fp8_cache_matches_oracle(lens, H, G, d, bs):
 @pytest.mark.parametrize("name", ["gqa_s8192_h32g8_d128", "varlen64_gqa_h32g8_d128"])
 def test_prefill_fp8_cache_full_size(name):
     _check_prefill_fp8(W.named_workload(name), False, name)
+

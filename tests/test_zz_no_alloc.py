@@ -8,8 +8,8 @@ prefill_attn_chunked, on the same inputs: two calls in a row must each match
 it (output within the suite's tolerance, KV cache bit-exact), and a call whose
 partials would not fit the array must be rejected before any launch.
 
-This file is collected last so that a run stopping at the first failure has
-already run every other test; it also passes alone in a fresh process.
+This file is collected after the other parity files, so that a run stopping at
+the first failure has already run them; it also passes alone in a fresh process.
 """
 import numpy as np
 import pytest
