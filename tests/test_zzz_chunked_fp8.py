@@ -20,6 +20,21 @@ from tests.test_gpu_fp8 import _assert_bytes_equal, _fp8_pool, _scales
 
 pytestmark = pytest.mark.gpu
 
+
+def _compare(gpu_out: torch.Tensor, ref: np.ndarray, vs: torch.Tensor, what: str):
+    """The suite's tolerance plus the staging term.  The call stages every
+    dequantized key and value rounded to bf16 (relative error <= 2^-9); an
+    output row is a convex combination of values, so the V staging moves it by
+    at most 2^-9 max |value| <= 2^-9 * 448 * max v_scale (the K staging moves
+    the scores by about 2^-9 of their size, far less at these magnitudes).
+    The mean bound is the suite's."""
+    g = gpu_out.to(torch.float64).numpy()
+    assert np.isfinite(g).all(), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    max_tol = U.MAX_ABS + 2.0 ** -9 * 448.0 * float(vs.max())
+    mx, mean = float(err.max()), float(err.mean())
+    assert mx <= max_tol and mean <= U.MEAN_ABS, f"{what}: max {mx:.3e} (bound {max_tol:.3e}) mean {mean:.3e}"
+
 def _chunk_case(lens, ctxs, H, G, d, bs, seed):
     """Sequences of ctx + n tokens whose first ctx are already in the FP8 cache
     (the oracle's codes); the last n are the call's chunk rows."""
@@ -59,7 +74,7 @@ def test_chunked_fp8_matches_oracle(lens, ctxs, H, G, d, bs):
     pool_d = pool.cuda()
     out = _run_chunked_fp8(q, k, v, cu, ctx, pool_d, w.block_table.cuda(), ks, vs, w.scale, max(lens), max(ctxs))
     _assert_bytes_equal(pool_d.cpu(), ref_pool, "fp8 pool after the chunk")
-    U.compare_out(out, ref_out, f"chunked fp8 {lens} {ctxs}")
+    _compare(out, ref_out, vs, f"chunked fp8 {lens} {ctxs}")
 
 
 def test_chunked_fp8_whole_sequence_in_chunks():
@@ -76,7 +91,7 @@ def test_chunked_fp8_whole_sequence_in_chunks():
     outs = []
     for q, k, v, cu, ctx, _ in W.chunk_views(w, 512):
         outs.append(_run_chunked_fp8(q, k, v, cu, ctx, pool_d, bt_d, ks, vs, w.scale, int(cu[-1]), int(ctx[0])))
-    U.compare_out(torch.cat(outs, 0), ref, "chunks of 512")
+    _compare(torch.cat(outs, 0), ref, vs, "chunks of 512")
     ref_pool = oracle.kv_write_fp8(w.k, w.v, w.cu_seqlens, _fp8_pool(w), w.block_table, bs, ks, vs)
     _assert_bytes_equal(pool_d.cpu(), ref_pool, "fp8 pool after all chunks")
 
@@ -99,4 +114,4 @@ def test_chunked_fp8_full_size_sampled():
     ref = oracle.chunked_fp8(w.q, w.k, w.v, w.cu_seqlens, torch.zeros(1, dtype=torch.int32), w.n_head, w.n_kv_head,
                              w.head_dim, w.scale, ks, vs, _fp8_pool(w), w.block_table, w.block_size, rows=rows,
                              heads=heads)
-    U.compare_out(out[rows, heads], ref, "chunked fp8 full size")
+    _compare(out[rows, heads], ref, vs, "chunked fp8 full size")
