@@ -29,7 +29,9 @@
 //  * FP8 mode (kFp8): the cache holds e4m3 codes with a scale per kv head;
 //    the ring holds code rows and the codes are widened to f16 inside the MMA
 //    fragments (see the Q K^T and P V steps), the scales folded into the
-//    scores and the output; kv_store_fp8_kernel quantizes rows into the cache.
+//    scores and the output; kv_store_fp8_kernel quantizes rows into the cache,
+//    and fp8_stage_kernel dequantizes the positions a chunked prefill attends
+//    to into bf16 pages for the chunked prefill kernel.
 // Earlier versions for the record: CUDA-core dot products (one FMA per
 // element) issued ~6.5k warp instructions per 64 keys and reached 19 % of the
 // DRAM bandwidth; a CTA-wide version with tensor-core MMAs and three barriers
