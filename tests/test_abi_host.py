@@ -313,3 +313,23 @@ def test_fp8_entry_points_validation(lib):
     assert lib.paged_decode_attn_fp8(*bad) == 4          # 129 keys do not fit 8 pages of 16
     bad = list(dec); bad[4] = 0
     assert lib.paged_decode_attn_fp8(*bad) == 0          # nothing to do
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """A C99 program includes the header, links against libprefill.so and calls
+    two host-only functions (no device work)."""
+    import subprocess
+    src = tmp_path / "abi_from_c.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <string.h>\n#include "prefill.h"\n'
+        'int main(void) {\n'
+        '    if (strcmp(prefill_status_string(PREFILL_OK), "ok") != 0) return 1;\n'
+        '    /* query block 1 of a 300-row prompt with no context: kv blocks 0 and 1 */\n'
+        '    if (prefill_num_kv_blocks(1, 0, 300, 128, 128) != 2) return 2;\n'
+        '    puts("ok");\n    return 0;\n}\n')
+    exe = tmp_path / "abi_from_c"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                           os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lprefill",
+                           "-Wl,-rpath," + libdir])
+    assert subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.strip() == "ok"
