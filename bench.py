@@ -492,6 +492,8 @@ def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
     """Time the oracle on random (row, head) pairs of the workload until about
     budget_s seconds of CPU work; return (TFLOP/s, cores, description)."""
     import oracle  # test infrastructure: only the CPU-baseline / reference legs use it
+    # one thread per core this process may run on
+    cores = oracle.set_num_threads(len(os.sched_getaffinity(0)))
     rng = np.random.default_rng(seed)
     done_flops, elapsed, nrows = 0.0, 0.0, 0
     batch = 64
@@ -507,8 +509,9 @@ def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
         done_flops += float(np.sum(4.0 * w.head_dim * (pos + 1)))
         nrows += batch
     desc = (f"{nrows} random (row, head) output rows of {w.name} through the fp64 oracle "
-            f"({elapsed:.1f} s); FLOPs counted as 4*head_dim*(keys) per row, the causal count")
-    return done_flops / elapsed / 1e12, oracle.num_threads(), desc, elapsed
+            f"({elapsed:.1f} s, {cores} threads = the cores in the process's CPU affinity set); "
+            f"FLOPs counted as 4*head_dim*(keys) per row, the causal count")
+    return done_flops / elapsed / 1e12, cores, desc, elapsed
 
 
 # ------------------------------------------------------------------ main
@@ -713,11 +716,14 @@ def reference_arm(args):
         if s >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
-    # ms for one whole step of the workload at the sampled rate
+    # ms for one whole step of the workload, EXTRAPOLATED from the sampled rate
+    # (each timed step runs only a bounded sample of the workload's rows)
     ms = w.causal_flops() / (value * 1e12) * 1e3
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "ms_per_step_kind": "extrapolated: one whole step of the workload at the rate measured on each step's sample",
+        "sample_s_per_step": round(per_step, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, 1),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",

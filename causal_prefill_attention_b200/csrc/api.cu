@@ -68,6 +68,12 @@ std::atomic<int> g_test_stall{0};
 // later calls; a separate buffer per stream keeps concurrent streams apart.
 // Kinds: the split-KV partials, and the staging of a chunked prefill over an
 // FP8 cache (which then also uses the split-KV partials).
+//
+// Growth is stream-ordered (cudaFreeAsync of the old buffer, cudaMallocAsync of
+// the new one, both on the call's stream): the old buffer is released only
+// after the work already queued on the stream that reads it, and the host never
+// waits.  A caller that cannot let the library allocate at all uses
+// prefill_attn_chunked_noalloc.
 enum WorkspaceKind { kSplitPartials = 0, kFp8Staging = 1 };
 struct Workspace {
     void *ptr = nullptr;
@@ -82,18 +88,20 @@ void *device_workspace(int kind, size_t bytes, void *stream) {
     std::lock_guard<std::mutex> lock(g_ws_mu);
     Workspace &w = g_ws[std::make_tuple(dev, stream, kind)];
     if (w.bytes < bytes) {
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
         if (w.ptr) {
-            cudaStreamSynchronize(static_cast<cudaStream_t>(stream));  // earlier calls may still read it
-            cudaFree(w.ptr);
+            cudaFreeAsync(w.ptr, st);  // after the queued work that reads it
             w.ptr = nullptr;
             w.bytes = 0;
         }
-        if (cudaMalloc(&w.ptr, bytes) != cudaSuccess) {
+        // round up so that slowly growing calls do not reallocate every time
+        const size_t want = bytes + bytes / 4;
+        if (cudaMallocAsync(&w.ptr, want, st) != cudaSuccess) {
             cudaGetLastError();
             w.ptr = nullptr;
             return nullptr;
         }
-        w.bytes = bytes;
+        w.bytes = want;
     }
     return w.ptr;
 }
@@ -110,7 +118,8 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
                 const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
                 int n_kv_head, int head_dim, float scale, prefill_bf16 *out, prefill_bf16 *cache, int num_blocks,
                 const int32_t *bt, int mbps, int bs, int32_t *status, prefill_stream_t stream, void *scratch,
-                size_t scratch_bytes, int window, uint8_t *cache8, const float *k_scale, const float *v_scale) {
+                size_t scratch_bytes, int window, uint8_t *cache8, const float *k_scale, const float *v_scale,
+                const float *k_fold, const float *v_fold) {
     if (!q || !k || !v || !cu || !out || !(cache || cache8) || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
     if (cache8 && (!k_scale || !v_scale)) return PREFILL_ERR_NULL;
     if (cache8 && (cache || chunked || window > 0)) return PREFILL_ERR_UNSUPPORTED;  // whole prompts only
@@ -183,16 +192,21 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     p.nsplit = 1;
     p.part_o = nullptr;
     p.part_ml = nullptr;
+    p.k_fold = k_fold;
+    p.v_fold = v_fold;
 
     int e;
     const bool pipelined = use_pipelined() && pf::fwd_pipelined_supported(p, head_dim);
-    if (cache8 && !pipelined) return PREFILL_ERR_UNSUPPORTED;  // the FP8 write lives in the pipelined kernel
+    // the FP8 write and the folded scales live in the pipelined kernel only
+    if ((cache8 || k_fold || v_fold) && !pipelined) return PREFILL_ERR_UNSUPPORTED;
     if (pipelined) {
         p.nsplit = pf::fwd_choose_splits(p);
+        // caller-supplied scratch of a fixed size: the largest split count whose
+        // partials fit it (1 needs none), so every call still runs
+        while (scratch && p.nsplit > 1 && pf::fwd_split_workspace_bytes(p, head_dim) > scratch_bytes) --p.nsplit;
         if (p.nsplit > 1) {
             const size_t o_bytes = (size_t)p.nsplit * p.total * p.n_head * head_dim * sizeof(float);
             const size_t need = pf::fwd_split_workspace_bytes(p, head_dim);
-            if (scratch && need > scratch_bytes) return PREFILL_ERR_SCRATCH_LIMIT;  // caller-supplied scratch too small
             char *ws = static_cast<char *>(scratch ? scratch : split_workspace(need, stream));
             if (ws) {
                 p.part_o = reinterpret_cast<float *>(ws);
@@ -324,14 +338,13 @@ int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const
     sp.mbps = max_blocks_per_seq;
     sp.block_size = block_size;
     if (pf::launch_kv_store_fp8(sp, head_dim, stream) != 0) return PREFILL_ERR_CUDA;
-    // 2. every key and value the chunk attends to, dequantized from the cache
+    // 2. every key and value the chunk attends to, as the e4m3 code values of
+    //    the cache (exact in bf16; the scales are applied by the attention)
     pf::Fp8StageParams gp;
     gp.cache8 = kv_cache_fp8;
     gp.block_table = block_table;
     gp.cu_seqlens = cu_seqlens_q;
     gp.context_lens = context_lens;
-    gp.k_scale = k_scale;
-    gp.v_scale = v_scale;
     gp.shadow = shadow;
     gp.shadow_table = table2;
     gp.k2 = k2;
@@ -346,11 +359,12 @@ int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const
     gp.mbps2 = mbps2;
     gp.max_span = (int)span;
     if (pf::launch_fp8_stage(gp, head_dim, stream) != 0) return PREFILL_ERR_CUDA;
-    // 3. the bf16 chunked attention over the staged rows (it also writes k2 / v2
-    //    into the shadow pool, which is scratch)
+    // 3. the bf16 chunked attention over the staged code values, with the K
+    //    scales folded into the scores and the V scales into the output (it
+    //    also writes k2 / v2 into the shadow pool, which is scratch)
     return pf::run_prefill(q, k2, v2, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len,
                            n_head, n_kv_head, head_dim, scale, out, shadow, num_seqs * mbps2, table2, mbps2,
-                           block_size, status_dev, stream, nullptr, 0);
+                           block_size, status_dev, stream, nullptr, 0, 0, nullptr, nullptr, nullptr, k_scale, v_scale);
 }
 
 int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,

@@ -761,8 +761,10 @@ __device__ __forceinline__ void f16x2_to_f32(uint32_t h, float &lo, float &hi) {
 }
 
 // One warp per (sequence, position): the K and V code rows of every kv head
-// (G * D bytes each, contiguous in the slot) are widened exactly to f16, scaled
-// in fp32 and rounded to bf16, 8 elements per lane step.
+// (G * D bytes each, contiguous in the slot) are widened to their code values
+// in bf16, 8 elements per lane step.  Every e4m3 value is exact in bf16 (at
+// most 4 significant bits, magnitudes 2^-9 .. 448), so nothing is rounded; the
+// per-kv-head scales are applied by the attention kernel (scores, output).
 template <int D>
 __global__ void __launch_bounds__(256) fp8_stage_kernel(const Fp8StageParams p) {
     const int i = blockIdx.y, lane = threadIdx.x & 31;
@@ -794,9 +796,7 @@ __global__ void __launch_bounds__(256) fp8_stage_kernel(const Fp8StageParams p) 
         uint16_t *dst = pos < ctx
             ? p.shadow + ((((size_t)i * p.mbps2 + pos / bs) * 2 + tt) * bs + pos % bs) * row
             : (tt ? p.v2 : p.k2) + (size_t)(c0 + pos - ctx) * row;
-        const float *sc = tt ? p.v_scale : p.k_scale;
         for (int x = lane * 8; x < (int)row; x += 32 * 8) {
-            const float s = __ldg(&sc[x / D]);
             const uint2 c = __ldg(reinterpret_cast<const uint2 *>(src + x));
             uint32_t w[4];
 #pragma unroll
@@ -804,7 +804,7 @@ __global__ void __launch_bounds__(256) fp8_stage_kernel(const Fp8StageParams p) 
                 const uint32_t two = ((e < 2 ? c.x : c.y) >> (16 * (e & 1))) & 0xffffu;
                 float lo, hi;
                 f16x2_to_f32(e4m3x2_to_f16x2(two), lo, hi);
-                w[e] = pack_bf16x2(lo * s, hi * s);
+                w[e] = pack_bf16x2(lo, hi);  // exact
             }
             *reinterpret_cast<uint4 *>(dst + x) = make_uint4(w[0], w[1], w[2], w[3]);
         }

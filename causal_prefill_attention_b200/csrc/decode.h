@@ -54,16 +54,16 @@ int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream);
 
 // Staging of a chunked prefill over an FP8 cache (decode.cu): sequence i's
 // positions 0 .. ctx_i + n_i - 1 are read from the FP8 cache through the block
-// table and dequantized (code value x scale, rounded to bf16); the prefix
-// (p < ctx_i) goes to a bf16 shadow pool whose block table gives sequence i
-// the pages i * mbps2 .. i * mbps2 + mbps2 - 1, the chunk's own rows to k2 / v2
-// (packed like the call's k / v).  The bf16 chunked kernel then runs on them.
+// table and widened to their e4m3 code values in bf16 (exact; no scale); the
+// prefix (p < ctx_i) goes to a bf16 shadow pool whose block table gives
+// sequence i the pages i * mbps2 .. i * mbps2 + mbps2 - 1, the chunk's own rows
+// to k2 / v2 (packed like the call's k / v).  The bf16 chunked kernel then runs
+// on them with the per-kv-head scales folded into its scores and output.
 struct Fp8StageParams {
     const uint8_t *cache8;        // [NB][2][bs][G][D] codes (the chunk's rows already stored)
     const int32_t *block_table;   // [B][mbps]
     const int32_t *cu_seqlens;    // [B + 1] chunk rows
     const int32_t *context_lens;  // [B]
-    const float *k_scale, *v_scale;
     uint16_t *shadow;             // [B * mbps2][2][bs][G][D] bf16
     int32_t *shadow_table;        // [B][mbps2]
     uint16_t *k2, *v2;            // [T][G][D] bf16

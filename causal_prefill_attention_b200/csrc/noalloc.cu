@@ -1,14 +1,14 @@
 // noalloc.cu -- prefill_attn_chunked_noalloc: chunked prefill for callers that
-// cannot allocate device memory.
+// cannot let the library allocate device memory.
 //
 // prefill_attn_chunked may need a split-KV workspace, which the library obtains
 // with cudaMalloc on the first call that splits.  Some callers cannot allow
-// that: code running inside CUDA graph stream capture (cudaMalloc is not a
-// capturable operation and breaks the capture), engines that own all device
-// memory through their own pool and forbid allocations behind their back, and
-// hosts whose memory budget is fixed at start-up.  This entry point runs the
-// same kernels with the split partials in a fixed, file-scope device array
-// instead, and never calls cudaMalloc, cudaFree or any allocating routine.
+// that: engines that own all device memory through their own pool and forbid
+// allocations behind its back, and hosts whose memory budget is fixed at
+// start-up.  This entry point runs the same kernels with the split partials in
+// a fixed, file-scope device array instead, and never calls cudaMalloc,
+// cudaFree or any allocating routine.  A call whose split partials would not
+// fit the array runs with fewer splits (down to none).
 //
 // The array is kScratchBytes (32 MiB) on every GPU that loads this library,
 // held until the process exits.  Every call shares it and it keeps the last

@@ -33,6 +33,11 @@ struct FwdParams {
     int nsplit;
     float *part_o;
     float *part_ml;
+    // per-kv-head factors folded into the scores (k_fold[g]) and into the output
+    // (v_fold[g]), or nullptr (factor 1): a chunked prefill over an FP8 cache
+    // stages e4m3 code values (exact in bf16) and applies the cache's scales here
+    const float *k_fold;
+    const float *v_fold;
 };
 
 struct TensorMaps {
@@ -53,17 +58,19 @@ size_t fwd_split_workspace_bytes(const FwdParams &p, int head_dim);
 int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
 
 // Host path shared by the C entry points (api.cu).  scratch / scratch_bytes:
-// caller-supplied split-KV scratch (nullptr: the library's own workspace);
-// a split that needs more than scratch_bytes returns PREFILL_ERR_SCRATCH_LIMIT.
+// caller-supplied split-KV scratch (nullptr: the library's own workspace); the
+// split count is lowered until the partials fit scratch_bytes (1 needs none).
 // window: sliding window of that many keys (0: plain causal).  cache8 (with
 // k_scale / v_scale): the K/V rows go to this FP8 cache instead of `cache`
 // (plain prefill only; cache is then nullptr): the attention kernel runs
 // without its cache writer and the FP8 store kernel follows on the stream.
+// k_fold / v_fold: per-kv-head factors applied to the scores and to the output
+// (FwdParams::k_fold / v_fold); the call then needs the pipelined kernel.
 int run_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int total, const int32_t *cu,
                 const int32_t *ctx_lens, bool chunked, int num_seqs, int max_q, long long max_ctx, int n_head,
                 int n_kv_head, int head_dim, float scale, uint16_t *out, uint16_t *cache, int num_blocks,
                 const int32_t *bt, int mbps, int bs, int32_t *status, struct CUstream_st *stream, void *scratch,
                 size_t scratch_bytes, int window = 0, uint8_t *cache8 = nullptr, const float *k_scale = nullptr,
-                const float *v_scale = nullptr);
+                const float *v_scale = nullptr, const float *k_fold = nullptr, const float *v_fold = nullptr);
 
 }  // namespace pf

@@ -26,7 +26,9 @@
 //     softmax of one query block overlaps the tensor-core work of the other.
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <map>
 #include <math_constants.h>
+#include <mutex>
 
 #include "block_rule.h"
 #include "params.h"
@@ -510,8 +512,6 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t tO = tmem + 256u + 128u * s + lane_off;
         const uint32_t b_sfull = bar(L::B_SFULL + s), b_pa = bar(L::B_PA + s), b_pb = bar(L::B_PB + s);
         const uint32_t b_ofull = bar(L::B_OFULL + s), b_oempty = bar(L::B_OEMPTY + s);
-        const float sl2 = p.scale_log2;
-        const float thr = kRescaleLog2 / sl2;  // the threshold in raw score units
         uint32_t ph_s = 0, ph_o = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -520,6 +520,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const Item it = decode_item<kWin, kChunk>(p, B, start, perm, P, u);
             if (it.skip || (s == 1 && !it.two)) continue;
             const int qb = it.qb0 + s;
+            // scores in log2 units: scale * log2(e), times the kv head's key factor when one is folded in
+            const float sl2 = p.k_fold ? p.scale_log2 * __ldg(&p.k_fold[it.g]) : p.scale_log2;
+            const float thr = kRescaleLog2 / sl2;  // the threshold in raw score units
+            const float vf = p.v_fold ? __ldg(&p.v_fold[it.g]) : 1.f;
             const int jb = kWin ? it.beg(s) : it.j_lo, je = it.end(s);
             float m_run = -CUDART_INF_F, l_run = 0.f;
             for (int j = jb; j < je; ++j) {
@@ -562,6 +566,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     tmem_ld32(tO + cc * 32, r);
+                    if (p.v_fold) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * vf);
+                    }
                     if (a < it.n) {
                         uint4 *d4 = reinterpret_cast<uint4 *>(po + cc * 32);
 #pragma unroll
@@ -571,7 +579,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (a < it.n) *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_run * sl2, l_run);
             } else {
-            const float inv_l = 1.f / l_run;
+            const float inv_l = vf / l_run;
             uint16_t *dst = p.out + ((size_t)(it.c0 + a) * p.n_head + it.h) * D;
             {
                 uint32_t r[32];
@@ -987,14 +995,25 @@ size_t smem_bytes(int P, int num_seqs) {
 }
 constexpr size_t kMaxSmem = 227 * 1024;
 
+// SM count of the current device, looked up once per device ordinal (a host
+// may hold GPUs of different sizes; calls may come from several threads).
 int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    static std::mutex mu;
+    static std::map<int, int> by_device;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
     }
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = by_device.find(dev);
+    if (it != by_device.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 148;
+    }
+    by_device[dev] = n;
     return n;
 }
 

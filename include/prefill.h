@@ -46,11 +46,14 @@
  * (typically a chunked-prefill chunk attending to a long cached prefix), the
  * kv range of each item is split across CTAs and the partial results are
  * merged by a second kernel on the same stream.  The partials live in a device
- * workspace that the library allocates (cudaMalloc) on the first such call for
- * a given (device, stream) and keeps for later calls, growing it when a larger
- * call needs more; calls that do not split allocate nothing.  Size:
- * splits x total rows x n_head x (head_dim + 2) x 4 bytes, splits <= 8.  If the
- * allocation fails the call runs unsplit.
+ * workspace that the library owns: allocated on the first such call for a
+ * given (device, stream) and kept for later calls, grown when a larger call
+ * needs more.  Allocation and growth are stream-ordered (cudaMallocAsync, and
+ * cudaFreeAsync of the smaller buffer, on `stream`), so a call never blocks the
+ * host or waits for the stream; calls that do not split allocate nothing.
+ * Size: splits x total rows x n_head x (head_dim + 2) x 4 bytes, splits <= 8.
+ * If the allocation fails the call runs unsplit.  prefill_attn_chunked_noalloc
+ * is the chunked call that allocates nothing.
  *
  * Errors: argument problems that the host can see are returned synchronously
  * and nothing is launched.  Problems only the device can see (a block-table
@@ -86,9 +89,9 @@ typedef enum {
     PREFILL_ERR_UNSUPPORTED = 3,  /* head_dim, block_size or scale outside the supported set */
     PREFILL_ERR_BLOCK_TABLE = 4,  /* block-table entry outside [0, num_blocks) or table too short */
     PREFILL_ERR_CUDA = 5,         /* launch or driver failure */
-    PREFILL_ERR_TIMEOUT = 6,      /* a device-side pipeline wait exceeded its iteration limit */
+    PREFILL_ERR_TIMEOUT = 6,      /* a device-side pipeline wait ran past its limit (about one second) */
     PREFILL_ERR_ALIGNMENT = 7,    /* a pointer is not 16-byte aligned */
-    PREFILL_ERR_SCRATCH_LIMIT = 8 /* prefill_attn_chunked_noalloc: the split partials exceed its static buffer */
+    PREFILL_ERR_SCRATCH_LIMIT = 8 /* reserved: no current entry point returns it (the value stays assigned) */
 } prefill_status;
 
 /*
@@ -352,31 +355,34 @@ int attn_out_projection(const prefill_bf16 *o, const prefill_bf16 *w_o, int toke
 
 /*
  * prefill_attn_chunked_noalloc -- prefill_attn_chunked for callers that cannot
- * allocate device memory.  The pages have no counterpart: this is a deployment
- * variant of the chunked call, not a step of the method.
+ * let the library allocate device memory.  The pages have no counterpart: this
+ * is a deployment variant of the chunked call, not a step of the method.
  *
  * prefill_attn_chunked may split long kv ranges (split-KV) and then obtains a
- * workspace with cudaMalloc.  Callers that cannot allow that -- code recorded
- * into a CUDA graph by stream capture (cudaMalloc cannot be captured), serving
- * engines that own all device memory through their own pool, processes whose
- * device-memory budget is fixed at start-up -- use this entry point instead.
- * It computes the same result with the same kernels, keeping the split
- * partials in a fixed device array that is part of the library: 32 MiB
+ * workspace with cudaMalloc.  Some callers cannot allow that: serving engines
+ * that own all device memory through their own pool (an allocation behind the
+ * pool's back can fail or fragment the memory it has reserved), and processes
+ * whose device-memory budget is fixed at start-up.  This entry point computes
+ * the same result with the same kernels, keeping the split partials in a
+ * fixed device array that is part of the library: 32 MiB
  * (prefill_noalloc_scratch_bytes()) on every GPU that loads the library, held
  * until the process exits.  It calls no cudaMalloc, cudaFree or allocating
  * library routine.
  *
- *   Arguments, layouts and errors as for prefill_attn_chunked, plus:
- *   PREFILL_ERR_SCRATCH_LIMIT  returned (before any launch) when the call would
- *     split and its partials -- splits x total_q x n_head x (head_dim + 2) x 4
- *     bytes -- do not fit the array.  Calls that do not split always fit.
+ *   Arguments, layouts and errors as for prefill_attn_chunked.  A call whose
+ *   chosen split count would need more than the array holds -- splits x
+ *   total_q x n_head x (head_dim + 2) x 4 bytes -- runs with the largest split
+ *   count that fits (down to 1, which needs no scratch), so every call that
+ *   prefill_attn_chunked accepts runs here too, with the same result up to
+ *   the rounding order of the split merge.
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any stream
  * capture.  Every call uses the same array, which keeps the last call's
- * contents (nothing in it needs to start at zero).  Calls whose GPU work
- * overlaps -- on different streams, or unordered from different threads --
- * race on the array: the caller must serialise them.
+ * contents (nothing in it needs to start at zero: each call writes every
+ * partial it later reads).  Calls whose GPU work overlaps -- on different
+ * streams, or unordered from different threads -- race on the array: the
+ * caller must serialise them.
  */
 int prefill_attn_chunked_noalloc(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
                                  int total_q, const int32_t *cu_seqlens_q, const int32_t *context_lens,

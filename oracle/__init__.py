@@ -54,6 +54,8 @@ def _configure(lib):
               lib.oracle_softmax_weights, lib.oracle_kv_write):
         f.restype = I
     lib.oracle_num_threads.restype = I
+    lib.oracle_set_num_threads.argtypes = [I]
+    lib.oracle_set_num_threads.restype = None
     F = ctypes.c_float
     lib.oracle_e4m3_encode.argtypes = [F]
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
@@ -200,6 +202,12 @@ def prefill(w, *, kv_cache=None, context_lens=None, rows=None, heads=None, windo
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Run the parallel loops on n threads; returns the count now in effect."""
+    _load().oracle_set_num_threads(int(n))
+    return num_threads()
 
 
 def qkv_projection(x, w, n_head: int, n_kv_head: int, head_dim: int):

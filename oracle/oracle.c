@@ -36,7 +36,7 @@
  *   lnwmold.com/news/496245 §4.1 -- sliding-window attention: each token
  *       attends only to its W nearest predecessors, n*W work instead of n^2.
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings where the pages are silent:
  *   the scale is the caller's float, widened to fp64; disallowed keys are
  *   left out of the sum (no -inf arithmetic); GQA groups are contiguous; a
  *   chunk is aligned bottom-right (row a sits at absolute position ctx + a);
@@ -523,5 +523,16 @@ int oracle_num_threads(void) {
     return omp_get_max_threads();
 #else
     return 1;
+#endif
+}
+
+/* Threads for the parallel loops that follow (n >= 1); a timing harness sets it
+ * to the cores the process may run on. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
 #endif
 }

@@ -62,18 +62,39 @@ def assert_cache_bits_equal(a: torch.Tensor, b: torch.Tensor, what: str = ""):
         raise AssertionError(f"{what}: {bad.shape[0]} cache elements differ, first at {bad[0].tolist()}")
 
 
-def sample_rows(w: W.Workload, n_random: int, seed: int = 0):
-    """(row, head) pairs: every sequence's first/last rows, block edges, random."""
+def sample_rows(w: W.Workload, n_random: int, seed: int = 0, block: int = 128):
+    """(row, head) pairs that reach every work item of the kernels.
+
+    A work item is (sequence, head, pair of 128-row query blocks, split of the
+    kv range), and every split of an item contributes to every row of its two
+    blocks.  So for every sequence, every 128-row query block and EVERY head,
+    the block's first and last valid rows are checked (on the 8k prompt:
+    64 blocks x 2 rows x 32 heads = 4096 pairs), plus each sequence's edge
+    rows and ``n_random`` random pairs."""
     rng = np.random.default_rng(seed)
     rows, heads = [], []
     for i, n in enumerate(w.seqlens):
         if n == 0:
             continue
         base = int(w.cu_seqlens[i])
-        for a in {0, 1, n - 1, min(127, n - 1), min(128, n - 1), n // 2}:
-            rows.append(base + a)
+        for b0 in range(0, n, block):
+            for a in sorted({b0, min(b0 + block, n) - 1}):
+                rows += [base + a] * w.n_head
+                heads += list(range(w.n_head))
+        for a in {1, n // 2}:
+            rows.append(base + min(a, n - 1))
             heads.append(int(rng.integers(0, w.n_head)))
     T = w.total_tokens
     rows += rng.integers(0, T, n_random).tolist()
     heads += rng.integers(0, w.n_head, n_random).tolist()
     return rows, heads
+
+
+def block_edge_rows(T: int, block: int = 128):
+    """First and last row of every ``block``-row tile of a T-row GEMM output
+    (every output tile of the projection kernels holds two of them)."""
+    rows = set()
+    for b0 in range(0, T, block):
+        rows.add(b0)
+        rows.add(min(b0 + block, T) - 1)
+    return sorted(rows)

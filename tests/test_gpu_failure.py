@@ -48,9 +48,14 @@ def test_hook_resets_after_one_launch():
 
 
 def test_stalled_split_call_leaves_no_stale_merge_state():
-    """A chunked call whose kv ranges are split (merged in-kernel by the split
-    that finishes last) is stalled, so some splits never arrive at their merge
-    counters; the next identical call must still merge every row correctly."""
+    """A chunked call whose kv ranges are split is stalled: some of its CTAs
+    give up before writing their split partials, so the workspace is left
+    holding a mix of this call's partials and stale ones.  The next identical
+    call must not read any of them as its own: its combine kernel may only
+    merge partials that its own attention kernel wrote, which every split of
+    every row does before the combine runs.  (The fixed array of the
+    no-allocation entry point relies on the same property: it keeps whatever
+    the last call left in it.)"""
     ctx, L, H, G, d, bs = 3000, 300, 8, 2, 128, 16
     full = W.make_workload([ctx + L], H, G, d, block_size=bs, seed=63, extra_pages=2)
     cache = oracle.kv_write(full.k[:ctx], full.v[:ctx], torch.tensor([0, ctx], dtype=torch.int32),

@@ -53,6 +53,16 @@ def test_varlen_with_empty_and_ragged_sequences():
     _full_check(W.make_workload([5, 0, 257, 1, 130, 0, 64], 4, 1, 128, seed=9, extra_pages=4), "varlen")
 
 
+def test_many_work_items_every_element():
+    """More work items than SMs, checked element by element: 8 sequences of
+    about 1k tokens (ragged tails) at 32 query / 8 kv heads give 1120 items
+    (pair of 128-row query blocks x head) over the 148 persistent CTAs, so
+    every CTA runs several items back to back (K/V ring phases carried across
+    items, TMEM and Q buffers reused, the zigzag deal)."""
+    w = W.make_workload([1024, 1000, 1100, 777, 1024, 1300, 900, 1024], 32, 8, 128, seed=15, extra_pages=2)
+    _full_check(w, "many items")
+
+
 def test_idempotent_rerun_rewrites_same_bits():
     w = W.make_workload([333], 8, 2, 128, seed=10)
     out1, cache1, s1 = U.run_prefill(w)
@@ -211,6 +221,14 @@ def _chunked_call(ctxs, lens, H, G, d, bs, seed):
 def test_split_kv_long_prefix(d):
     """4 work items against a ~3k prefix: the kv range is split and merged."""
     _chunked_call([3000], [300], 8, 2, d, 16, seed=71)
+
+
+def test_chunked_many_work_items_every_element():
+    """A chunked call with more work items than SMs (8 sequences x 2 pairs x
+    32 heads = 512, so no split-KV), every element against the oracle: each
+    CTA gathers several prefixes through the block table, back to back."""
+    _chunked_call([1000, 1537, 512, 2000, 0, 700, 1300, 64], [512, 500, 512, 300, 512, 511, 512, 257], 32, 8, 128, 16,
+                  seed=73)
 
 
 def test_split_kv_mixed_batch():

@@ -52,11 +52,13 @@ def test_identity_weight_copies_activations_bit_exact():
 
 def test_full_size_sampled_rows():
     """8192 tokens x hidden 4096 -> 32 q heads + 2 x 8 kv heads of 128 (the
-    headline attention's inputs); sampled rows against the oracle."""
+    headline attention's inputs); both edge rows of every 128-row output tile
+    and random rows, every column, against the oracle."""
     T, hid, H, G, d = 8192, 4096, 32, 8, 128
     x, w = W.make_projection(T, hid, H, G, d, seed=511)
     q, k, v = _run(x, w, H, G, d)
-    rows = [0, 1, 127, 128, 4095, 4096, 8190, 8191] + np.random.default_rng(5).integers(0, T, 56).tolist()
+    # both edge rows of every 128-row output tile (every tile of the kernel), plus random rows
+    rows = U.block_edge_rows(T) + np.random.default_rng(5).integers(0, T, 56).tolist()
     rq, rk, rv = oracle.qkv_projection(x[rows], w, H, G, d)
     U.compare_out(q[rows], rq, "q full")
     U.compare_out(k[rows], rk, "k full")
@@ -98,11 +100,12 @@ def test_out_projection_identity_weight_bit_exact():
 
 
 def test_out_projection_full_size_sampled_rows():
-    """8192 tokens: 32 heads x 128 merged -> hidden 4096; sampled rows."""
+    """8192 tokens: 32 heads x 128 merged -> hidden 4096; both edge rows of
+    every 128-row output tile and random rows, every column."""
     T, H, d, hid = 8192, 32, 128, 4096
     o, w_o = _out_inputs(T, H, d, hid, seed=531)
     y = _run_out(o, w_o)
-    rows = [0, 1, 127, 128, 4095, 4096, 8190, 8191] + np.random.default_rng(6).integers(0, T, 56).tolist()
+    rows = U.block_edge_rows(T) + np.random.default_rng(6).integers(0, T, 56).tolist()
     U.compare_out(y[rows], oracle.out_projection(o[rows], w_o), "y full")
     assert torch.isfinite(y.float()).all()
 

@@ -22,18 +22,13 @@ pytestmark = pytest.mark.gpu
 
 
 def _compare(gpu_out: torch.Tensor, ref: np.ndarray, vs: torch.Tensor, what: str):
-    """The suite's tolerance plus the staging term.  The call stages every
-    dequantized key and value rounded to bf16 (relative error <= 2^-9); an
-    output row is a convex combination of values, so the V staging moves it by
-    at most 2^-9 max |value| <= 2^-9 * 448 * max v_scale (the K staging moves
-    the scores by about 2^-9 of their size, far less at these magnitudes).
-    The mean bound is the suite's."""
-    g = gpu_out.to(torch.float64).numpy()
-    assert np.isfinite(g).all(), f"{what}: non-finite output"
-    err = np.abs(g - ref)
-    max_tol = U.MAX_ABS + 2.0 ** -9 * 448.0 * float(vs.max())
-    mx, mean = float(err.max()), float(err.mean())
-    assert mx <= max_tol and mean <= U.MEAN_ABS, f"{what}: max {mx:.3e} (bound {max_tol:.3e}) mean {mean:.3e}"
+    """The suite's tolerance (max 2e-2, mean 2e-3).  The call stages the e4m3
+    code values, which bf16 holds exactly, and applies the per-kv-head scales
+    in fp32 inside the attention (K's to the scores, V's to the output), so
+    the only departures from the fp64 oracle are the fp32 accumulation and the
+    bf16 P and output roundings of the bf16 path."""
+    return U.compare_out(gpu_out, ref, what)
+
 
 def _chunk_case(lens, ctxs, H, G, d, bs, seed):
     """Sequences of ctx + n tokens whose first ctx are already in the FP8 cache
@@ -97,8 +92,9 @@ def test_chunked_fp8_whole_sequence_in_chunks():
 
 
 def test_chunked_fp8_full_size_sampled():
-    """The 8k GQA prompt in 16 chunks of 512 over the FP8 cache; sampled rows of
-    every chunk against the oracle, the final pool byte-exact."""
+    """The 8k GQA prompt in 16 chunks of 512 over the FP8 cache; the first and
+    last row of every 128-row block of every chunk, for every head, and random
+    rows against the oracle; the final pool byte-exact."""
     w = W.named_workload("chunked512_gqa_s8192_h32g8_d128")
     ks, vs = _scales(w.k), _scales(w.v)
     pool_d, bt_d = _fp8_pool(w).cuda(), w.block_table.cuda()
@@ -108,9 +104,9 @@ def test_chunked_fp8_full_size_sampled():
     out = torch.cat(outs, 0)
     ref_pool = oracle.kv_write_fp8(w.k, w.v, w.cu_seqlens, _fp8_pool(w), w.block_table, w.block_size, ks, vs)
     _assert_bytes_equal(pool_d.cpu(), ref_pool, "fp8 pool, 16 chunks")
-    rng = np.random.default_rng(8)
-    rows = [0, 511, 512, 4095, 4096, 8191] + rng.integers(0, w.total_tokens, 42).tolist()
-    heads = rng.integers(0, w.n_head, len(rows)).tolist()
+    rows, heads = U.sample_rows(w, 42, seed=8)  # every (128-row block, head): first and last row
+    rows += [511, 512, 4095, 4096]
+    heads += [3, 30, 0, 17]
     ref = oracle.chunked_fp8(w.q, w.k, w.v, w.cu_seqlens, torch.zeros(1, dtype=torch.int32), w.n_head, w.n_kv_head,
                              w.head_dim, w.scale, ks, vs, _fp8_pool(w), w.block_table, w.block_size, rows=rows,
                              heads=heads)
