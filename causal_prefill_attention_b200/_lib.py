@@ -24,7 +24,7 @@ EXPORTED = ("prefill_attn", "prefill_attn_chunked", "prefill_status_string",
             "prefill_attn_chunked_noalloc", "prefill_noalloc_scratch_bytes",
             "prefill_attn_sliding_window", "prefill_first_kv_block", "prefill_kv_block_rule_window",
             "paged_decode_attn", "qkv_projection", "kv_cache_store_fp8", "paged_decode_attn_fp8",
-            "attn_out_projection", "prefill_attn_fp8_cache", "prefill_attn_chunked_fp8")
+            "attn_out_projection", "prefill_attn_fp8_cache", "prefill_attn_chunked_fp8", "prefill_test_exp2_fma2")
 
 _lib = None
 
@@ -79,6 +79,8 @@ def load() -> ctypes.CDLL:
         lib.kv_cache_store_fp8.restype = I
         lib.paged_decode_attn_fp8.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P, P, I, P, I, I, P, P]
         lib.paged_decode_attn_fp8.restype = I
+        lib.prefill_test_exp2_fma2.argtypes = [P, P, I, P]
+        lib.prefill_test_exp2_fma2.restype = I
         _lib = lib
     return _lib
 
@@ -344,6 +346,18 @@ def inject_stall(enable: bool = True) -> None:
     """Test hook: the next pipelined launch withholds one Q tile so that a
     bounded device wait expires and the call reports PREFILL_ERR_TIMEOUT."""
     load().prefill_test_inject_stall(1 if enable else 0)
+
+
+def exp2_fma2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """Test hook: the kernel's FMA-pipe exponential applied to a CUDA float32
+    tensor (C ABI ``prefill_test_exp2_fma2``)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x: expected a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    rc = load().prefill_test_exp2_fma2(_ptr(x), _ptr(y), x.numel(), _stream_ptr(stream))
+    if rc != 0:
+        raise PrefillError(rc, "prefill_test_exp2_fma2")
+    return y
 
 
 def num_kv_blocks(qb: int, ctx: int, n: int, bm: int = 128, bn: int = 128) -> int:

@@ -62,6 +62,9 @@ bool use_pipelined() {
 }
 
 std::atomic<int> g_test_stall{0};
+// Launch counter: tags the rows a launch splits, so that the merge kernel never
+// takes another launch's leftovers in a reused workspace for its own.
+std::atomic<uint32_t> g_epoch{1};
 
 // Device workspaces: one buffer per (device, stream, kind), allocated on the
 // first call that needs it and grown when a larger call needs more.  Kept for
@@ -192,6 +195,8 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     p.nsplit = 1;
     p.part_o = nullptr;
     p.part_ml = nullptr;
+    p.part_nsp = nullptr;
+    p.epoch = g_epoch.fetch_add(1) & 0x0fffffffu;
     p.k_fold = k_fold;
     p.v_fold = v_fold;
 
@@ -211,6 +216,8 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
             if (ws) {
                 p.part_o = reinterpret_cast<float *>(ws);
                 p.part_ml = reinterpret_cast<float *>(ws + o_bytes);
+                p.part_nsp = reinterpret_cast<uint32_t *>(ws + o_bytes +
+                                                          (size_t)p.nsplit * p.total * p.n_head * 2 * sizeof(float));
             } else {
                 p.nsplit = 1;  // no workspace: run unsplit
             }
@@ -566,6 +573,12 @@ int attn_out_projection(const prefill_bf16 *o, const prefill_bf16 *w_o, int toke
 }
 
 void prefill_test_inject_stall(int enable) { g_test_stall.store(enable ? 1 : 0); }
+
+int prefill_test_exp2_fma2(const float *x, float *y, int n, prefill_stream_t stream) {
+    if (n < 0) return PREFILL_ERR_SHAPE;
+    if (n > 0 && (!x || !y)) return PREFILL_ERR_NULL;
+    return pf::launch_exp2_fma2_probe(x, y, n, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+}
 
 const char *prefill_status_string(int s) {
     switch (s) {

@@ -29,10 +29,15 @@ struct FwdParams {
     int window;                   // sliding window: row P sees keys P-window+1 .. P (<= 0: none)
     // split-KV: kv ranges split into up to nsplit parts; the partial results go to
     // part_o [nsplit][total][n_head][D] (fp32, unnormalised) and part_ml
-    // [nsplit][total][n_head][2] (running max in log2 units, exp-sum)
+    // [nsplit][total][n_head][2] (running max in log2 units, exp-sum), and
+    // part_nsp [total] holds, for every row of a valid sequence, its pair's split
+    // count tagged with this launch's epoch ((epoch << 4) | splits), so that the
+    // merge kernel skips rows that this launch did not split (or did not reach)
     int nsplit;
     float *part_o;
     float *part_ml;
+    uint32_t *part_nsp;
+    uint32_t epoch;
     // per-kv-head factors folded into the scores (k_fold[g]) and into the output
     // (v_fold[g]), or nullptr (factor 1): a chunked prefill over an FP8 cache
     // stages e4m3 code values (exact in bf16) and applies the cache's scales here
@@ -54,6 +59,8 @@ bool fwd_pipelined_supported(const FwdParams &p, int head_dim);
 // Split count for the pipelined kernel (1 = no split) and its workspace bytes.
 int fwd_choose_splits(const FwdParams &p);
 size_t fwd_split_workspace_bytes(const FwdParams &p, int head_dim);
+// exp2_fma2 (the FMA-pipe exponential of the pipelined kernel) applied to n floats (test hook).
+int launch_exp2_fma2_probe(const float *x, float *y, int n, void *stream);
 // One-CTA-per-query-block kernel (prefill_fwd_v0.cu): no size limits.
 int launch_fwd_v0(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream);
 

@@ -53,9 +53,14 @@ constexpr uint32_t kPOff = 0;
 // Running max of a row that has seen no visible key yet (finite, far below any score).
 constexpr float kNoKeyMax = -1e30f;
 // Which of the 32 column pairs in each 64-column half of an unmasked block take
-// their exponentials on the FMA pipe (exp2_fma2) instead of MUFU (ex2).
+// their exponentials on the FMA pipe (exp2_fma2) instead of MUFU (ex2): pairs
+// 0, 8, 16 and 24, one exponential in eight.  MUFU gives 16 results per clock
+// per SM, as many as the tensor core needs at head_dim 128, so moving a few off
+// it shortens the softmax; measured on the 8k GQA prompt: +2 to +4 % with one
+// in eight, +3 % with one in four, slower beyond (the ALU pipe, at half rate,
+// then limits the polynomial's clamps and exponent adds).
 #ifndef PF_EXP2_EMU_MASK
-#define PF_EXP2_EMU_MASK 0x00000000u
+#define PF_EXP2_EMU_MASK 0x01010101u
 #endif
 constexpr uint32_t kEmuMask = PF_EXP2_EMU_MASK;
 
@@ -444,6 +449,12 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     for (int x = tid; x <= P; x += NTHREADS) cur[x] = 0;
     __syncthreads();
+    // Nothing above read global memory.  From here on the previous kernels on
+    // the stream (e.g. the chunk before this one, whose K/V this call reads from
+    // the cache) are complete and their writes visible; the next launch may be
+    // scheduled now and waits the same way for this one.
+    griddep_wait();
+    griddep_launch_dependents();
     {
         bool bad = false;
         for (int i = tid; i < p.num_seqs; i += NTHREADS) {
@@ -557,6 +568,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ph_o ^= 1;
             tc_fence_after();
             const int a = qb * BM + row;
+            if (p.part_nsp && it.h == 0 && it.split == 0 && a < it.n)
+                p.part_nsp[it.c0 + a] = (p.epoch << 4) | (uint32_t)it.nsp;
             if (it.nsp > 1) {
                 // split-KV: unnormalised O, the running max (log2 units) and the
                 // exp-sum go to the workspace; the combine kernel merges the splits
@@ -908,84 +921,70 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp == WARP_MMA) tmem_dealloc(tmem, 512);
 }
 
-// Split-KV combine: one CTA per packed row t, one warp per query head (heads
-// strided by the warp count); the row's sequence and split count are found
-// once per CTA.  O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with
-// M = max_s m_s -- the merge rule the online softmax applies between blocks.
-constexpr int kCombineWarps = 16;
+// Split-KV merge: one warp per (packed row t, query head h), four per CTA.  The
+// row's split count comes from part_nsp, written by this launch's attention
+// kernel for every row of a valid sequence with the launch's epoch (a stale or
+// unsplit row is left alone).  All partial loads are issued before any use;
+// then O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s --
+// the merge rule the online softmax applies between blocks.
+constexpr int kCombineWarps = 4;
+constexpr int kMaxSplits = 8;
 template <int D>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(const FwdParams p) {
     constexpr int E = D / 32;  // elements per lane
-    __shared__ int s_nsp;
-    const int t = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        int lo = 0, hi = p.num_seqs - 1;  // last sequence starting at or before row t
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.cu_seqlens[mid] <= t) lo = mid; else hi = mid - 1;
-        }
-        int nsp = 0;
-        bool bad = false;
-        if (seq_pairs(p, lo, &bad) > 0) {
-            const int c0 = p.cu_seqlens[lo], n = p.cu_seqlens[lo + 1] - c0;
-            const int a = t - c0;
-            if (a >= 0 && a < n) {
-                const int ctx = p.context_lens ? p.context_lens[lo] : 0;
-                const int qb0 = (a / (2 * BM)) * 2;
-                const bool two = (qb0 + 1) * BM < n;
-                const int nmax = two ? num_kv_blocks(qb0 + 1, ctx, n, BM, BN) : num_kv_blocks(qb0, ctx, n, BM, BN);
-                nsp = useful_splits(nmax - first_kv_block(qb0, ctx, n, BM, BN, p.window), p.nsplit);
+    griddep_wait();  // the attention kernel's partials are complete
+    griddep_launch_dependents();
+    const long long task = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (task >= (long long)p.total * p.n_head) return;
+    const int t = (int)(task / p.n_head), h = (int)(task - (long long)t * p.n_head);
+    const uint32_t tag = p.part_nsp[t];
+    if ((tag >> 4) != (p.epoch & 0x0fffffffu)) return;  // not a row this launch split
+    int nsp = (int)(tag & 15u);
+    if (nsp <= 1) return;
+    if (nsp > p.nsplit) nsp = p.nsplit;
+    const size_t row = (size_t)t * p.n_head + h, stride = (size_t)p.total * p.n_head;
+    float2 ml = make_float2(-CUDART_INF_F, 0.f);
+    if (lane < nsp) ml = *reinterpret_cast<const float2 *>(p.part_ml + (row + lane * stride) * 2);
+    float v[kMaxSplits][E];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+        if (sp < nsp) {
+            const float *po = p.part_o + (row + sp * stride) * D + lane * E;
+            if constexpr (E == 4) {
+                const float4 f = *reinterpret_cast<const float4 *>(po);
+                v[sp][0] = f.x; v[sp][1] = f.y; v[sp][2] = f.z; v[sp][3] = f.w;
+            } else {
+                const float2 f = *reinterpret_cast<const float2 *>(po);
+                v[sp][0] = f.x; v[sp][1] = f.y;
             }
         }
-        s_nsp = nsp;
     }
-    __syncthreads();
-    const int nsp = s_nsp;
-    if (nsp <= 1) return;  // row not split (the attention kernel wrote it) or not part of a valid sequence
-    for (int h = warp; h < p.n_head; h += kCombineWarps) {
-        const size_t base_row = (size_t)t * p.n_head + h;
-        const size_t stride_row = (size_t)p.total * p.n_head;
-        float M = -CUDART_INF_F;
-        float m[8], l[8];
+    float M = ml.x;
 #pragma unroll
-        for (int sp = 0; sp < 8; ++sp) {
-            if (sp < nsp) {
-                const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (base_row + sp * stride_row) * 2);
-                m[sp] = ml.x;
-                l[sp] = ml.y;
-                M = fmaxf(M, ml.x);
-            }
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float wgt = lane < nsp ? ex2(ml.x - M) : 0.f;
+    float L = wgt * ml.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+        const float w_sp = __shfl_sync(0xffffffffu, wgt, sp);
+        if (sp < nsp) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = fmaf(w_sp, v[sp][e], acc[e]);
         }
-        float L = 0.f, acc[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int sp = 0; sp < 8; ++sp) {
-            if (sp < nsp) {
-                const float wgt = ex2(m[sp] - M);
-                L += wgt * l[sp];
-                const float *po = p.part_o + (base_row + sp * stride_row) * D + lane * E;
-                float v[E];
-                if constexpr (E == 4) {
-                    const float4 f = *reinterpret_cast<const float4 *>(po);
-                    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-                } else {
-                    const float2 f = *reinterpret_cast<const float2 *>(po);
-                    v[0] = f.x; v[1] = f.y;
-                }
-#pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, v[e], acc[e]);
-            }
-        }
-        const float inv = 1.f / L;
-        uint16_t *dst = p.out + base_row * D + lane * E;
-        if constexpr (E == 4) {
-            *reinterpret_cast<uint2 *>(dst) =
-                make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-        } else {
-            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-        }
+    }
+    const float inv = 1.f / L;
+    uint16_t *dst = p.out + row * D + lane * E;
+    if constexpr (E == 4) {
+        *reinterpret_cast<uint2 *>(dst) =
+            make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    } else {
+        *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
     }
 }
 
@@ -1027,12 +1026,26 @@ int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const long long items_bound = (long long)p.num_seqs * p.n_head * P;
     const long long items = items_bound * (p.nsplit > 0 ? p.nsplit : 1);
     const int grid_s = (int)(items < sm_count() ? items : sm_count());
-    prefill_fwd_kernel<D, NST, MODE><<<grid_s, NTHREADS, smem, (cudaStream_t)stream>>>(maps.q, maps.k, maps.v,
-                                                                                        maps.cache, p, P);
-    e = cudaGetLastError();
+    // programmatic dependent launches: each kernel may be scheduled while the
+    // one before it on the stream drains, and waits for it (griddep_wait)
+    // before touching global memory
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid_s);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = (cudaStream_t)stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, prefill_fwd_kernel<D, NST, MODE>, maps.q, maps.k, maps.v, maps.cache, p, P);
     if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
-    combine_splits_kernel<D><<<(unsigned)p.total, 32 * kCombineWarps, 0, (cudaStream_t)stream>>>(p);
-    return (int)cudaGetLastError();
+    const long long tasks = (long long)p.total * p.n_head;
+    cfg.gridDim = dim3((unsigned)((tasks + kCombineWarps - 1) / kCombineWarps));
+    cfg.blockDim = dim3(32 * kCombineWarps);
+    cfg.dynamicSmemBytes = 0;
+    return (int)cudaLaunchKernelEx(&cfg, combine_splits_kernel<D>, p);
 }
 
 template <int D>
@@ -1080,7 +1093,7 @@ int fwd_choose_splits(const FwdParams &p) {
     if (p.window > 0) nk = imin(nk, cdiv(p.window, BN) + 2);  // a windowed query block's range
     int best = 1;
     double best_cost = (double)nk;  // one wave of whole ranges
-    for (int sp = 2; sp <= 8; ++sp) {
+    for (int sp = 2; sp <= kMaxSplits; ++sp) {
         if (nk / sp < kMinSplitBlocks) break;
         const double waves = (double)((items * sp + sms - 1) / sms);
         const double cost = waves * cdiv(nk, sp) + kSplitCostSteps;
@@ -1094,7 +1107,28 @@ int fwd_choose_splits(const FwdParams &p) {
 
 size_t fwd_split_workspace_bytes(const FwdParams &p, int head_dim) {
     if (p.nsplit <= 1) return 0;
-    return (size_t)p.nsplit * p.total * p.n_head * ((size_t)head_dim + 2) * sizeof(float);
+    return (size_t)p.nsplit * p.total * p.n_head * ((size_t)head_dim + 2) * sizeof(float) +
+           (size_t)p.total * sizeof(uint32_t);
+}
+
+namespace {
+// y[i] = exp2_fma2(x[i]) for a test of the polynomial against exp2 (one pair per thread).
+__global__ void exp2_fma2_probe_kernel(const float *x, float *y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+    float ra, rb;
+    exp2_fma2(a, b, ra, rb);
+    y[i] = ra;
+    if (i + 1 < n) y[i + 1] = rb;
+}
+}  // namespace
+
+int launch_exp2_fma2_probe(const float *x, float *y, int n, void *stream) {
+    if (n <= 0) return 0;
+    const int pairs = (n + 1) / 2;
+    exp2_fma2_probe_kernel<<<(pairs + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+    return (int)cudaGetLastError();
 }
 
 int launch_fwd(const TensorMaps &maps, const FwdParams &p, int head_dim, void *stream) {

@@ -357,6 +357,16 @@ __device__ __forceinline__ void exp2_fma2(float y0, float y1, float &r0, float &
     r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// Programmatic dependent launch: wait until the grids this launch depends on
+// (the previous kernels on the stream) have completed and their memory is
+// visible; a no-op for a launch without the programmatic-serialization
+// attribute.  launch_dependents lets the next launch on the stream be scheduled
+// early (its own griddep_wait still holds it until this grid completes).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void report(int32_t *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }

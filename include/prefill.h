@@ -51,7 +51,8 @@
  * needs more.  Allocation and growth are stream-ordered (cudaMallocAsync, and
  * cudaFreeAsync of the smaller buffer, on `stream`), so a call never blocks the
  * host or waits for the stream; calls that do not split allocate nothing.
- * Size: splits x total rows x n_head x (head_dim + 2) x 4 bytes, splits <= 8.
+ * Size: splits x total rows x n_head x (head_dim + 2) x 4 bytes + 4 bytes per
+ * row, splits <= 8.
  * If the allocation fails the call runs unsplit.  prefill_attn_chunked_noalloc
  * is the chunked call that allocates nothing.
  *
@@ -371,7 +372,7 @@ int attn_out_projection(const prefill_bf16 *o, const prefill_bf16 *w_o, int toke
  *
  *   Arguments, layouts and errors as for prefill_attn_chunked.  A call whose
  *   chosen split count would need more than the array holds -- splits x
- *   total_q x n_head x (head_dim + 2) x 4 bytes -- runs with the largest split
+ *   total_q x n_head x (head_dim + 2) x 4 + 4 x total_q bytes -- runs with the largest split
  *   count that fits (down to 1, which needs no scratch), so every call that
  *   prefill_attn_chunked accepts runs here too, with the same result up to
  *   the rounding order of the split merge.
@@ -407,6 +408,18 @@ size_t prefill_noalloc_scratch_bytes(void);
  * reported and that the CUDA context stays usable.
  */
 void prefill_test_inject_stall(int enable);
+
+/*
+ * Test hook for the FMA-pipe exponential (no counterpart on the pages).  The
+ * pipelined kernel takes one exponential in eight of an unmasked block's
+ * softmax as a polynomial on the FMA pipe instead of the MUFU ex2 unit, to
+ * shorten the softmax; this call applies that same device function to n floats
+ * so that tests can bound its error against exp2: y[i] ~= 2^x[i] for x[i] in
+ * [-125, 127] (inputs below -125 give about 2^-125).  x, y: device float [n].
+ * Returns PREFILL_ERR_NULL / PREFILL_ERR_SHAPE for bad arguments, else
+ * launches one small kernel on `stream`.
+ */
+int prefill_test_exp2_fma2(const float *x, float *y, int n, prefill_stream_t stream);
 
 /* Human-readable name of a prefill_status value (static storage). */
 const char *prefill_status_string(int status);

@@ -333,3 +333,10 @@ def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
                            os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lprefill",
                            "-Wl,-rpath," + libdir])
     assert subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.strip() == "ok"
+
+
+def test_exp2_hook_rejects_bad_arguments(lib):
+    lib.prefill_test_exp2_fma2.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    assert lib.prefill_test_exp2_fma2(None, FAKE, 4, None) == 1
+    assert lib.prefill_test_exp2_fma2(FAKE, None, 4, None) == 1
+    assert lib.prefill_test_exp2_fma2(FAKE, FAKE, -1, None) == 2
