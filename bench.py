@@ -133,6 +133,9 @@ class PlainRunner:
         _lib.prefill_attn(self.q, self.k, self.v, self.cu, self.w.max_seqlen, self.w.scale, self.out, self.cache,
                           self.bt, status=self.status, stream=self.stream)
 
+    def output(self) -> torch.Tensor:
+        return self.out
+
     def check_status(self):
         s = int(self.status.item())
         if s:
@@ -162,6 +165,9 @@ class ChunkedRunner:
             _lib.prefill_attn_chunked(q, k, v, cu, ctx, L, c, self.w.scale, out, self.cache, self.bt,
                                       status=self.status, stream=self.stream)
 
+    def output(self) -> torch.Tensor:
+        return torch.cat([part[-1] for part in self.parts], 0)
+
     def check_status(self):
         s = int(self.status.item())
         if s:
@@ -170,8 +176,9 @@ class ChunkedRunner:
 
 class ChunkedFp8Runner(ChunkedRunner):
     """The chunked workload over an FP8 (e4m3) cache: one prefill_attn_chunked_fp8
-    call per 512-token chunk (FP8 store of the chunk, staging of the dequantized
-    prefix, the bf16 chunked kernel: 3 launches, 4 when the call splits)."""
+    call per 512-token chunk (FP8 store of the chunk's codes, then the attention
+    kernel reading every key and value as e4m3 codes: 2 launches, 3 when the
+    call splits)."""
 
     def __init__(self, w: W.Workload, chunk: int, stream):
         super().__init__(w, chunk, stream)
@@ -488,14 +495,17 @@ def e2e_run(w: W.Workload, steps, warmup, stream):
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
-def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
+def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0, gpu_out=None):
     """Time the oracle on random (row, head) pairs of the workload until about
-    budget_s seconds of CPU work; return (TFLOP/s, cores, description)."""
+    budget_s seconds of CPU work; return (TFLOP/s, cores, description, seconds,
+    errors).  With gpu_out (the timed run's output, on the host) the same rows
+    are compared with it: errors = (max |d|, sum |d|, elements), else None."""
     import oracle  # test infrastructure: only the CPU-baseline / reference legs use it
     # one thread per core this process may run on
     cores = oracle.set_num_threads(len(os.sched_getaffinity(0)))
     rng = np.random.default_rng(seed)
     done_flops, elapsed, nrows = 0.0, 0.0, 0
+    err_max, err_sum, err_n = 0.0, 0.0, 0
     batch = 64
     while elapsed < budget_s:
         rows = rng.integers(0, w.total_tokens, batch)
@@ -503,15 +513,51 @@ def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
         starts = w.cu_seqlens.numpy()
         pos = rows - starts[np.searchsorted(starts, rows, side="right") - 1]
         t0 = time.perf_counter()
-        oracle.attention_rows(w.q, w.k, w.v, w.cu_seqlens, w.n_head, w.n_kv_head, w.head_dim, w.scale,
-                              rows.tolist(), heads.tolist())
+        ref = oracle.attention_rows(w.q, w.k, w.v, w.cu_seqlens, w.n_head, w.n_kv_head, w.head_dim, w.scale,
+                                    rows.tolist(), heads.tolist())
         elapsed += time.perf_counter() - t0
+        if gpu_out is not None:
+            d = np.abs(gpu_out[rows, heads].to(torch.float64).numpy() - ref)
+            err_max, err_sum, err_n = max(err_max, float(d.max())), err_sum + float(d.sum()), err_n + d.size
         done_flops += float(np.sum(4.0 * w.head_dim * (pos + 1)))
         nrows += batch
     desc = (f"{nrows} random (row, head) output rows of {w.name} through the fp64 oracle "
             f"({elapsed:.1f} s, {cores} threads = the cores in the process's CPU affinity set); "
             f"FLOPs counted as 4*head_dim*(keys) per row, the causal count")
-    return done_flops / elapsed / 1e12, cores, desc, elapsed
+    errors = (err_max, err_sum, err_n) if gpu_out is not None else None
+    return done_flops / elapsed / 1e12, cores, desc, elapsed, errors
+
+
+def kv_cache_matches_oracle(w: W.Workload, cache_host: torch.Tensor) -> bool:
+    """The timed run's paged cache, bit for bit, against the oracle's KV write
+    of the same workload (part of the CPU-baseline leg)."""
+    import oracle  # test infrastructure: only the CPU-baseline / reference legs use it
+    ref = oracle.kv_write(w.k, w.v, w.cu_seqlens, w.empty_cache(), w.block_table, w.block_size)
+    return bool(torch.equal(ref.view(torch.int16), cache_host.view(torch.int16)))
+
+
+def kv_bytes(w: W.Workload) -> dict:
+    """Algorithmic bytes of the cache write (every token's K and V rows, bf16) and,
+    for a chunked workload, of the prefix gather (each chunk reads the K and V
+    rows of every earlier token once per kv head: the GQA reuse)."""
+    d = {"kv_write_bytes": 2 * w.total_tokens * w.n_kv_head * w.head_dim * 2}
+    if w.chunk:
+        ctxs = range(0, w.total_tokens, w.chunk)
+        d["gather_bytes"] = sum(2 * c * w.n_kv_head * w.head_dim * 2 for c in ctxs)
+    return d
+
+
+def kv_rates(w: W.Workload, ms: float) -> dict:
+    """kv_bytes with their rates over the whole step time.  The write and the
+    gather run inside the attention kernel, overlapped with its tensor-core
+    work, so these are effective rates (bytes moved per step time), not the
+    bandwidth of a separate copy."""
+    d = kv_bytes(w)
+    out = dict(d)
+    out["kv_write_gbs_effective"] = round(d["kv_write_bytes"] / (ms * 1e-3) / 1e9, 1)
+    if "gather_bytes" in d:
+        out["gather_gbs_effective"] = round(d["gather_bytes"] / (ms * 1e-3) / 1e9, 1)
+    return out
 
 
 # ------------------------------------------------------------------ main
@@ -573,7 +619,8 @@ def main():
             dx = time_steps(rx, max(5, args.steps // 2), 3, stream, flush)
             mx = statistics.median(dx)
             extra[name] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
-                           "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches}
+                           "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1), "launches": rx.launches,
+                           **kv_rates(wx, mx)}
             del rx, wx
             torch.cuda.empty_cache()
         name, base, win = WINDOW_LINE
@@ -646,7 +693,7 @@ def main():
             mx = statistics.median(dx)
             extra[wx.name + "_fp8kv"] = {"ms": round(mx, 4), "tflops": round(rx.flops / (mx * 1e-3) / 1e12, 2),
                                          "prompt_tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
-                                         "calls": len(rx.parts), "launches_per_call": "3 (4 when split)",
+                                         "calls": len(rx.parts), "launches_per_call": "2 (3 when split)",
                                          "kv_format": "e4m3, per-kv-head scales"}
             del rx
             torch.cuda.empty_cache()
@@ -656,8 +703,14 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1:
-        v, cores, desc, el = oracle_sample(w, args.cpu_budget)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        out_h = runner.output().cpu()
+        v, cores, desc, el, errs = oracle_sample(w, args.cpu_budget, gpu_out=out_h)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+               # the same sampled rows compared with the timed run's output, and the
+               # timed run's paged cache against the oracle's KV write, bit for bit
+               "parity_sample": {"rows": errs[2] // w.head_dim, "max_abs": errs[0], "mean_abs": errs[1] / errs[2],
+                                 "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3},
+                                 "kv_cache_bit_exact": kv_cache_matches_oracle(w, runner.cache.cpu())}}
 
     if rank == 0:
         clocks = clk.summary()
@@ -689,6 +742,7 @@ def main():
             "e2e": {"value": round(e2e_tflops, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": runner.launches * args.steps,
+            "kv": kv_rates(w, ms),
             "clocks": clocks,
             "workloads": extra,
         }
@@ -712,7 +766,7 @@ def reference_arm(args):
     per_step = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
     vals = []
     for s in range(args.warmup + args.steps):
-        v, cores, desc, el = oracle_sample(w, per_step, seed=s)
+        v, cores, desc, el, _ = oracle_sample(w, per_step, seed=s)
         if s >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)

@@ -50,6 +50,18 @@ bool encode(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims, c
     return r == CUDA_SUCCESS;
 }
 
+// uint8 tensor map (e4m3 codes) without swizzle: rows land as plain bytes.
+bool encode_u8(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+               const cuuint32_t *box) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // The pipelined kernel runs unless LIBPREFILL_KERNEL=simple selects the
 // one-CTA-per-block kernel (used to compare the two on the same inputs).
 bool use_pipelined() {
@@ -125,7 +137,14 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
                 const float *k_fold, const float *v_fold) {
     if (!q || !k || !v || !cu || !out || !(cache || cache8) || !bt || (chunked && !ctx_lens)) return PREFILL_ERR_NULL;
     if (cache8 && (!k_scale || !v_scale)) return PREFILL_ERR_NULL;
-    if (cache8 && (cache || chunked || window > 0)) return PREFILL_ERR_UNSUPPORTED;  // whole prompts only
+    if (cache8 && (cache || window > 0)) return PREFILL_ERR_UNSUPPORTED;
+    // chunked over an FP8 cache: every key and value the chunk attends to is a
+    // cache value, the scales folded into the kernel's scores and output
+    const bool fp8_chunk = cache8 && chunked;
+    if (fp8_chunk) {
+        k_fold = k_scale;
+        v_fold = v_scale;
+    }
     if (total < 0 || num_seqs < 0 || max_q < 0 || max_ctx < 0) return PREFILL_ERR_SHAPE;
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
     if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
@@ -142,6 +161,20 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pool))
         return PREFILL_ERR_ALIGNMENT;
     if (total == 0 || num_seqs == 0 || max_q == 0) return PREFILL_OK;
+    if (fp8_chunk && (!use_pipelined() || (long long)total * n_kv_head * head_dim > (1ll << 40)))
+        return PREFILL_ERR_UNSUPPORTED;
+
+    // FP8 chunk: its codes go to the pool (the attention reads them back as the
+    // chunk's own keys and values) and into a dense copy [total][G][D] of the
+    // call's rows, from which the kernel loads its own tiles by TMA
+    uint8_t *k8 = nullptr, *v8 = nullptr;
+    if (fp8_chunk) {
+        const size_t rowb = (size_t)n_kv_head * head_dim;
+        char *ws = static_cast<char *>(device_workspace(kFp8Staging, 2 * (size_t)total * rowb, stream));
+        if (!ws) return PREFILL_ERR_CUDA;
+        k8 = reinterpret_cast<uint8_t *>(ws);
+        v8 = reinterpret_cast<uint8_t *>(ws + (size_t)total * rowb);
+    }
 
     pf::TensorMaps maps;
     const cuuint64_t D = head_dim, H = n_head, G = n_kv_head, T = total;
@@ -155,13 +188,25 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
         const cuuint32_t box[4] = {64, 1, 128, (cuuint32_t)NCH};
         if (!encode(&maps.q, q, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
-    {
+    if (fp8_chunk) {
+        // dense codes {D bytes, head, token, 1}, box {D, 1, 128, 1}: a tile's rows as plain bytes
+        const cuuint64_t dims[4] = {D, G, T, 1}, strides[3] = {D, G * D, T * G * D};
+        const cuuint32_t box[4] = {(cuuint32_t)D, 1, 128, 1};
+        if (!encode_u8(&maps.k, k8, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
+        if (!encode_u8(&maps.v, v8, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
+    } else {
         const cuuint64_t dims[4] = {64, G, T, NCH}, strides[3] = {D * 2, G * D * 2, 128};
         const cuuint32_t box[4] = {64, 1, 128, (cuuint32_t)NCH};
         if (!encode(&maps.k, k, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
         if (!encode(&maps.v, v, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
-    if (cache) {
+    if (fp8_chunk) {
+        // the FP8 pool {D bytes, head, slot, page * 2 + K/V}, box {D, 1, bs, 1}: one whole page
+        const cuuint64_t dims[4] = {D, G, (cuuint64_t)bs, (cuuint64_t)num_blocks * 2};
+        const cuuint64_t strides[3] = {D, G * D, (cuuint64_t)bs * G * D};
+        const cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)bs, 1};
+        if (!encode_u8(&maps.cache, cache8, 4, dims, strides, box)) return PREFILL_ERR_CUDA;
+    } else if (cache) {
         const cuuint64_t dims[4] = {D, G, (cuuint64_t)bs, (cuuint64_t)num_blocks * 2};
         const cuuint64_t strides[3] = {D * 2, G * D * 2, (cuuint64_t)bs * G * D * 2};
         const cuuint32_t box[4] = {64, 1, (cuuint32_t)bs, 1};
@@ -199,11 +244,33 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
     p.epoch = g_epoch.fetch_add(1) & 0x0fffffffu;
     p.k_fold = k_fold;
     p.v_fold = v_fold;
+    p.fp8 = fp8_chunk ? 1 : 0;
 
     int e;
     const bool pipelined = use_pipelined() && pf::fwd_pipelined_supported(p, head_dim);
     // the FP8 write and the folded scales live in the pipelined kernel only
     if ((cache8 || k_fold || v_fold) && !pipelined) return PREFILL_ERR_UNSUPPORTED;
+    auto store_fp8 = [&](const int32_t *ctxs, uint8_t *dk8, uint8_t *dv8) -> int {
+        pf::Fp8StoreParams sp;
+        sp.k = k;
+        sp.v = v;
+        sp.cu_seqlens = cu;
+        sp.context_lens = ctxs;
+        sp.k_scale = k_scale;
+        sp.v_scale = v_scale;
+        sp.cache8 = cache8;
+        sp.dense_k8 = dk8;
+        sp.dense_v8 = dv8;
+        sp.block_table = bt;
+        sp.status = status;
+        sp.total = total;
+        sp.num_seqs = num_seqs;
+        sp.n_kv_head = n_kv_head;
+        sp.num_blocks = num_blocks;
+        sp.mbps = mbps;
+        sp.block_size = bs;
+        return pf::launch_kv_store_fp8(sp, head_dim, stream);
+    };
     if (pipelined) {
         p.nsplit = pf::fwd_choose_splits(p);
         // caller-supplied scratch of a fixed size: the largest split count whose
@@ -222,28 +289,15 @@ int run_prefill(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16
                 p.nsplit = 1;  // no workspace: run unsplit
             }
         }
-        e = pf::launch_fwd(maps, p, head_dim, stream);
-        if (e == 0 && cache8) {
-            // FP8 cache: quantize this call's K/V rows into their slots.  A
-            // separate pass: quantizing inside the attention kernel (by its
-            // spare warps, from L2) measured slower than this launch.
-            pf::Fp8StoreParams sp;
-            sp.k = k;
-            sp.v = v;
-            sp.cu_seqlens = cu;
-            sp.context_lens = nullptr;
-            sp.k_scale = k_scale;
-            sp.v_scale = v_scale;
-            sp.cache8 = cache8;
-            sp.block_table = bt;
-            sp.status = status;
-            sp.total = total;
-            sp.num_seqs = num_seqs;
-            sp.n_kv_head = n_kv_head;
-            sp.num_blocks = num_blocks;
-            sp.mbps = mbps;
-            sp.block_size = bs;
-            e = pf::launch_kv_store_fp8(sp, head_dim, stream);
+        // FP8 chunk: the chunk's codes are stored first (the kernel reads them back)
+        e = fp8_chunk ? store_fp8(ctx_lens, k8, v8) : 0;
+        if (e == 0) e = pf::launch_fwd(maps, p, head_dim, stream);
+        if (e == 0 && cache8 && !fp8_chunk) {
+            // FP8 cache of a whole prompt: quantize this call's K/V rows into their
+            // slots after the attention (over the bf16 inputs).  A separate pass:
+            // quantizing inside the attention kernel (by its spare warps, from L2)
+            // measured slower than this launch.
+            e = store_fp8(nullptr, nullptr, nullptr);
         }
     } else {
         e = pf::launch_fwd_v0(maps, p, head_dim, stream);
@@ -292,86 +346,11 @@ int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const
                              const float *k_scale, const float *v_scale, prefill_bf16 *out, uint8_t *kv_cache_fp8,
                              int num_blocks, const int32_t *block_table, int max_blocks_per_seq, int block_size,
                              int32_t *status_dev, prefill_stream_t stream) {
-    if (!q || !k || !v || !cu_seqlens_q || !context_lens || !k_scale || !v_scale || !out || !kv_cache_fp8 ||
-        !block_table)
-        return PREFILL_ERR_NULL;
-    if (total_q < 0 || num_seqs < 0 || max_q_len < 0 || max_context_len < 0) return PREFILL_ERR_SHAPE;
-    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head != 0) return PREFILL_ERR_SHAPE;
-    if (head_dim != 64 && head_dim != 128) return PREFILL_ERR_UNSUPPORTED;
-    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return PREFILL_ERR_UNSUPPORTED;
-    if (!(std::isfinite(scale) && scale > 0.f)) return PREFILL_ERR_UNSUPPORTED;
-    if (num_blocks < 1 || max_blocks_per_seq < 1) return PREFILL_ERR_BLOCK_TABLE;
-    // each bound must fit the table (the exact per-sequence check, context +
-    // chunk length, runs on the device, where the lengths are)
-    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size ||
-        (long long)max_q_len > (long long)max_blocks_per_seq * block_size)
-        return PREFILL_ERR_BLOCK_TABLE;
-    const long long span = (long long)max_context_len + max_q_len;  // bound on every context + chunk length
-    if (num_seqs > 65535 || n_head > 65535 || span > (1 << 30)) return PREFILL_ERR_UNSUPPORTED;
-    if ((long long)num_blocks * 2 * block_size * n_kv_head * head_dim > (1ll << 40)) return PREFILL_ERR_SHAPE;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(kv_cache_fp8))
-        return PREFILL_ERR_ALIGNMENT;
-    if (total_q == 0 || num_seqs == 0 || max_q_len == 0) return PREFILL_OK;
-
-    // staging: the bf16 shadow pool (mbps2 pages per sequence), k2 / v2, the shadow table
-    const int mbps2 = (int)((span + block_size - 1) / block_size);
-    if ((long long)num_seqs * mbps2 >= (1ll << 30)) return PREFILL_ERR_UNSUPPORTED;
-    const size_t row = (size_t)n_kv_head * head_dim * 2;  // bytes of one token's K (or V) row in bf16
-    const size_t shadow_bytes = (size_t)num_seqs * mbps2 * 2 * block_size * row;
-    const size_t kv2_bytes = (size_t)total_q * row;
-    const size_t table_bytes = (size_t)num_seqs * mbps2 * sizeof(int32_t);
-    char *ws = static_cast<char *>(device_workspace(kFp8Staging, shadow_bytes + 2 * kv2_bytes + table_bytes, stream));
-    if (!ws) return PREFILL_ERR_CUDA;
-    prefill_bf16 *shadow = reinterpret_cast<prefill_bf16 *>(ws);
-    prefill_bf16 *k2 = reinterpret_cast<prefill_bf16 *>(ws + shadow_bytes);
-    prefill_bf16 *v2 = reinterpret_cast<prefill_bf16 *>(ws + shadow_bytes + kv2_bytes);
-    int32_t *table2 = reinterpret_cast<int32_t *>(ws + shadow_bytes + 2 * kv2_bytes);
-
-    // 1. the chunk's codes into the FP8 cache
-    pf::Fp8StoreParams sp;
-    sp.k = k;
-    sp.v = v;
-    sp.cu_seqlens = cu_seqlens_q;
-    sp.context_lens = context_lens;
-    sp.k_scale = k_scale;
-    sp.v_scale = v_scale;
-    sp.cache8 = kv_cache_fp8;
-    sp.block_table = block_table;
-    sp.status = status_dev;
-    sp.total = total_q;
-    sp.num_seqs = num_seqs;
-    sp.n_kv_head = n_kv_head;
-    sp.num_blocks = num_blocks;
-    sp.mbps = max_blocks_per_seq;
-    sp.block_size = block_size;
-    if (pf::launch_kv_store_fp8(sp, head_dim, stream) != 0) return PREFILL_ERR_CUDA;
-    // 2. every key and value the chunk attends to, as the e4m3 code values of
-    //    the cache (exact in bf16; the scales are applied by the attention)
-    pf::Fp8StageParams gp;
-    gp.cache8 = kv_cache_fp8;
-    gp.block_table = block_table;
-    gp.cu_seqlens = cu_seqlens_q;
-    gp.context_lens = context_lens;
-    gp.shadow = shadow;
-    gp.shadow_table = table2;
-    gp.k2 = k2;
-    gp.v2 = v2;
-    gp.status = status_dev;
-    gp.total = total_q;
-    gp.num_seqs = num_seqs;
-    gp.n_kv_head = n_kv_head;
-    gp.num_blocks = num_blocks;
-    gp.mbps = max_blocks_per_seq;
-    gp.block_size = block_size;
-    gp.mbps2 = mbps2;
-    gp.max_span = (int)span;
-    if (pf::launch_fp8_stage(gp, head_dim, stream) != 0) return PREFILL_ERR_CUDA;
-    // 3. the bf16 chunked attention over the staged code values, with the K
-    //    scales folded into the scores and the V scales into the output (it
-    //    also writes k2 / v2 into the shadow pool, which is scratch)
-    return pf::run_prefill(q, k2, v2, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len,
-                           n_head, n_kv_head, head_dim, scale, out, shadow, num_seqs * mbps2, table2, mbps2,
-                           block_size, status_dev, stream, nullptr, 0, 0, nullptr, nullptr, nullptr, k_scale, v_scale);
+    if (!kv_cache_fp8 || !context_lens) return PREFILL_ERR_NULL;
+    return pf::run_prefill(q, k, v, total_q, cu_seqlens_q, context_lens, true, num_seqs, max_q_len, max_context_len,
+                           n_head, n_kv_head, head_dim, scale, out, nullptr, num_blocks, block_table,
+                           max_blocks_per_seq, block_size, status_dev, stream, nullptr, 0, 0, kv_cache_fp8, k_scale,
+                           v_scale);
 }
 
 int prefill_attn_sliding_window(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v, int total_q,

@@ -29,9 +29,9 @@
 //  * FP8 mode (kFp8): the cache holds e4m3 codes with a scale per kv head;
 //    the ring holds code rows and the codes are widened to f16 inside the MMA
 //    fragments (see the Q K^T and P V steps), the scales folded into the
-//    scores and the output; kv_store_fp8_kernel quantizes rows into the cache,
-//    and fp8_stage_kernel dequantizes the positions a chunked prefill attends
-//    to into bf16 pages for the chunked prefill kernel.
+//    scores and the output; kv_store_fp8_kernel quantizes rows into the cache
+//    (and, for a chunked prefill over the FP8 cache, into a dense copy of the
+//    chunk's codes that the prefill kernel loads its own tiles from).
 // Earlier versions for the record: CUDA-core dot products (one FMA per
 // element) issued ~6.5k warp instructions per 64 keys and reached 19 % of the
 // DRAM bandwidth; a CTA-wide version with tensor-core MMAs and three barriers
@@ -714,6 +714,10 @@ namespace {
 // codes (x / scale, nearest even, saturating) into the token's cache slot.
 template <int D>
 __global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams p) {
+    // launched as a programmatic dependent: the kernels before it on the stream
+    // (which may still read the slots and the dense copy it writes) are complete
+    griddep_wait();
+    griddep_launch_dependents();
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (t >= p.total) return;
     int lo = 0, hi = p.num_seqs - 1;  // sequence holding row t: last i with cu_seqlens[i] <= t
@@ -749,84 +753,30 @@ __global__ void __launch_bounds__(256) kv_store_fp8_kernel(const Fp8StoreParams 
             const uint32_t c23 = quant_e4m3x2(__uint_as_float(v2.y << 16), __uint_as_float(v2.y & 0xffff0000u), sc);
             uint8_t *dst = p.cache8 + (((size_t)page * 2 + tt) * bs + pos % bs) * G * D + x;
             *reinterpret_cast<uint32_t *>(dst) = c01 | (c23 << 16);
-        }
-    }
-}
-
-// the two f16 halves of a word as fp32 (exact), the low half first
-__device__ __forceinline__ void f16x2_to_f32(uint32_t h, float &lo, float &hi) {
-    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-        : "=f"(lo), "=f"(hi)
-        : "r"(h));
-}
-
-// One warp per (sequence, position): the K and V code rows of every kv head
-// (G * D bytes each, contiguous in the slot) are widened to their code values
-// in bf16, 8 elements per lane step.  Every e4m3 value is exact in bf16 (at
-// most 4 significant bits, magnitudes 2^-9 .. 448), so nothing is rounded; the
-// per-kv-head scales are applied by the attention kernel (scores, output).
-template <int D>
-__global__ void __launch_bounds__(256) fp8_stage_kernel(const Fp8StageParams p) {
-    const int i = blockIdx.y, lane = threadIdx.x & 31;
-    const int pos = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (blockIdx.x == 0)
-        for (int x = threadIdx.x; x < p.mbps2; x += blockDim.x) p.shadow_table[(size_t)i * p.mbps2 + x] = i * p.mbps2 + x;
-    const int c0 = __ldg(&p.cu_seqlens[i]), n = __ldg(&p.cu_seqlens[i + 1]) - c0;
-    const int ctx = __ldg(&p.context_lens[i]);
-    const int bs = p.block_size;
-    if (pos >= p.max_span) return;
-    if (n < 0 || c0 < 0 || c0 + n > p.total || ctx < 0 || (long long)ctx + n > p.max_span) {
-        if (pos == 0 && lane == 0) report(p.status, PREFILL_ERR_SHAPE);
-        return;
-    }
-    if (pos >= ctx + n) return;
-    if (pos / bs >= p.mbps) {
-        if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
-        return;
-    }
-    const int page = __ldg(&p.block_table[(size_t)i * p.mbps + pos / bs]);
-    if (page < 0 || page >= p.num_blocks) {
-        if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
-        return;
-    }
-    const size_t G = p.n_kv_head, row = G * D;
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-        const uint8_t *src = p.cache8 + (((size_t)page * 2 + tt) * bs + pos % bs) * row;
-        uint16_t *dst = pos < ctx
-            ? p.shadow + ((((size_t)i * p.mbps2 + pos / bs) * 2 + tt) * bs + pos % bs) * row
-            : (tt ? p.v2 : p.k2) + (size_t)(c0 + pos - ctx) * row;
-        for (int x = lane * 8; x < (int)row; x += 32 * 8) {
-            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(src + x));
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint32_t two = ((e < 2 ? c.x : c.y) >> (16 * (e & 1))) & 0xffffu;
-                float lo, hi;
-                f16x2_to_f32(e4m3x2_to_f16x2(two), lo, hi);
-                w[e] = pack_bf16x2(lo, hi);  // exact
-            }
-            *reinterpret_cast<uint4 *>(dst + x) = make_uint4(w[0], w[1], w[2], w[3]);
+            uint8_t *dense = tt ? p.dense_v8 : p.dense_k8;
+            if (dense) *reinterpret_cast<uint32_t *>(dense + (size_t)t * G * D + x) = c01 | (c23 << 16);
         }
     }
 }
 
 }  // namespace
 
-int launch_fp8_stage(const Fp8StageParams &p, int head_dim, void *stream) {
-    if (p.num_seqs == 0 || p.max_span == 0) return 0;
-    const dim3 grid((unsigned)((p.max_span + 7) / 8), (unsigned)p.num_seqs);
-    if (head_dim == 64) fp8_stage_kernel<64><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-    else fp8_stage_kernel<128><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-    return (int)cudaGetLastError();
-}
-
 int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream) {
     if (p.total == 0) return 0;
-    const unsigned grid = (unsigned)((p.total + 7) / 8);  // one warp per token
-    if (head_dim == 64) kv_store_fp8_kernel<64><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-    else kv_store_fp8_kernel<128><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-    return (int)cudaGetLastError();
+    // one warp per token; a programmatic dependent launch (the kernel waits for
+    // its predecessors before touching memory), so that its launch, and the
+    // launch of the attention kernel that follows it, overlap the kernel before
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((p.total + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.stream = (cudaStream_t)stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    if (head_dim == 64) return (int)cudaLaunchKernelEx(&cfg, kv_store_fp8_kernel<64>, p);
+    return (int)cudaLaunchKernelEx(&cfg, kv_store_fp8_kernel<128>, p);
 }
 
 }  // namespace pf

@@ -40,37 +40,20 @@ int decode_keys_per_unit(int max_ctx);
 int launch_decode(const DecodeParams &p, int head_dim, bool fp8, void *stream);
 
 // FP8 store of a call's K/V rows into their cache slots (decode.cu).
+// Every member has a default, so that a call site that does not know a
+// member (e.g. the optional dense copy) leaves it null, never uninitialised.
 struct Fp8StoreParams {
-    const uint16_t *k, *v;        // [T][n_kv_head][D]
-    const int32_t *cu_seqlens;    // [B + 1]
-    const int32_t *context_lens;  // [B] or nullptr
-    const float *k_scale, *v_scale;
-    uint8_t *cache8;              // [NB][2][bs][n_kv_head][D]
-    const int32_t *block_table;   // [B][mbps]
-    int32_t *status;
-    int total, num_seqs, n_kv_head, num_blocks, mbps, block_size;
+    const uint16_t *k = nullptr, *v = nullptr;  // [T][n_kv_head][D]
+    const int32_t *cu_seqlens = nullptr;        // [B + 1]
+    const int32_t *context_lens = nullptr;      // [B] or nullptr
+    const float *k_scale = nullptr, *v_scale = nullptr;
+    uint8_t *cache8 = nullptr;                  // [NB][2][bs][n_kv_head][D]
+    uint8_t *dense_k8 = nullptr, *dense_v8 = nullptr;  // nullable: the same codes packed like k / v
+    const int32_t *block_table = nullptr;       // [B][mbps]
+    int32_t *status = nullptr;
+    int total = 0, num_seqs = 0, n_kv_head = 0, num_blocks = 0, mbps = 0, block_size = 0;
 };
 int launch_kv_store_fp8(const Fp8StoreParams &p, int head_dim, void *stream);
 
-// Staging of a chunked prefill over an FP8 cache (decode.cu): sequence i's
-// positions 0 .. ctx_i + n_i - 1 are read from the FP8 cache through the block
-// table and widened to their e4m3 code values in bf16 (exact; no scale); the
-// prefix (p < ctx_i) goes to a bf16 shadow pool whose block table gives
-// sequence i the pages i * mbps2 .. i * mbps2 + mbps2 - 1, the chunk's own rows
-// to k2 / v2 (packed like the call's k / v).  The bf16 chunked kernel then runs
-// on them with the per-kv-head scales folded into its scores and output.
-struct Fp8StageParams {
-    const uint8_t *cache8;        // [NB][2][bs][G][D] codes (the chunk's rows already stored)
-    const int32_t *block_table;   // [B][mbps]
-    const int32_t *cu_seqlens;    // [B + 1] chunk rows
-    const int32_t *context_lens;  // [B]
-    uint16_t *shadow;             // [B * mbps2][2][bs][G][D] bf16
-    int32_t *shadow_table;        // [B][mbps2]
-    uint16_t *k2, *v2;            // [T][G][D] bf16
-    int32_t *status;
-    int total;                    // rows of k2 / v2 (= the call's chunk rows)
-    int num_seqs, n_kv_head, num_blocks, mbps, block_size, mbps2, max_span;
-};
-int launch_fp8_stage(const Fp8StageParams &p, int head_dim, void *stream);
 
 }  // namespace pf

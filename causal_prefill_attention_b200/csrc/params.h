@@ -33,23 +33,29 @@ struct FwdParams {
     // part_nsp [total] holds, for every row of a valid sequence, its pair's split
     // count tagged with this launch's epoch ((epoch << 4) | splits), so that the
     // merge kernel skips rows that this launch did not split (or did not reach)
-    int nsplit;
-    float *part_o;
-    float *part_ml;
-    uint32_t *part_nsp;
-    uint32_t epoch;
+    int nsplit = 1;
+    float *part_o = nullptr;
+    float *part_ml = nullptr;
+    uint32_t *part_nsp = nullptr;
+    uint32_t epoch = 0;
     // per-kv-head factors folded into the scores (k_fold[g]) and into the output
     // (v_fold[g]), or nullptr (factor 1): a chunked prefill over an FP8 cache
     // stages e4m3 code values (exact in bf16) and applies the cache's scales here
-    const float *k_fold;
-    const float *v_fold;
+    const float *k_fold = nullptr;
+    const float *v_fold = nullptr;
+    // chunked prefill over an FP8 cache (the call has stored the chunk's codes
+    // already): the kernel reads every key and value as e4m3 codes -- the prefix
+    // through the block table from the FP8 pool (tensor map `cache`), the chunk's
+    // own rows from a dense copy of their codes (tensor maps `k`, `v`) -- and runs
+    // its products on f16 operands; cache (bf16) is nullptr
+    int fp8 = 0;
 };
 
 struct TensorMaps {
     CUtensorMap q;      // {64, H, T, D/64} (chunk outermost), box {64, 1, 128, D/64}
-    CUtensorMap k;      // {64, G, T, D/64}, box {64, 1, 128, D/64}
-    CUtensorMap v;      // {64, G, T, D/64}, box {64, 1, 128, D/64}
-    CUtensorMap cache;  // {D, G, bs, 2*NB}, box {64, 1, bs, 1}
+    CUtensorMap k;      // {64, G, T, D/64}, box {64, 1, 128, D/64}; FP8: uint8 {D, G, T, 1}, box {D, 1, 128, 1}
+    CUtensorMap v;      // as k
+    CUtensorMap cache;  // {D, G, bs, 2*NB}, box {64, 1, bs, 1}; FP8: uint8, box {D, 1, bs, 1}
 };
 
 // Launchers (defined per kernel file); return a cudaError_t value.

@@ -64,24 +64,41 @@ constexpr float kNoKeyMax = -1e30f;
 #endif
 constexpr uint32_t kEmuMask = PF_EXP2_EMU_MASK;
 
-template <int D, int NST>
+// Shared-memory layout.  F8: the chunked mode over an FP8 cache, whose K/V tiles
+// arrive as e4m3 bytes ([128 rows][D bytes], unswizzled) and are widened to
+// f16 in the stage: at head_dim 128 the bytes land in the upper half of the
+// stage itself (row r's bytes sit exactly where its second 64-column chunk
+// goes, so each row is read before it is overwritten), at head_dim 64 in a
+// separate staging area (STG, 8 KB per stage).
+template <int D, int NST, bool F8 = false>
 struct Lay {
     static constexpr int NCH = D / 64;
     static constexpr uint32_t TILE = NCH * CHUNK;
     static constexpr uint32_t Q0 = 0, Q1 = TILE, KV = 2 * TILE;
-    static constexpr uint32_t BAR = KV + NST * TILE;
-    // barrier slots; P is handed over in two halves (columns 0..63 -> PA, 64..127 -> PB)
+    static constexpr uint32_t RAW8 = 128u * D;  // e4m3 bytes of one K or V tile
+    static constexpr uint32_t STG = KV + NST * TILE;
+    static constexpr uint32_t BAR = STG + ((F8 && D == 64) ? NST * RAW8 : 0u);
+    // barrier slots; P is handed over in two halves (columns 0..63 -> PA, 64..127 -> PB);
+    // QRAW / KVRAW: the e4m3 (or bf16 Q) bytes have landed, before conversion (F8 only)
     static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NST, B_SFULL = 4 + 2 * NST,
                          B_PA = 6 + 2 * NST, B_PB = 8 + 2 * NST, B_OFULL = 10 + 2 * NST, B_OEMPTY = 12 + 2 * NST,
-                         NBAR = 14 + 2 * NST;
+                         B_QRAW = 14 + 2 * NST, B_KVRAW = 16 + 2 * NST, NBAR = 16 + 3 * NST;
     static constexpr uint32_t TMEM_SLOT = BAR + NBAR * 8, ABORT = TMEM_SLOT + 4;
-    static constexpr uint32_t SCHED = BAR + 256;
+    static constexpr uint32_t SCHED = BAR + 512;
     static_assert(ABORT + 4 <= SCHED, "barrier area overflow");
+    // byte offset (from the aligned base) of the e4m3 bytes of stage st
+    static constexpr uint32_t raw8(int st) { return D == 128 ? KV + st * TILE + CHUNK : STG + st * RAW8; }
 };
+
+// P to TMEM: bf16 pairs, or f16 pairs when the tensor-core operands are f16
+template <bool kF16>
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+    return kF16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
 
 // P = 2^(S*scale*log2e - m*scale*log2e) for 64 columns (half h) of one row:
 // packed FMA, exponentials, packed row sums into (sa*, sb*), bf16 pairs in pw.
-template <int h, bool kEmu>
+template <int h, bool kEmu, bool kF16>
 __device__ __forceinline__ void exp_half(const float (&x)[BN], float sl2, float nms, uint32_t (&pw)[32], float &sa0,
                                          float &sa1, float &sb0, float &sb1) {
 #pragma unroll
@@ -95,7 +112,7 @@ __device__ __forceinline__ void exp_half(const float (&x)[BN], float sl2, float 
             p1 = ex2(y1);
         }
         if (c & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
-        pw[c] = pack_bf16x2(p0, p1);
+        pw[c] = pack_p<kF16>(p0, p1);
     }
 }
 
@@ -123,7 +140,7 @@ __device__ __forceinline__ float rowmax128(const float (&x)[BN]) {
 // it by more than the threshold (2^8 in P), and only then is half 0 redone
 // and O rescaled.  Blocks whose max stays below that bound give P up to 2^8,
 // which the final O / l divides out exactly (same max for P and l).
-template <int D, bool kFull>
+template <int D, bool kFull, bool kF16>
 __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, float sl2, float thr, float &m_run,
                                               float &l_run, uint32_t tS, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
                                               int lane) {
@@ -135,7 +152,7 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
     float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
     {
         uint32_t pw[32];
-        exp_half<0, kFull>(x, sl2, -m_ref * sl2, pw, sa0, sa1, sb0, sb1);
+        exp_half<0, kFull, kF16>(x, sl2, -m_ref * sl2, pw, sa0, sa1, sb0, sb1);
         tmem_st32(tS + kPOff, pw);
     }
     float m_new = m_ref, alpha = first ? 0.f : 1.f;
@@ -150,7 +167,7 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
             sa0 = sa1 = sb0 = sb1 = 0.f;
             {
                 uint32_t pw[32];
-                exp_half<0, kFull>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
+                exp_half<0, kFull, kF16>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
                 tmem_st32(tS + kPOff, pw);
             }
 #pragma unroll 1
@@ -168,7 +185,7 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
     __syncwarp();
     if (lane == 0) mbar_arrive(b_pa);
     uint32_t pw[32];
-    exp_half<1, kFull>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
+    exp_half<1, kFull, kF16>(x, sl2, -m_new * sl2, pw, sa0, sa1, sb0, sb1);
     tmem_st32(tS + kPOff + 32, pw);
     tmem_wait_st();
     tc_fence_before();
@@ -181,7 +198,7 @@ __device__ __forceinline__ void softmax_block(const float (&x)[BN], bool first, 
 // Exponentials of 64 scores held in y64 (same arithmetic as exp_half),
 // written to TMEM as bf16 pairs at taddr in two 16-column stores so that only
 // 16 packed words are live at a time.
-template <bool kEmu>
+template <bool kEmu, bool kF16>
 __device__ __forceinline__ void exp64_store(const float (&y64)[64], float sl2, float nms, uint32_t taddr,
                                             float &sa0, float &sa1, float &sb0, float &sb1) {
 #pragma unroll
@@ -199,7 +216,7 @@ __device__ __forceinline__ void exp64_store(const float (&y64)[64], float sl2, f
                 p1 = ex2(y1);
             }
             if (c & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
-            pw[cc] = pack_bf16x2(p0, p1);
+            pw[cc] = pack_p<kF16>(p0, p1);
         }
         tmem_st16(taddr + hh * 16, pw);
     }
@@ -220,7 +237,7 @@ __device__ __forceinline__ float rowmax64x2(const float (&a)[64], const float (&
 // second 64 are still being read from TMEM; the block max is checked once both
 // halves are in (half 0 is redone and O rescaled only if it moved past the
 // threshold).  P goes to TMEM in two halves, announced on b_pa / b_pb.
-template <int D, bool kFull>
+template <int D, bool kFull, bool kF16>
 __device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lo, int lim, float sl2, float thr, float &m_run,
                                                      float &l_run, uint32_t tO, uint32_t b_pa, uint32_t b_pb,
                                                      int lane) {
@@ -240,7 +257,7 @@ __device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lo, int li
             if (c < lo || c >= lim) x0[c] = -CUDART_INF_F;
     }
     float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-    exp64_store<kFull>(x0, sl2, -m_run * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
+    exp64_store<kFull, kF16>(x0, sl2, -m_run * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
     tmem_wait_ld_tie64(r1);
 #pragma unroll
     for (int c = 0; c < 64; ++c)
@@ -252,7 +269,7 @@ __device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lo, int li
         m_new = need ? mt : m_run;
         alpha = ex2((m_run - m_new) * sl2);
         sa0 = sa1 = sb0 = sb1 = 0.f;
-        exp64_store<kFull>(x0, sl2, -m_new * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
+        exp64_store<kFull, kF16>(x0, sl2, -m_new * sl2, tS + kPOff, sa0, sa1, sb0, sb1);
 #pragma unroll 1
         for (int cc = 0; cc < D / 16; ++cc) {
             uint32_t r[16];
@@ -266,7 +283,7 @@ __device__ __forceinline__ void softmax_block_stream(uint32_t tS, int lo, int li
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(b_pa);
-    exp64_store<kFull>(x1, sl2, -m_new * sl2, tS + kPOff + 32, sa0, sa1, sb0, sb1);
+    exp64_store<kFull, kF16>(x1, sl2, -m_new * sl2, tS + kPOff + 32, sa0, sa1, sb0, sb1);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -328,8 +345,12 @@ __device__ __forceinline__ int seq_pairs(const FwdParams &p, int i, bool *bad) {
 // keys), kChunk reads a cached prefix (p.context_lens).  Without them every
 // window term, and every prefix branch (the context is the constant 0), folds
 // away at compile time.  kNoWrite leaves the cache alone (no writer warp; the
-// K/V ring is released by the MMA warp alone).
-constexpr int kModeWindow = 1, kModeChunk = 2, kModeNoWrite = 4;
+// K/V ring is released by the MMA warp alone).  kFp8 (with kChunk, kNoWrite)
+// reads every key and value as e4m3 codes -- the prefix from the FP8 cache's
+// pages, the chunk's own rows from a dense copy of their codes -- widened to
+// f16 in shared memory by warps 10-11, with Q converted to f16 the same way,
+// so the tensor cores run kind::f16 on f16 operands (P is packed as f16 too).
+constexpr int kModeWindow = 1, kModeChunk = 2, kModeNoWrite = 4, kModeFp8 = 8;
 template <bool kWin, bool kChunk>
 __device__ __forceinline__ Item decode_item(const FwdParams &p, const int *B, const int *start, const uint16_t *perm,
                                             int P, int u_split) {
@@ -401,12 +422,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_cache,
                    const FwdParams p, const int P) {
-    using L = Lay<D, NST>;
     constexpr bool kWin = (MODE & kModeWindow) != 0, kChunk = (MODE & kModeChunk) != 0;
     constexpr bool kWrite = (MODE & kModeNoWrite) == 0;
-    static_assert(kWrite || !kChunk, "a chunk's prefix is read from the cache that it appends to");
-    constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
-    constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+    constexpr bool kFp8 = (MODE & kModeFp8) != 0;
+    using L = Lay<D, NST, kFp8>;
+    // a bf16 chunk appends to the cache it reads its prefix from; an FP8 chunk's
+    // codes are stored before the kernel runs
+    static_assert(kWrite || !kChunk || kFp8, "a chunk's prefix is read from the cache that it appends to");
+    static_assert(!kFp8 || (kChunk && !kWrite && !kWin), "the FP8 mode is the chunked mode without a window");
+    constexpr uint32_t IDESC_QK = kFp8 ? idesc_f16_f32(BM, BN, false, false) : idesc_bf16_f32(BM, BN, false, false);
+    constexpr uint32_t IDESC_PV = kFp8 ? idesc_f16_f32(BM, D, false, true) : idesc_bf16_f32(BM, D, false, true);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -428,7 +453,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_prefetch_desc(&tm_v);
         if (kWrite || kChunk) tma_prefetch_desc(&tm_cache);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(L::B_QFULL + s), 1);
+            mbar_init(bar(L::B_QFULL + s), kFp8 ? 2 : 1);  // TMA (or the two converter warps)
+            if (kFp8) mbar_init(bar(L::B_QRAW + s), 1);
             mbar_init(bar(L::B_QEMPTY + s), 1);
             mbar_init(bar(L::B_SFULL + s), 1);
             mbar_init(bar(L::B_PA + s), 4);
@@ -437,7 +463,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar(L::B_OEMPTY + s), 4);
         }
         for (int s = 0; s < NST; ++s) {
-            mbar_init(bar(L::B_KVFULL + s), 1);
+            mbar_init(bar(L::B_KVFULL + s), kFp8 ? 2 : 1);
+            if (kFp8) mbar_init(bar(L::B_KVRAW + s), 1);
             mbar_init(bar(L::B_KVEMPTY + s), kWrite ? 2 : 1);  // MMA commit (+ KV writer)
         }
         *abort = 0;
@@ -546,9 +573,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int lo = (kWin && !kb.full) ? col_lo(kb, row, BN) : 0;
                 if (j != jb) {
                     if (kb.full)
-                        softmax_block_stream<D, true>(tS, lo, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
+                        softmax_block_stream<D, true, kFp8>(tS, lo, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
                     else
-                        softmax_block_stream<D, false>(tS, lo, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb, lane);
+                        softmax_block_stream<D, false, kFp8>(tS, lo, lim, sl2, thr, m_run, l_run, tO, b_pa, b_pb,
+                                                             lane);
                 } else {
                     float x[BN];
                     {
@@ -558,8 +586,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         for (int c = 0; c < BN; ++c)
                             x[c] = (c >= lo && c < lim) ? __uint_as_float(r[c]) : -CUDART_INF_F;
                     }
-                    if (kb.full) softmax_block<D, true>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
-                    else softmax_block<D, false>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
+                    if (kb.full)
+                        softmax_block<D, true, kFp8>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
+                    else
+                        softmax_block<D, false, kFp8>(x, true, sl2, thr, m_run, l_run, tS, tO, b_pa, b_pb, lane);
                 }
             }
             if (!ok) break;
@@ -645,7 +675,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     q_lastph = (q_lastph & ~(1u << s)) | (((ph_qe >> s) & 1u) << s);
                     ph_qe ^= 1u << s;
                     if (lane == 0) {
-                        const uint32_t b = bar(L::B_QFULL + s);
+                        const uint32_t b = bar(kFp8 ? L::B_QRAW + s : L::B_QFULL + s);
                         mbar_expect_tx(b, L::TILE);
                         tma_load_4d(base + (s ? L::Q1 : L::Q0), &tm_q, b, 0, it.h, it.c0 + (it.qb0 + s) * BM, 0);
                     }
@@ -656,6 +686,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // load overlaps the previous block's copies, and serves both K and V.
                 auto lane_page = [&](int jj) -> int {
                     const KvBlock kk = kv_block(it.qb0, jj, it.ctx, it.n, BM, BN, 0);
+                    if (kFp8) {
+                        if (!kk.prefix || lane >= cdiv(kk.lim_const, bs)) return 0;
+                        return __ldg(&p.block_table[(size_t)it.i * p.mbps + kk.key_begin / bs + lane]);
+                    }
                     if (!kk.prefix || lane >= (kk.lim_const / bs) * L::NCH) return 0;
                     return __ldg(&p.block_table[(size_t)it.i * p.mbps + kk.key_begin / bs + lane / L::NCH]);
                 };
@@ -675,7 +709,25 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         const uint32_t b = bar(L::B_KVFULL + stage);
                         kv_filled |= 1u << stage;
                         kv_lastph = (kv_lastph & ~(1u << stage)) | (phase << stage);
-                        if (!kb.prefix) {
+                        if (kFp8) {
+                            // e4m3 bytes into the stage's staging bytes; the converter warps
+                            // widen them (rows past the valid keys are zeroed there)
+                            const uint32_t d8 = base + L::raw8(stage);
+                            const uint32_t b8 = bar(L::B_KVRAW + stage);
+                            if (!kb.prefix) {
+                                if (lane == 0) {
+                                    mbar_expect_tx(b8, L::RAW8);
+                                    tma_load_4d(d8, t ? &tm_v : &tm_k, b8, 0, it.g, it.c0 + kb.src_row, 0);
+                                }
+                            } else {
+                                // whole pages, one box per lane (the last page may be partly valid)
+                                const int pages = cdiv(kb.lim_const, bs);
+                                if (lane == 0) mbar_expect_tx(b8, (uint32_t)(pages * bs * D));
+                                __syncwarp();
+                                if (lane < pages)
+                                    tma_load_4d(d8 + lane * bs * D, &tm_cache, b8, 0, it.g, 0, page_cur * 2 + t);
+                            }
+                        } else if (!kb.prefix) {
                             if (lane == 0) {
                                 mbar_expect_tx(b, L::TILE);
                                 tma_load_4d(dst, t ? &tm_v : &tm_k, b, 0, it.g, it.c0 + kb.src_row, 0);
@@ -728,9 +780,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // drain: every copy this warp issued has landed before the CTA can exit
             // (immediate on the normal path, where the consumers waited for them)
             for (int st = 0; st < NST; ++st)
-                if ((kv_filled >> st) & 1u) mbar_wait(bar(L::B_KVFULL + st), (kv_lastph >> st) & 1u);
+                if ((kv_filled >> st) & 1u)
+                    mbar_wait(bar(kFp8 ? L::B_KVRAW + st : L::B_KVFULL + st), (kv_lastph >> st) & 1u);
             for (int s = 0; s < 2; ++s)
-                if ((q_filled >> s) & 1u) mbar_wait(bar(L::B_QFULL + s), (q_lastph >> s) & 1u);
+                if ((q_filled >> s) & 1u)
+                    mbar_wait(bar(kFp8 ? L::B_QRAW + s : L::B_QFULL + s), (q_lastph >> s) & 1u);
             if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
         } else if (warp == WARP_MMA) {
             // ================= tcgen05 MMA issuer: the whole warp runs the loop with
@@ -839,6 +893,92 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                 }
                 used |= it.two ? 3u : 1u;
+            }
+            if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
+            __syncwarp();
+        } else if (kFp8 && warp >= WARP_WRITER) {
+            // ================= converters (FP8 mode, warps 10-11): each Q tile bf16 -> f16
+            // in place, each K/V tile e4m3 -> f16 into the stage; every e4m3 value is
+            // exact in f16, and rows past the block's valid keys become zeros (their
+            // bytes may be another sequence's, a stale page's, or anything)
+            const int cw = warp - WARP_WRITER;  // 0 or 1
+            int stage = 0;
+            uint32_t phase = 0, ph_qr = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int u = zigzag(k, cta, G);
+                if (u >= total) break;
+                const Item it = decode_item<kWin, kChunk>(p, B, start, perm, P, u);
+                if (it.skip) continue;
+                const int ns = it.two ? 2 : 1;
+                for (int s = 0; s < ns; ++s) {
+                    if (!wait_bar(bar(L::B_QRAW + s), (ph_qr >> s) & 1u, abort)) { ok = false; break; }
+                    ph_qr ^= 1u << s;
+                    uint4 *q4 = reinterpret_cast<uint4 *>(gbase + (s ? L::Q1 : L::Q0));
+                    for (int x = cw * 32 + lane; x < (int)(L::TILE / 16); x += 64) {
+                        uint4 w = q4[x];
+                        uint32_t *wv = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            wv[e] = pack_f16x2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
+                        q4[x] = w;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(L::B_QFULL + s));
+                }
+                if (!ok) break;
+                for (int j = it.j_lo; j < it.j_hi && ok; ++j) {
+                    const KvBlock kb = kv_block(it.qb0, j, it.ctx, it.n, BM, BN, 0);
+                    const int valid = kb.prefix ? kb.lim_const : imin(BN, it.n - kb.src_row);
+                    for (int t = 0; t < 2; ++t) {
+                        if (!wait_bar(bar(L::B_KVRAW + stage), phase, abort)) { ok = false; break; }
+                        const uint8_t *src8 = gbase + L::raw8(stage);
+                        uint8_t *tile = gbase + L::KV + stage * L::TILE;
+                        // D = 128: 8 lanes per 128-byte row, 4 rows per warp per round
+                        // D = 64: 4 lanes per 64-byte row, 8 rows per warp per round
+                        // Four rounds at a time: their loads are issued together, then
+                        // (after every lane's loads) their rows are written.  A row's
+                        // second chunk overlaps only that row's own bytes (D = 128).
+                        constexpr int LPR = D / 16, RPW = 32 / LPR, ROUNDS = BN / (2 * RPW), BATCH = 4;
+                        const int qp = lane % LPR;  // columns 16 qp .. 16 qp + 15
+                        const int ch = qp >> 2, u0 = (qp & 3) * 2;
+#pragma unroll 1
+                        for (int rb = 0; rb < ROUNDS; rb += BATCH) {
+                            uint4 c[BATCH];
+#pragma unroll
+                            for (int b = 0; b < BATCH; ++b) {
+                                const int r = (rb + b) * 2 * RPW + cw * RPW + lane / LPR;
+                                c[b] = r < valid ? *reinterpret_cast<const uint4 *>(src8 + r * D + qp * 16)
+                                                 : make_uint4(0, 0, 0, 0);
+                            }
+                            __syncwarp();  // the rows' bytes are read before their second chunks are written
+#pragma unroll
+                            for (int b = 0; b < BATCH; ++b) {
+                                const int r = (rb + b) * 2 * RPW + cw * RPW + lane / LPR;
+                                uint32_t h[8];
+                                h[0] = e4m3x2_to_f16x2_exact(c[b].x & 0xffffu);
+                                h[1] = e4m3x2_to_f16x2_exact(c[b].x >> 16);
+                                h[2] = e4m3x2_to_f16x2_exact(c[b].y & 0xffffu);
+                                h[3] = e4m3x2_to_f16x2_exact(c[b].y >> 16);
+                                h[4] = e4m3x2_to_f16x2_exact(c[b].z & 0xffffu);
+                                h[5] = e4m3x2_to_f16x2_exact(c[b].z >> 16);
+                                h[6] = e4m3x2_to_f16x2_exact(c[b].w & 0xffffu);
+                                h[7] = e4m3x2_to_f16x2_exact(c[b].w >> 16);
+                                uint8_t *row = tile + ch * CHUNK + r * 128;
+                                *reinterpret_cast<uint4 *>(row + ((u0 ^ (r & 7)) << 4)) =
+                                    make_uint4(h[0], h[1], h[2], h[3]);
+                                *reinterpret_cast<uint4 *>(row + (((u0 + 1) ^ (r & 7)) << 4)) =
+                                    make_uint4(h[4], h[5], h[6], h[7]);
+                            }
+                            __syncwarp();
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(L::B_KVFULL + stage));
+                        if (++stage == NST) { stage = 0; phase ^= 1; }
+                    }
+                }
             }
             if (!ok && lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
             __syncwarp();
@@ -988,9 +1128,9 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(cons
     }
 }
 
-template <int D, int NST>
+template <int D, int NST, bool F8 = false>
 size_t smem_bytes(int P, int num_seqs) {
-    return Lay<D, NST>::SCHED + (size_t)(P + 1) * 12 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
+    return Lay<D, NST, F8>::SCHED + (size_t)(P + 1) * 12 + (((size_t)num_seqs * 2 + 15) & ~size_t(15)) + 1024;
 }
 constexpr size_t kMaxSmem = 227 * 1024;
 
@@ -1019,7 +1159,7 @@ int sm_count() {
 template <int D, int NST, int MODE>
 int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
-    const size_t smem = smem_bytes<D, NST>(P, p.num_seqs);
+    const size_t smem = smem_bytes<D, NST, (MODE & kModeFp8) != 0>(P, p.num_seqs);
     cudaError_t e = cudaFuncSetAttribute(prefill_fwd_kernel<D, NST, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
@@ -1051,9 +1191,10 @@ int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
 template <int D>
 int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
     const int P = cdiv(p.max_q, 2 * BM);
-    const bool nst5 = smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem;
+    const bool nst5 = p.fp8 ? smem_bytes<D, 5, true>(P, p.num_seqs) <= kMaxSmem
+                            : smem_bytes<D, 5>(P, p.num_seqs) <= kMaxSmem;
     const int mode = (p.window > 0 ? kModeWindow : 0) | (p.context_lens ? kModeChunk : 0) |
-                     (p.cache ? 0 : kModeNoWrite);
+                     (p.cache ? 0 : kModeNoWrite) | (p.fp8 ? kModeFp8 : 0);
     switch (mode) {
         case 0: return nst5 ? launch_nst<D, 5, 0>(maps, p, stream) : launch_nst<D, 4, 0>(maps, p, stream);
         case 1: return nst5 ? launch_nst<D, 5, 1>(maps, p, stream) : launch_nst<D, 4, 1>(maps, p, stream);
@@ -1062,6 +1203,9 @@ int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
         case kModeNoWrite:
             return nst5 ? launch_nst<D, 5, kModeNoWrite>(maps, p, stream)
                         : launch_nst<D, 4, kModeNoWrite>(maps, p, stream);
+        case kModeChunk | kModeNoWrite | kModeFp8:
+            return nst5 ? launch_nst<D, 5, kModeChunk | kModeNoWrite | kModeFp8>(maps, p, stream)
+                        : launch_nst<D, 4, kModeChunk | kModeNoWrite | kModeFp8>(maps, p, stream);
         default: return (int)cudaErrorInvalidValue;  // no cache with a window or a prefix: not built
     }
 }
@@ -1072,7 +1216,9 @@ int launch(const TensorMaps &maps, const FwdParams &p, void *stream) {
 bool fwd_pipelined_supported(const FwdParams &p, int head_dim) {
     const int P = cdiv(p.max_q, 2 * BM);
     if (P > 2048 || p.num_seqs > 4096) return false;
-    const size_t smem = head_dim == 64 ? smem_bytes<64, 4>(P, p.num_seqs) : smem_bytes<128, 4>(P, p.num_seqs);
+    const size_t smem = p.fp8 ? (head_dim == 64 ? smem_bytes<64, 4, true>(P, p.num_seqs)
+                                                : smem_bytes<128, 4, true>(P, p.num_seqs))
+                              : (head_dim == 64 ? smem_bytes<64, 4>(P, p.num_seqs) : smem_bytes<128, 4>(P, p.num_seqs));
     return smem <= kMaxSmem;
 }
 

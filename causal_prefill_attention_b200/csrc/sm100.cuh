@@ -195,6 +195,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
+// Instruction descriptor for kind::f16 with f16 A and B (format code 0), fp32
+// accumulator; otherwise as idesc_bf16_f32.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                          // accumulator format: f32
+           | ((a_mn ? 1u : 0u) << 15)         // A major
+           | ((b_mn ? 1u : 0u) << 16)         // B major
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout, version 1).
 // lbo / sbo are byte offsets: for K-major operands sbo = 1024 (8 rows of 128 B)
 // and lbo is unused; for MN-major operands lbo = distance between 64-element
@@ -303,6 +313,19 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t d;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// Two floats to packed f16x2 (round to nearest even): lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// Two e4m3 codes (low byte first) to their values as packed f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_exact(uint32_t two_codes) {
+    uint32_t d;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(d) : "r"(two_codes));
     return d;
 }
 

@@ -293,13 +293,20 @@ int prefill_attn_fp8_cache(const prefill_bf16 *q, const prefill_bf16 *k, const p
  * them).  Arguments, limits and errors as for prefill_attn_chunked, with
  * k_scale / v_scale (device fp32 [n_kv_head], > 0) and the uint8 pool.
  *
- * Three launches on `stream`: the FP8 store of the chunk, a staging kernel that
- * dequantizes (code value x scale, rounded to bf16) every position the chunk
- * attends to into a bf16 workspace, and the bf16 chunked attention over it.
- * The workspace -- num_seqs x ceil((max_context_len + max_q_len) / block_size)
- * bf16 pages, plus 2 x total_q x n_kv_head x head_dim bf16 -- is allocated
- * like the split-KV workspace (first call per device and stream, grown when
- * needed, kept); PREFILL_ERR_CUDA if that allocation fails.
+ * Two launches on `stream` (three when the kv ranges are split): the FP8
+ * store of the chunk's codes, into the pool and into a dense per-call copy of
+ * the chunk's rows; then the attention kernel, which TMA-loads every key and
+ * value as e4m3 bytes -- the prefix page by page through block_table, the
+ * chunk's own rows from the dense copy -- widens them to f16 in shared memory
+ * (exact: an e4m3 value has at most 4 significant bits), converts q to f16 the
+ * same way and runs its products on f16 tensor-core operands, with each kv
+ * head's K scale folded into its scores and V scale into its output (fp32).
+ * q is taken as f16: exact for bf16 values of magnitude 2^-14 .. 65504 (larger
+ * magnitudes overflow; smaller ones lose low bits).  The dense copy, 2 x
+ * total_q x n_kv_head x head_dim bytes, is a workspace allocated like the
+ * split-KV one (first call per device and stream, grown stream-ordered, kept);
+ * PREFILL_ERR_CUDA if that allocation fails.  PREFILL_ERR_UNSUPPORTED where the
+ * pipelined kernel's schedule does not fit (as for prefill_attn_fp8_cache).
  */
 int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 *v,
                              int total_q, const int32_t *cu_seqlens_q, const int32_t *context_lens,
