@@ -175,6 +175,11 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
     constexpr int KSTEPS = D / 16;  // 16-column steps of Q K^T
     constexpr int NT = D / 8;       // 8-column output tiles
     extern __shared__ __align__(128) uint8_t smem[];
+    // a programmatic dependent launch: the kernels before it on the stream (which
+    // wrote the cache and the inputs) are complete from here on; nothing above
+    // this line reads global memory
+    griddep_wait();
+    griddep_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t ring = smem_u32(smem) + (uint32_t)warp * L::WARP_RING;
     const int W = gridDim.x * WARPS, worker = blockIdx.x * WARPS + warp;
@@ -614,6 +619,8 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
 // max and one warp sum; the O rows are then summed with independent loads.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+    griddep_wait();  // the decode kernel's partials are complete (programmatic dependent launch)
+    griddep_launch_dependents();
     const int i = blockIdx.x;
     const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -682,12 +689,24 @@ int launch_d(const DecodeParams &p, void *stream) {
     const long long ctas_needed = (units + WARPS - 1) / WARPS;
     const long long slots = (long long)kCtasPerSm * sms;
     const int grid = (int)(ctas_needed < slots ? ctas_needed : slots);
-    paged_decode_kernel<D, kFp8><<<grid, DTHREADS, smem, (cudaStream_t)stream>>>(p);
-    e = cudaGetLastError();
+    // programmatic dependent launches: each kernel may be scheduled while the one
+    // before it on the stream drains, and waits for it before touching memory
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(DTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = (cudaStream_t)stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, paged_decode_kernel<D, kFp8>, p);
     if (e != cudaSuccess || p.max_units <= 1) return (int)e;
-    dim3 cgrid((unsigned)p.num_seqs, (unsigned)cdiv(p.n_head, 4));
-    decode_combine_kernel<D><<<cgrid, 128, 0, (cudaStream_t)stream>>>(p);
-    return (int)cudaGetLastError();
+    cfg.gridDim = dim3((unsigned)p.num_seqs, (unsigned)cdiv(p.n_head, 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    return (int)cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
 }
 
 }  // namespace
