@@ -712,11 +712,13 @@ int launch_d(const DecodeParams &p, void *stream) {
 }  // namespace
 
 int decode_keys_per_unit(int max_ctx) {
-    // units of 128 keys (per-warp work within ~3 % of the mean on 64 varlen
-    // sequences, where 256-key units leave an 18 % spread), longer for very
-    // long contexts (at most kDecodeMaxUnits per sequence); always a multiple
-    // of the 16-key step
-    int u = 128;
+    // units of 256 keys, longer for very long contexts (at most
+    // kDecodeMaxUnits per sequence); always a multiple of the 16-key step.
+    // On 64 varlen sequences 128-key units even out the keys per warp better
+    // (within ~3 % of the mean against an 18 % spread), but the step measured
+    // 3 % slower: half as many units means half the partials to write and
+    // merge, which outweighs the spread
+    int u = 256;
     while (cdiv(max_ctx + 1, u) > kDecodeMaxUnits) u *= 2;
     return u;
 }
