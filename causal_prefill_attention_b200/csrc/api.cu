@@ -62,6 +62,30 @@ bool encode_u8(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims
     return r == CUDA_SUCCESS;
 }
 
+// uint8 tensor map with 128-byte swizzle (e4m3 codes in 128-byte rows).
+bool encode_u8_sw128(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+                     const cuuint32_t *box) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Decode runs the whole-page kernel where it applies unless
+// LIBPREFILL_DECODE=warp selects the per-warp kernel (used to compare the two
+// on the same inputs).
+bool use_whole_page_decode() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("LIBPREFILL_DECODE");
+        v = (e && std::strcmp(e, "warp") == 0) ? 0 : 1;
+    }
+    return v == 1;
+}
+
 // The pipelined kernel runs unless LIBPREFILL_KERNEL=simple selects the
 // one-CTA-per-block kernel (used to compare the two on the same inputs).
 bool use_pipelined() {
@@ -415,6 +439,34 @@ int run_decode(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.part_o = nullptr;
     p.part_ml = nullptr;
+    p.cache8 = fp8 ? static_cast<uint8_t *>(kv_cache) : nullptr;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    if (n_kv_head % 8 == 0 && (!fp8 || head_dim == 128) && use_whole_page_decode()) {
+        // the cache as [page * 2 + t][kv head][position][column] (innermost last):
+        // a box of 16 positions x 8 kv heads x 128 bytes is one step of one slab
+        const cuuint64_t es = fp8 ? 1 : 2;
+        const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)block_size, (cuuint64_t)n_kv_head,
+                                    2 * (cuuint64_t)num_blocks};
+        const cuuint64_t strides[3] = {(cuuint64_t)n_kv_head * head_dim * es, (cuuint64_t)head_dim * es,
+                                       (cuuint64_t)block_size * n_kv_head * head_dim * es};
+        const cuuint32_t box[4] = {fp8 ? 128u : 64u, 16u, 8u, 1u};
+        CUtensorMap tm;
+        const bool enc = fp8 ? encode_u8_sw128(&tm, kv_cache, 4, dims, strides, box)
+                             : encode(&tm, kv_cache, 4, dims, strides, box);
+        if (!enc) return PREFILL_ERR_CUDA;
+        p.grid = pf::device_sm_count();
+        // partial rows [piece id][n_head / slabs] (fp32 O, then max and sum), then
+        // the [num_seqs + 1] step scan, in the split-KV partials' workspace
+        const size_t rows = (size_t)p.grid * (n_head / (n_kv_head / 8)) + (size_t)num_seqs * n_head;
+        const size_t fbytes = rows * ((size_t)head_dim + 2) * sizeof(float);
+        char *ws = static_cast<char *>(split_workspace(fbytes + ((size_t)num_seqs + 1) * sizeof(int32_t), stream));
+        if (!ws) return PREFILL_ERR_CUDA;
+        p.part_o = reinterpret_cast<float *>(ws);
+        p.part_ml = reinterpret_cast<float *>(ws + rows * head_dim * sizeof(float));
+        p.seg_cum = reinterpret_cast<int32_t *>(ws + fbytes);
+        return pf::launch_decode_tma(p, &tm, head_dim, fp8, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+    }
     if (p.max_units > 1) {
         // partials [max_units][num_seqs][n_head][head_dim + 2] fp32, in the same
         // per-(device, stream) workspace as the prefill split-KV partials
@@ -424,9 +476,6 @@ int run_decode(const prefill_bf16 *q, const prefill_bf16 *k, const prefill_bf16 
         p.part_o = reinterpret_cast<float *>(ws);
         p.part_ml = reinterpret_cast<float *>(ws + rows * head_dim * sizeof(float));
     }
-    p.cache8 = fp8 ? static_cast<uint8_t *>(kv_cache) : nullptr;
-    p.k_scale = k_scale;
-    p.v_scale = v_scale;
     return pf::launch_decode(p, head_dim, fp8, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 

@@ -676,6 +676,586 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
 }
 
+// ------------------------------------------------------------------ whole-page decode
+// The kernel for kv-head counts that are a multiple of 8 (and, for the FP8
+// cache, head_dim 128).  The cache stores a page's tokens with all kv heads of
+// a token side by side ([bs][n_kv_head][D] per page half), so the 16 tokens of
+// a step hold 8 kv heads' rows in one contiguous 16 x 8 x D run of each half.
+// One CTA per SM takes work units (sequence, slab of 8 kv heads, key split):
+//  * warp 8 (producer) TMA-loads each step's K and V for the whole slab --
+//    boxes of 16 tokens x 8 heads x 128 bytes, 128-byte swizzled -- into a
+//    ring of 64 KB stages (bf16, head_dim 128; 32 KB otherwise), so the DRAM
+//    reads are whole contiguous page runs and one thread issues them;
+//  * warps 0-7 compute, warp w the kv head 8 * slab + w, exactly as the
+//    per-warp kernel does (Q K^T and P V on m16n8k16 MMAs from ldmatrix
+//    fragments, lazy running max), and release the stage (count 8);
+//  * the new token (position ctx, last key split) is written over its row of
+//    the loaded step by the warp of its kv head, rows past it are zeroed in V
+//    (their bytes are whatever the page holds), and its K/V go to the cache.
+// Units, key splits and the partials' layout are those of the per-warp
+// kernel, so decode_combine_kernel merges the splits of either.
+constexpr int TW = 8;          // compute warps: the kv heads of a slab
+constexpr int TTHREADS = 384;  // + a warpgroup whose warp 8 is the TMA producer (9-11 idle)
+
+template <int D, bool kFp8>
+struct TLay {
+    static constexpr int NCH = kFp8 ? 1 : D / 64;   // 128-byte chunks of a (token, head) row
+    static constexpr uint32_t HEADB = KS * 128;     // one head's 16 token rows of one chunk
+    static constexpr uint32_t CHB = TW * HEADB;     // one chunk of the slab (16 KB)
+    static constexpr uint32_t TILE = NCH * CHB;     // K (or V): 16 tokens x 8 heads
+    static constexpr uint32_t STAGE = 2 * TILE;     // K, then V
+    static constexpr int NST = (192 * 1024) / STAGE;
+    static constexpr uint32_t BAR = NST * STAGE;    // full[NST], empty[NST]
+    static constexpr uint32_t ABORT = BAR + 2 * NST * 8;
+    static constexpr uint32_t CTX = ABORT + 16;     // int32 [kDecodeMaxSeqs]
+    static constexpr uint32_t CUM = CTX + kDecodeMaxSeqs * 4;  // int32 [kDecodeMaxSeqs + 1]
+    static constexpr uint32_t BYTES = CUM + (kDecodeMaxSeqs + 1) * 4;
+    static_assert(!kFp8 || D == 128, "FP8 rows of D codes are one 128-byte swizzle row");
+    static_assert(NST >= 3, "ring depth");
+    static_assert(BYTES + 1024 <= 227 * 1024, "the CTA must fit the SM");
+};
+
+// byte offset of 16-byte slot s (0 .. 8 * NCH - 1) of token row t within one
+// head's part of a tile (bf16): 64-column chunks CHB apart, slots swizzled by
+// the row, as the TMA's 128-byte swizzle lays them out (1024-byte aligned
+// tiles; a head's 16 rows start on a 2 KB boundary)
+template <int D, bool kFp8>
+__device__ __forceinline__ uint32_t tslot_off(int t, int s) {
+    using L = TLay<D, kFp8>;
+    return (uint32_t)(s >> 3) * L::CHB + (uint32_t)t * 128 + (uint32_t)(((s & 7) ^ (t & 7)) << 4);
+}
+
+// Work of the whole-page kernel, balanced by 16-key steps.  The call's steps
+// form one list: sequence by sequence, and within a sequence slab by slab
+// (segment s = i * nslab + slab holds the sequence's cdiv(ctx + 1, 16) steps for
+// the kv heads of that slab).  CTA c takes steps [c T, (c + 1) T) of the list,
+// T = max(kMinStepsPerCta, cdiv(S, grid)) for S steps in all, so every CTA gets
+// the same number of steps whatever the context lengths.  A piece is the part
+// of one segment inside one CTA's range; a segment cut by CTA boundaries has
+// pieces c0 .. c1 (c0 = seg_start / T, c1 = (seg_end - 1) / T), and piece
+// (c, s) has the id c + s, unique and below grid + segments (a later CTA can
+// only overlap a later or the same segment), which numbers its partial rows.
+constexpr int kMinStepsPerCta = 16;  // 256 keys: no finer cuts of a short call
+__host__ __device__ __forceinline__ int steps_per_cta(int S, int grid) {
+    const int t = (S + grid - 1) / grid;
+    return t > kMinStepsPerCta ? t : kMinStepsPerCta;
+}
+
+struct TPiece {
+    int i, slab, ctx, k0, k1, nsteps;  // keys [k0, k1) of sequence i, kv heads of slab
+    int pid, npieces;                  // piece id (partial rows), pieces of its segment
+    int gnext;                         // first list step after this piece
+};
+// The piece that starts at list step g (below the CTA's end gend).
+__device__ __forceinline__ TPiece get_piece(const DecodeParams &p, const int *sctx, const int *scum, int nslab,
+                                            int T, int cta, int g, int gend) {
+    int lo = 0, hi = p.num_seqs - 1;  // last sequence with scum[i] <= g (sequences without steps are skipped)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (scum[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    TPiece o;
+    o.i = lo;
+    o.ctx = sctx[lo];
+    const int ns = cdiv(o.ctx + 1, KS);
+    const int rel = g - scum[lo];
+    o.slab = rel / ns;
+    const int seg_start = scum[lo] + o.slab * ns, seg_end = seg_start + ns;
+    const int a = g - seg_start, b = min(seg_end, gend) - seg_start;
+    o.k0 = a * KS;
+    o.k1 = min(b * KS, o.ctx + 1);
+    o.nsteps = b - a;
+    o.npieces = (seg_end - 1) / T - seg_start / T + 1;
+    o.pid = cta + lo * nslab + o.slab;
+    o.gnext = seg_start + b;
+    return o;
+}
+
+template <int D, bool kFp8>
+__global__ void __launch_bounds__(TTHREADS, 1)
+paged_decode_tma_kernel(const __grid_constant__ CUtensorMap tm, const DecodeParams p) {
+    using L = TLay<D, kFp8>;
+    constexpr int KSTEPS = D / 16;  // 16-column steps of Q K^T
+    constexpr int NT = D / 8;       // 8-column output tiles
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle atoms: 1024-byte aligned tiles
+    uint8_t *sm = smem_raw + (base - raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bs = p.block_size, r = p.n_head / p.n_kv_head;
+    const size_t G = p.n_kv_head;
+    const int nslab = p.n_kv_head / TW;
+    volatile int *abort = reinterpret_cast<volatile int *>(sm + L::ABORT);
+    auto full = [&](int s) -> uint32_t { return base + L::BAR + 8u * s; };
+    auto empty = [&](int s) -> uint32_t { return base + L::BAR + 8u * (L::NST + s); };
+    if (tid == 0) {
+        tma_prefetch_desc(&tm);
+        for (int s = 0; s < L::NST; ++s) {
+            mbar_init(full(s), 1);    // the producer's expect_tx (+ the TMA bytes)
+            mbar_init(empty(s), TW);  // one arrive per compute warp
+        }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    // a programmatic dependent launch: nothing above this line reads global memory
+    griddep_wait();
+    griddep_launch_dependents();
+
+    // context lengths and an exclusive scan of the units per sequence
+    int *sctx = reinterpret_cast<int *>(sm + L::CTX);
+    int *scum = reinterpret_cast<int *>(sm + L::CUM);
+    __shared__ int s_wsum[TTHREADS / 32];
+    {
+        constexpr int PER = (kDecodeMaxSeqs + TTHREADS - 1) / TTHREADS;  // covers index num_seqs too
+        int cnt[PER], run = 0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int i = tid * PER + e;
+            int c = 0;
+            if (i < p.num_seqs) {
+                const int ctx = __ldg(&p.context_lens[i]);
+                sctx[i] = ctx;
+                if (ctx < 0 || ctx > p.max_ctx || (long long)ctx + 1 > (long long)p.mbps * p.block_size) {
+                    if (blockIdx.x == 0) report(p.status, PREFILL_ERR_SHAPE);
+                } else {
+                    c = cdiv(ctx + 1, KS) * nslab;  // the sequence's steps, all slabs
+                }
+            }
+            cnt[e] = run;
+            run += c;
+        }
+        int incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int base_u = incl - run;
+        for (int w2 = 0; w2 < warp; ++w2) base_u += s_wsum[w2];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int i = tid * PER + e;
+            if (i <= p.num_seqs) {
+                scum[i] = base_u + cnt[e];
+                if (blockIdx.x == 0 && p.seg_cum) p.seg_cum[i] = base_u + cnt[e];  // for the merge kernel
+            }
+        }
+    }
+    __syncthreads();  // the last CTA-wide barrier
+    const int S = scum[p.num_seqs];
+    const int T = steps_per_cta(S, gridDim.x), cta = blockIdx.x;
+    const int gbeg = min(cta * T, S), gend = min(gbeg + T, S);  // this CTA's steps
+
+    // register split (384 threads x 168 at launch = 64,512): compute warpgroups
+    // 2 x 128 x 224, the producer's warpgroup 128 x 56
+    if (warp >= TW) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+        if (warp != TW) return;
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    }
+    if (warp == TW) {
+        // ================= producer: one step = K and V of 16 tokens x 8 kv heads
+        int stage = 0;
+        uint32_t phase = 0, filled = 0, lastph = 0;
+        bool ok = true;
+        for (int g = gbeg; ok && g < gend;) {
+            const TPiece u = get_piece(p, sctx, scum, nslab, T, cta, g, gend);
+            g = u.gnext;
+            for (int s = 0; s < u.nsteps; ++s) {
+                const int p0 = u.k0 + s * KS;  // a step lies in one page (pages hold multiples of 16)
+                int page = 0;
+                if (lane == 0) page = __ldg(&p.block_table[(size_t)u.i * p.mbps + p0 / bs]);
+                page = __shfl_sync(0xffffffffu, page, 0);
+                if (page < 0 || page >= p.num_blocks) {
+                    if (lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                    page = p.num_blocks;  // outside the map: the boxes read zeros
+                }
+                if (!mbar_wait(empty(stage), phase ^ 1u, abort)) { ok = false; break; }
+                filled |= 1u << stage;
+                lastph = (lastph & ~(1u << stage)) | (phase << stage);
+                if (lane == 0) mbar_expect_tx(full(stage), L::STAGE);
+                __syncwarp();
+                if (lane < 2 * L::NCH) {  // lanes issue together: K chunks, then V chunks
+                    const int t = lane / L::NCH, c = lane % L::NCH;
+                    tma_load_4d(base + stage * L::STAGE + t * L::TILE + c * L::CHB, &tm, full(stage), c * 64,
+                                p0 % bs, u.slab * TW, page * 2 + t);
+                }
+                if (++stage == L::NST) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (!ok) {
+            *abort = 1;
+            if (lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
+        }
+        // no copy may be in flight when the CTA ends
+        for (int st = 0; st < L::NST; ++st)
+            if ((filled >> st) & 1u) mbar_wait(full(st), (lastph >> st) & 1u);
+        return;
+    }
+
+    // ================= compute warps: warp w runs kv head 8 * slab + w of each unit
+    const int row0 = lane >> 2, row1 = row0 + 8, c2 = 2 * (lane & 3);
+    auto load_q = [&](int i, int g, uint32_t (&qa)[KSTEPS][4]) {
+        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(p.q + ((size_t)i * p.n_head + (size_t)g * r) * D);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            // FP8: the columns of a 16-column step are permuted to the K codes'
+            // order in the widened fragments (see paged_decode_kernel)
+            const int c = kFp8 ? kk * 16 + 2 * c2 : kk * 16 + c2;
+            const int c_hi = kFp8 ? c + 2 : c + 8;
+            qa[kk][0] = row0 < r ? __ldg(q0 + (row0 * D + c) / 2) : 0u;
+            qa[kk][1] = row1 < r ? __ldg(q0 + (row1 * D + c) / 2) : 0u;
+            qa[kk][2] = row0 < r ? __ldg(q0 + (row0 * D + c_hi) / 2) : 0u;
+            qa[kk][3] = row1 < r ? __ldg(q0 + (row1 * D + c_hi) / 2) : 0u;
+            if constexpr (kFp8) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    qa[kk][e] = pack_f16x2(__uint_as_float(qa[kk][e] << 16), __uint_as_float(qa[kk][e] & 0xffff0000u));
+            }
+        }
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    bool has = gbeg < gend;
+    TPiece uc;
+    if (has) uc = get_piece(p, sctx, scum, nslab, T, cta, gbeg, gend);
+    uint32_t qa[KSTEPS][4], qn[KSTEPS][4];
+    if (has) load_q(uc.i, uc.slab * TW + warp, qa);
+#pragma unroll 1
+    while (has) {
+        const int g = uc.slab * TW + warp;
+        const float sl2 = kFp8 ? p.scale_log2 * __ldg(&p.k_scale[g]) : p.scale_log2, thr = kLazyLog2 / sl2;
+        float m_ref[2] = {-CUDART_INF_F, -CUDART_INF_F};
+        float l_part[2] = {0.f, 0.f};
+        float o[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+        const bool has_n = uc.gnext < gend;
+        TPiece un;
+        if (has_n) un = get_piece(p, sctx, scum, nslab, T, cta, uc.gnext, gend);
+#pragma unroll 1
+        for (int sc = 0; sc < uc.nsteps; ++sc) {
+            if (!mbar_wait(full(stage), phase, abort)) { ok = false; break; }
+            const uint32_t kt = base + stage * L::STAGE + warp * L::HEADB;  // this head's K rows
+            const uint32_t vt = kt + L::TILE;                                // and V rows
+            const int p0 = uc.k0 + sc * KS;
+            if (uc.ctx >= p0 && uc.ctx < p0 + KS) {
+                // the new token's step: its row comes from the inputs (and goes to
+                // its cache slot); V rows past it are zeroed, since P is 0 there but
+                // the page's bytes may hold anything (a NaN would survive 0 x NaN)
+                const int nr = uc.ctx - p0;
+                const int page = __ldg(&p.block_table[(size_t)uc.i * p.mbps + uc.ctx / bs]);
+                const bool page_ok = page >= 0 && page < p.num_blocks;
+                if (!page_ok && lane == 0) report(p.status, PREFILL_ERR_BLOCK_TABLE);
+                if constexpr (kFp8) {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const uint16_t *src = (t ? p.v : p.k) + ((size_t)uc.i * G + g) * D;
+                        const float sc_t = __ldg(&(t ? p.v_scale : p.k_scale)[g]);
+                        const int e = lane * 4;  // 4 codes per lane (D = 128)
+                        const uint2 x = __ldg(reinterpret_cast<const uint2 *>(src + e));
+                        const uint32_t c01 = quant_e4m3x2(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u), sc_t);
+                        const uint32_t c23 = quant_e4m3x2(__uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u), sc_t);
+                        const uint32_t word = c01 | (c23 << 16);
+                        *reinterpret_cast<uint32_t *>(sm + ((t ? vt : kt) - base) + f8_off<D>(nr, e / 16) + e % 16) = word;
+                        if (page_ok)
+                            *reinterpret_cast<uint32_t *>(p.cache8 + ((((size_t)page * 2 + t) * bs + uc.ctx % bs) * G + g) * D + e) = word;
+                    }
+                    for (int x = lane; x < (KS - 1 - nr) * (D / 16); x += 32) {
+                        const int row = nr + 1 + x / (D / 16), seg = x % (D / 16);
+                        *reinterpret_cast<uint4 *>(sm + (vt - base) + f8_off<D>(row, seg)) = make_uint4(0, 0, 0, 0);
+                    }
+                } else {
+                    constexpr int SPR = D / 8;  // 16-byte slots per row
+                    if (lane < 2 * SPR) {
+                        const int t = lane / SPR, s = lane % SPR;
+                        const uint4 val =
+                            __ldg(reinterpret_cast<const uint4 *>((t ? p.v : p.k) + ((size_t)uc.i * G + g) * D) + s);
+                        *reinterpret_cast<uint4 *>(sm + ((t ? vt : kt) - base) + tslot_off<D, kFp8>(nr, s)) = val;
+                        if (page_ok)
+                            reinterpret_cast<uint4 *>(p.cache + ((((size_t)page * 2 + t) * bs + uc.ctx % bs) * G + g) * D)[s] = val;
+                    }
+                    for (int x = lane; x < (KS - 1 - nr) * SPR; x += 32) {
+                        const int row = nr + 1 + x / SPR, s = x % SPR;
+                        *reinterpret_cast<uint4 *>(sm + (vt - base) + tslot_off<D, kFp8>(row, s)) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                fence_proxy_async_smem();  // these writes come before the stage's next TMA fill
+                __syncwarp();
+            }
+
+            if (sc == uc.nsteps - 1 && has_n) load_q(un.i, un.slab * TW + warp, qn);  // the next unit's queries
+
+            // ---- S = Q K^T for the step's 16 keys (two 8-key tiles)
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+                const int m = lane >> 3;
+                if constexpr (kFp8) {
+                    const int kr = (m & 1) * 8 + (lane & 7);
+#pragma unroll
+                    for (int j = 0; j < D / 32; ++j) {
+                        uint32_t w[4];
+                        ldsm_x4(kt + f8_off<D>(kr, 2 * j + (m >> 1)), w);
+                        mma16816<true>(s0, qa[2 * j], e4m3x2_to_f16x2(w[0] & 0xffffu), e4m3x2_to_f16x2(w[0] >> 16));
+                        mma16816<true>(s1, qa[2 * j], e4m3x2_to_f16x2(w[1] & 0xffffu), e4m3x2_to_f16x2(w[1] >> 16));
+                        mma16816<true>(t0, qa[2 * j + 1], e4m3x2_to_f16x2(w[2] & 0xffffu), e4m3x2_to_f16x2(w[2] >> 16));
+                        mma16816<true>(t1, qa[2 * j + 1], e4m3x2_to_f16x2(w[3] & 0xffffu), e4m3x2_to_f16x2(w[3] >> 16));
+                    }
+                } else {
+                    const int kr = (m >> 1) * 8 + (lane & 7);  // matrices: keys 0-7 / 8-15 x columns +0 / +8
+#pragma unroll
+                    for (int kk = 0; kk < KSTEPS; kk += 2) {
+                        uint32_t kb[4], kc[4];
+                        ldsm_x4(kt + tslot_off<D, kFp8>(kr, 2 * kk + (m & 1)), kb);
+                        ldsm_x4(kt + tslot_off<D, kFp8>(kr, 2 * kk + 2 + (m & 1)), kc);
+                        mma16816<false>(s0, qa[kk], kb[0], kb[1]);
+                        mma16816<false>(s1, qa[kk], kb[2], kb[3]);
+                        mma16816<false>(t0, qa[kk + 1], kc[0], kc[1]);
+                        mma16816<false>(t1, qa[kk + 1], kc[2], kc[3]);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    s0[e] += t0[e];
+                    s1[e] += t1[e];
+                }
+            }
+            const int nvalid = uc.k1 - p0;
+            if (c2 >= nvalid) s0[0] = s0[2] = -CUDART_INF_F;
+            if (c2 + 1 >= nvalid) s0[1] = s0[3] = -CUDART_INF_F;
+            if (c2 + 8 >= nvalid) s1[0] = s1[2] = -CUDART_INF_F;
+            if (c2 + 9 >= nvalid) s1[1] = s1[3] = -CUDART_INF_F;
+            float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
+            float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            const bool mv0 = mx0 > m_ref[0] + thr, mv1 = mx1 > m_ref[1] + thr;
+            if (__any_sync(0xffffffffu, mv0 || mv1)) {
+                const float n0 = mv0 ? mx0 : m_ref[0], n1 = mv1 ? mx1 : m_ref[1];
+                const float a0 = ex2((m_ref[0] - n0) * sl2), a1 = ex2((m_ref[1] - n1) * sl2);
+                m_ref[0] = n0;
+                m_ref[1] = n1;
+                l_part[0] *= a0;
+                l_part[1] *= a1;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    o[nt][0] *= a0;
+                    o[nt][1] *= a0;
+                    o[nt][2] *= a1;
+                    o[nt][3] *= a1;
+                }
+            }
+            const float nm0 = -m_ref[0] * sl2, nm1 = -m_ref[1] * sl2;
+            const float p00 = ex2(fmaf(s0[0], sl2, nm0)), p01 = ex2(fmaf(s0[1], sl2, nm0));
+            const float p02 = ex2(fmaf(s0[2], sl2, nm1)), p03 = ex2(fmaf(s0[3], sl2, nm1));
+            const float p10 = ex2(fmaf(s1[0], sl2, nm0)), p11 = ex2(fmaf(s1[1], sl2, nm0));
+            const float p12 = ex2(fmaf(s1[2], sl2, nm1)), p13 = ex2(fmaf(s1[3], sl2, nm1));
+            l_part[0] += (p00 + p01) + (p10 + p11);
+            l_part[1] += (p02 + p03) + (p12 + p13);
+            uint32_t pa[4];
+            if constexpr (kFp8) {
+                pa[0] = pack_f16x2(p00, p01);
+                pa[1] = pack_f16x2(p02, p03);
+                pa[2] = pack_f16x2(p10, p11);
+                pa[3] = pack_f16x2(p12, p13);
+            } else {
+                pa[0] = pack_bf16x2(p00, p01);
+                pa[1] = pack_bf16x2(p02, p03);
+                pa[2] = pack_bf16x2(p10, p11);
+                pa[3] = pack_bf16x2(p12, p13);
+            }
+            // ---- O += P V over all output columns
+            {
+                const int m = lane >> 3;
+                const int vr = (m & 1) * 8 + (lane & 7);
+                if constexpr (kFp8) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t w[4];
+                        ldsm_x4_t(vt + f8_off<D>(vr, 2 * c + (m >> 1)), w);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t lo = w[2 * h], hi = w[2 * h + 1];
+                            mma16816<true>(o[4 * c + 2 * h], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0020)),
+                                           e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0020)));
+                            mma16816<true>(o[4 * c + 2 * h + 1], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0031)),
+                                           e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0031)));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NT / 2; ++c) {
+                        uint32_t vb[4];
+                        ldsm_x4_t(vt + tslot_off<D, kFp8>(vr, 2 * c + (m >> 1)), vb);
+                        mma16816<false>(o[2 * c], pa, vb[0], vb[1]);
+                        mma16816<false>(o[2 * c + 1], pa, vb[2], vb[3]);
+                    }
+                }
+            }
+            __syncwarp();  // every lane's reads of the stage are done
+            if (lane == 0) mbar_arrive(empty(stage));
+            if (++stage == L::NST) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+
+        // ---- end of the unit: row sums over the 4 lanes of a row, then rows < r out
+        float l0 = l_part[0], l1 = l_part[1];
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+        const bool whole = uc.npieces == 1;
+        const size_t hrow = (size_t)uc.i * p.n_head + (size_t)g * r;
+        // partial rows of this piece: [pid][8 r heads of the slab]
+        const size_t prow0 = (size_t)uc.pid * (TW * r) + (size_t)warp * r;
+        const float vsc = kFp8 ? __ldg(&p.v_scale[g]) : 1.f;  // the V codes' scale
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = hh ? row1 : row0;
+            if (h >= r) continue;
+            const float lsum = hh ? l1 : l0;
+            const size_t row = hrow + h;
+            const size_t prow = prow0 + h;
+            if constexpr (kFp8) {
+                const float f = whole ? vsc / lsum : vsc;
+#pragma unroll
+                for (int sg = 0; sg < D / 16; ++sg) {
+                    const float *ev = o[4 * (sg >> 1) + 2 * (sg & 1)], *od = o[4 * (sg >> 1) + 2 * (sg & 1) + 1];
+                    const float v0 = ev[2 * hh] * f, v1 = od[2 * hh] * f, v2 = ev[2 * hh + 1] * f, v3 = od[2 * hh + 1] * f;
+                    const int col = 16 * sg + 2 * c2;
+                    if (whole)
+                        *reinterpret_cast<uint2 *>(p.out + row * D + col) = make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
+                    else
+                        *reinterpret_cast<float4 *>(p.part_o + prow * D + col) = make_float4(v0, v1, v2, v3);
+                }
+            } else if (whole) {
+                const float inv = 1.f / lsum;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<uint32_t *>(p.out + row * D + nt * 8 + c2) =
+                        pack_bf16x2(o[nt][2 * hh] * inv, o[nt][2 * hh + 1] * inv);
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<float2 *>(p.part_o + prow * D + nt * 8 + c2) =
+                        make_float2(o[nt][2 * hh], o[nt][2 * hh + 1]);
+            }
+            if (!whole && (lane & 3) == 0)
+                *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_ref[hh] * sl2, lsum);
+        }
+        has = has_n;
+        uc = un;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) qa[kk][e] = qn[kk][e];
+    }
+    if (!ok) {
+        *abort = 1;
+        if (lane == 0) report(p.status, PREFILL_ERR_TIMEOUT);
+    }
+}
+
+// Merge of the pieces of a segment cut by CTA boundaries (the whole-page
+// kernel's split work): one warp per (sequence, query head), the
+// online-softmax merge rule over the pieces' (max, sum, O) -- any number of
+// pieces, 32 at a time.  A segment in one piece was written by the kernel.
+template <int D>
+__global__ void __launch_bounds__(128) decode_merge_pieces_kernel(const DecodeParams p) {
+    griddep_wait();  // the decode kernel's partials and step scan are complete
+    griddep_launch_dependents();
+    const int i = blockIdx.x;
+    const int hq = blockIdx.y * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (hq >= p.n_head) return;
+    const int ctx = p.context_lens[i];
+    if (ctx < 0 || ctx > p.max_ctx || (long long)ctx + 1 > (long long)p.mbps * p.block_size) return;
+    const int nslab = p.n_kv_head / TW, r = p.n_head / p.n_kv_head;
+    const int g = hq / r, slab = g / TW, w = g % TW, h = hq % r;
+    const int T = steps_per_cta(p.seg_cum[p.num_seqs], p.grid);
+    const int ns = cdiv(ctx + 1, KS);
+    const int seg_start = p.seg_cum[i] + slab * ns, seg_end = seg_start + ns;
+    const int c0 = seg_start / T, np = (seg_end - 1) / T - c0 + 1;
+    if (np <= 1) return;
+    const size_t base_row = (size_t)(c0 + i * nslab + slab) * ((size_t)TW * r) + (size_t)w * r + h;
+    const size_t pstride = (size_t)TW * r;  // rows between consecutive pieces of the segment
+    constexpr int E = D / 32;
+    float M = -CUDART_INF_F;
+    for (int c = lane; c < np; c += 32) M = fmaxf(M, __ldcg(p.part_ml + (base_row + c * pstride) * 2));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int cb = 0; cb < np; cb += 32) {
+        float wl = 0.f;
+        if (cb + lane < np) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + (base_row + (cb + lane) * pstride) * 2));
+            wl = ex2(ml.x - M);
+            L += wl * ml.y;
+        }
+        const int nb = min(32, np - cb);
+#pragma unroll 4
+        for (int j = 0; j < nb; ++j) {
+            const float wgt = __shfl_sync(0xffffffffu, wl, j);
+            const float *src = p.part_o + (base_row + (cb + j) * pstride) * D + lane * E;
+            if constexpr (E == 4) {
+                const float4 f = __ldcg(reinterpret_cast<const float4 *>(src));
+                acc[0] += wgt * f.x;
+                acc[1] += wgt * f.y;
+                acc[2] += wgt * f.z;
+                acc[3] += wgt * f.w;
+            } else {
+                const float2 f = __ldcg(reinterpret_cast<const float2 *>(src));
+                acc[0] += wgt * f.x;
+                acc[1] += wgt * f.y;
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    const float inv = 1.f / L;
+    uint16_t *dst = p.out + ((size_t)i * p.n_head + hq) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+}
+
+template <int D, bool kFp8>
+int launch_dt(const DecodeParams &p, const CUtensorMap &tm, void *stream) {
+    using L = TLay<D, kFp8>;
+    const size_t smem = L::BYTES + 1024;
+    cudaError_t e = cudaFuncSetAttribute(paged_decode_tma_kernel<D, kFp8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return (int)e;
+    const int grid = p.grid;  // steps_per_cta divides the call's steps over exactly this many CTAs
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(TTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = (cudaStream_t)stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, paged_decode_tma_kernel<D, kFp8>, tm, p);
+    // no segment can be cut when all steps fit in one CTA's share
+    const long long steps_bound = (long long)p.num_seqs * (p.n_kv_head / TW) * cdiv(p.max_ctx + 1, KS);
+    if (e != cudaSuccess || steps_bound <= kMinStepsPerCta) return (int)e;
+    cfg.gridDim = dim3((unsigned)p.num_seqs, (unsigned)cdiv(p.n_head, 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    return (int)cudaLaunchKernelEx(&cfg, decode_merge_pieces_kernel<D>, p);
+}
+
 template <int D, bool kFp8>
 int launch_d(const DecodeParams &p, void *stream) {
     using L = DecLay<D, kFp8>;
@@ -726,6 +1306,11 @@ int decode_keys_per_unit(int max_ctx) {
 int launch_decode(const DecodeParams &p, int head_dim, bool fp8, void *stream) {
     if (fp8) return head_dim == 64 ? launch_d<64, true>(p, stream) : launch_d<128, true>(p, stream);
     return head_dim == 64 ? launch_d<64, false>(p, stream) : launch_d<128, false>(p, stream);
+}
+
+int launch_decode_tma(const DecodeParams &p, const CUtensorMap *tm, int head_dim, bool fp8, void *stream) {
+    if (fp8) return launch_dt<128, true>(p, *tm, stream);
+    return head_dim == 64 ? launch_dt<64, false>(p, *tm, stream) : launch_dt<128, false>(p, *tm, stream);
 }
 
 namespace {

@@ -1,5 +1,7 @@
 // decode.h -- launch parameters of the paged decode kernels (decode.cu).
 #pragma once
+#include <cuda.h>
+
 #include <cstdint>
 
 namespace pf {
@@ -34,10 +36,22 @@ struct DecodeParams {
     // part_o [max_units][B][n_head][D] (fp32, unnormalised), part_ml [..][2] (max in log2 units, sum)
     float *part_o;
     float *part_ml;
+    // whole-page kernel: its grid (CTAs; the call's 16-key steps are divided
+    // evenly over them), and [num_seqs + 1] steps before each sequence (written
+    // by the kernel for the merge kernel).  Its partial rows are
+    // [piece id][n_head / slabs] (see get_piece), at most
+    // grid * n_head / slabs + num_seqs * n_head rows.
+    int grid = 0;
+    int32_t *seg_cum = nullptr;
 };
 
 int decode_keys_per_unit(int max_ctx);
 int launch_decode(const DecodeParams &p, int head_dim, bool fp8, void *stream);
+// The whole-page kernel (n_kv_head a multiple of 8; head_dim 128 for the FP8
+// cache): tm maps the cache as [2 * num_blocks][n_kv_head][block_size][head_dim]
+// (innermost last; the token dimension is strided past the kv heads), boxes of
+// 16 tokens x 8 kv heads x 128 bytes with 128-byte swizzle.
+int launch_decode_tma(const DecodeParams &p, const CUtensorMap *tm, int head_dim, bool fp8, void *stream);
 
 // FP8 store of a call's K/V rows into their cache slots (decode.cu).
 // Every member has a default, so that a call site that does not know a

@@ -86,4 +86,7 @@ int run_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int tot
                 size_t scratch_bytes, int window = 0, uint8_t *cache8 = nullptr, const float *k_scale = nullptr,
                 const float *v_scale = nullptr, const float *k_fold = nullptr, const float *v_fold = nullptr);
 
+// SM count of the current device (cached per device ordinal).
+int device_sm_count();
+
 }  // namespace pf

@@ -1227,6 +1227,8 @@ bool fwd_pipelined_supported(const FwdParams &p, int head_dim) {
 // per step on the 512-row chunks of an 8k GQA prompt.
 constexpr double kSplitCostSteps = 6.0;
 
+int device_sm_count() { return sm_count(); }
+
 int fwd_choose_splits(const FwdParams &p) {
     // Split only when the call has fewer work items than SMs: pick the split
     // count (up to 8) that minimises waves x blocks per split + the split's
