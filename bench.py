@@ -212,6 +212,17 @@ class WindowRunner(PlainRunner):
 WINDOW_LINE = ("swa4096_gqa_s8192_h32g8_d128", "gqa_s8192_h32g8_d128", 4096)
 
 
+def decode_launches(num_seqs: int, n_kv_head: int, max_ctx: int) -> int:
+    """Kernels one decode call launches.  kv-head counts that are a multiple of
+    8 (the workloads here) run the whole-page kernel, then the merge of the
+    sequences cut between CTAs unless the call's 16-key steps fit one CTA's
+    share (16 steps); other counts run the per-warp kernel, then a merge when a
+    sequence has more than one 256-key unit."""
+    if n_kv_head % 8 == 0:
+        return 1 + int(num_seqs * (n_kv_head // 8) * -(-(max_ctx + 1) // 16) > 16)
+    return 1 + int(-(-(max_ctx + 1) // 256) > 1)
+
+
 class DecodeRunner:
     """One decode step (paged_decode_attn) for the 64 sequences of the varlen
     workload: their prompts are prefilled once by prefill_attn (which writes the
@@ -239,7 +250,7 @@ class DecodeRunner:
         self.bytes = (int(ctx.sum()) * G * D * 2 * 2        # cached K and V, read once
                       + B * H * D * 2 * 2                   # q in, out
                       + B * G * D * 2 * 2 * 2)              # new k, v in and into the cache
-        self.launches = 2 if -(-(self.max_ctx + 1) // 512) > 1 else 1
+        self.launches = decode_launches(B, G, self.max_ctx)
         self.tokens = B
 
     def step(self):
@@ -375,7 +386,7 @@ class DecodeFp8Runner:
                       + B * H * D * 2 * 2                 # q in, out
                       + B * G * D * 2 * 2                 # new k, v in
                       + B * G * D * 2)                    # their codes into the cache
-        self.launches = 2 if -(-(self.max_ctx + 1) // 128) > 1 else 1
+        self.launches = decode_launches(len(w.seqlens), w.n_kv_head, self.max_ctx)
         self.tokens = B
         self.prompt = (pk.to(d), pv.to(d), pcu.to(d))
         # bytes of one store of the prompts: bf16 K and V read, their codes written
@@ -598,6 +609,43 @@ def kv_rates(w: W.Workload, ms: float) -> dict:
 
 
 # ------------------------------------------------------------------ main
+def _only_runner(name: str, stream):
+    if name == DECODE_LINE[0]:
+        return DecodeRunner(W.named_workload(DECODE_LINE[1]), DECODE_LINE[2], stream), True
+    if name == DECODE_FP8_LINE[0]:
+        return DecodeFp8Runner(W.named_workload(DECODE_FP8_LINE[1]), DECODE_FP8_LINE[2], stream), True
+    if name == QKV_LINE[0]:
+        return QkvRunner(*QKV_LINE[1:], stream), False
+    if name == OUT_LINE[0]:
+        return OutProjRunner(*OUT_LINE[1:], stream), False
+    if name == WINDOW_LINE[0]:
+        return WindowRunner(W.named_workload(WINDOW_LINE[1]), WINDOW_LINE[2], stream), False
+    raise ValueError(name)
+
+
+ONLY_LINES = ("decode64_gqa_h32g8_d128", "decode64_fp8_gqa_h32g8_d128", "qkv_proj_s8192_h4096_n6144",
+              "out_proj_s8192_h4096", "swa4096_gqa_s8192_h32g8_d128")
+
+
+def run_only(args) -> int:
+    """One secondary line alone: W warm-up steps, then K timed steps (CUDA
+    events, L2 flushed before each), one JSON line with the median."""
+    stream = torch.cuda.current_stream()
+    runner, hbm = _only_runner(args.only, stream)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    durs = time_steps(runner, args.steps, args.warmup, stream, flush, clean=hbm)
+    runner.check_status()
+    m = statistics.median(durs)
+    line = {"line": args.only, "ms": round(m, 4), "steps": args.steps, "warmup": args.warmup,
+            "launches_per_step": runner.launches}
+    if hbm:
+        line["gbs"] = round(runner.bytes / (m * 1e-3) / 1e9, 1)
+    else:
+        line["tflops"] = round(runner.flops / (m * 1e-3) / 1e12, 2)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -608,6 +656,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--workload", default=HEADLINE, choices=list(W.NAMED),
                     help="workload timed as the step (default: the 8k GQA prompt)")
+    ap.add_argument("--only", default=None, choices=list(ONLY_LINES),
+                    help="time one secondary line alone and print its numbers (a profiling aid; "
+                         "not the contract line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -630,6 +681,10 @@ def main():
 
     _lib.load()
     stream = torch.cuda.current_stream()
+    if args.only:
+        if rank == 0:
+            return run_only(args)
+        return 0
     w = W.named_workload(args.workload)
     runner = ChunkedRunner(w, w.chunk, stream) if w.chunk else PlainRunner(w, stream)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -706,7 +761,7 @@ def main():
         extra[name] = {"ms": round(mx, 4), "gbs": round(rx.bytes / (mx * 1e-3) / 1e9, 1),
                        "frac_of_hbm": round(rx.bytes / (mx * 1e-3) / 1e9 / pk["hbm"], 4),
                        "bytes_per_step": rx.bytes, "tokens_per_s": round(rx.tokens / (mx * 1e-3), 1),
-                       "launches": rx.launches,
+                       "launches": rx.launches, "kernel": "whole-page TMA decode + piece merge",
                        "l2": "256 MiB written then read back before each step (no dirty lines)"}
         del rx
         torch.cuda.empty_cache()
