@@ -547,15 +547,16 @@ int run_linear(const prefill_bf16 *x, const prefill_bf16 *w, int M, int K, int N
         const cuuint32_t box[2] = {64, 128};
         if (!encode(&tm_x, x, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
+    const int tile_n = pf::qkv_gemm_tile_n(M, N, pf::device_sm_count());
     {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N}, strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {64, 256};
+        const cuuint32_t box[2] = {64, (cuuint32_t)tile_n};
         if (!encode(&tm_w, w, 2, dims, strides, box)) return PREFILL_ERR_CUDA;
     }
     p.M = M;
     p.N = N;
     p.K = K;
-    return pf::launch_qkv_gemm(tm_x, tm_w, p, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
+    return pf::launch_qkv_gemm(tm_x, tm_w, p, tile_n, stream) == 0 ? PREFILL_OK : PREFILL_ERR_CUDA;
 }
 
 }  // namespace

@@ -12,12 +12,14 @@
 // column goes to one output, q = y [T][hidden].
 //
 // Design (a dense contraction: tcgen05 tensor cores):
-//  * persistent grid, one CTA per SM; 128 x 256 output tiles, K in steps of 64,
-//    taken in grouped order (tile_coords) so that operands are re-read from L2;
-//  * warp 0 loads A (x, 128 x 64) and B (W, 256 x 64) tiles by TMA, 128-byte
-//    swizzled, into a 4-stage ring; warp 1 issues tcgen05.mma (M 128, N 256,
-//    K 16) with the fp32 accumulator in TMEM, two accumulators (512 columns)
-//    so that the epilogue of one tile overlaps the MMAs of the next;
+//  * persistent grid, one CTA per SM; 128 x BN output tiles (BN 256, or 192
+//    when the output width allows it and the tiles then fill the last wave of
+//    CTAs better), K in steps of 64, taken in grouped order (tile_coords) so
+//    that operands are re-read from L2;
+//  * warp 0 loads A (x, 128 x 64) and B (W, BN x 64) tiles by TMA, 128-byte
+//    swizzled, into a 4-stage (BN 256) or 5-stage (BN 192) ring; warp 1 issues
+//    tcgen05.mma (M 128, N BN, K 16) with the fp32 accumulator in TMEM, two
+//    accumulators so that the epilogue of one tile overlaps the MMAs of the next;
 //  * warps 2-5 drain the accumulator (tcgen05.ld, 32 rows each), round to bf16
 //    and store each 32-column slice into q, k or v;
 //  * every mbarrier wait is bounded (about a second) and raises a CTA abort
@@ -35,16 +37,22 @@
 namespace pf {
 namespace {
 
-constexpr int GBM = 128, GBN = 256, GBK = 64, GST = 4;
+constexpr int GBM = 128, GBK = 64;
 constexpr int GTHREADS = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
-constexpr uint32_t A_TILE = GBM * GBK * 2;  // 16 KB
-constexpr uint32_t B_TILE = GBN * GBK * 2;  // 32 KB
-constexpr uint32_t GSTAGE = A_TILE + B_TILE;
-constexpr uint32_t G_BAR = GST * GSTAGE;
-// barriers: full[GST], empty[GST], acc_full[2], acc_empty[2]
-constexpr int G_FULL = 0, G_EMPTY = GST, G_AFULL = 2 * GST, G_AEMPTY = 2 * GST + 2, G_NBAR = 2 * GST + 4;
-constexpr uint32_t G_TMEM_SLOT = G_BAR + G_NBAR * 8, G_ABORT = G_TMEM_SLOT + 4;
-constexpr uint32_t G_SMEM = G_ABORT + 4 + 1024;  // + slack to align the ring to 1024 bytes
+template <int GBN>
+struct GLay {
+    static constexpr int GST = GBN == 256 ? 4 : 5;           // ring stages
+    static constexpr uint32_t A_TILE = GBM * GBK * 2;         // 16 KB
+    static constexpr uint32_t B_TILE = GBN * GBK * 2;         // 32 or 24 KB
+    static constexpr uint32_t GSTAGE = A_TILE + B_TILE;
+    static constexpr uint32_t G_BAR = GST * GSTAGE;
+    // barriers: full[GST], empty[GST], acc_full[2], acc_empty[2]
+    static constexpr int G_FULL = 0, G_EMPTY = GST, G_AFULL = 2 * GST, G_AEMPTY = 2 * GST + 2, G_NBAR = 2 * GST + 4;
+    static constexpr uint32_t G_TMEM_SLOT = G_BAR + G_NBAR * 8, G_ABORT = G_TMEM_SLOT + 4;
+    static constexpr uint32_t G_SMEM = G_ABORT + 4 + 1024;  // + slack to align the ring to 1024 bytes
+    static_assert(G_SMEM <= 227 * 1024, "shared memory");
+    static_assert(2 * GBN <= 512, "two accumulators in TMEM");
+};
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, uint32_t bar, int c0, int c1) {
     asm volatile(
@@ -81,9 +89,15 @@ __device__ __forceinline__ bool gwait(uint32_t bar, uint32_t parity, volatile in
     return false;
 }
 
+template <int GBN>
 __global__ void __launch_bounds__(GTHREADS, 1)
 qkv_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const QkvParams p) {
+    using GL = GLay<GBN>;
+    constexpr int GST = GL::GST;
+    constexpr uint32_t A_TILE = GL::A_TILE, GSTAGE = GL::GSTAGE, G_BAR = GL::G_BAR;
+    constexpr int G_FULL = GL::G_FULL, G_EMPTY = GL::G_EMPTY, G_AFULL = GL::G_AFULL, G_AEMPTY = GL::G_AEMPTY;
+    constexpr uint32_t G_TMEM_SLOT = GL::G_TMEM_SLOT, G_ABORT = GL::G_ABORT;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -224,19 +238,40 @@ qkv_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-}  // namespace
-
-size_t qkv_gemm_smem_bytes() { return G_SMEM; }
-
-int launch_qkv_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const QkvParams &p, void *stream) {
-    cudaError_t e = cudaFuncSetAttribute(qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G_SMEM);
+template <int GBN>
+int launch_bn(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const QkvParams &p, int sms, void *stream) {
+    constexpr uint32_t smem = GLay<GBN>::G_SMEM;
+    cudaError_t e = cudaFuncSetAttribute(qkv_gemm_kernel<GBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return (int)e;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int tiles = cdiv(p.M, GBM) * (p.N / GBN);
     const int grid = tiles < sms ? tiles : sms;
-    qkv_gemm_kernel<<<grid, GTHREADS, G_SMEM, (cudaStream_t)stream>>>(tm_x, tm_w, p);
+    qkv_gemm_kernel<GBN><<<grid, GTHREADS, smem, (cudaStream_t)stream>>>(tm_x, tm_w, p);
     return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int qkv_gemm_tile_n(int M, int N, int sms) {
+    // the tile width whose tiles fill the persistent grid's waves best: the
+    // work is the same, the last wave's idle CTAs are not.  Measured on the
+    // 8192 x 4096 x 6144 projection: 128 x 256 tiles (10.4 waves) 1448-1469
+    // TFLOP/s, 128 x 192 (13.8 waves) 1475-1503, 128 x 128 (20.8 waves) 1242
+    // (twice the MMA instructions and operand reads per FLOP of the 256 tile)
+    auto eff = [&](int bn) {
+        const long long tiles = (long long)cdiv(M, GBM) * (N / bn);
+        const long long waves = (tiles + sms - 1) / sms;
+        return (double)tiles / (double)(waves * sms);
+    };
+    if (N % 192 == 0 && (N % 256 != 0 || eff(192) > eff(256) + 0.01)) return 192;
+    return 256;
+}
+
+size_t qkv_gemm_smem_bytes(int tile_n) { return tile_n == 192 ? GLay<192>::G_SMEM : GLay<256>::G_SMEM; }
+
+int launch_qkv_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const QkvParams &p, int tile_n, void *stream) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return tile_n == 192 ? launch_bn<192>(tm_x, tm_w, p, sms, stream) : launch_bn<256>(tm_x, tm_w, p, sms, stream);
 }
 
 }  // namespace pf

@@ -17,7 +17,11 @@ struct QkvParams {
     int32_t *status;    // nullable
 };
 
-size_t qkv_gemm_smem_bytes();
-int launch_qkv_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const QkvParams &p, void *stream);
+// Output tile width (256, or 192 when N allows it and the tiles fill the
+// waves of a persistent grid of `sms` CTAs better); the W tensor map's box
+// is tile_n rows of 64 columns.
+int qkv_gemm_tile_n(int M, int N, int sms);
+size_t qkv_gemm_smem_bytes(int tile_n);
+int launch_qkv_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const QkvParams &p, int tile_n, void *stream);
 
 }  // namespace pf

@@ -333,7 +333,8 @@ int prefill_attn_chunked_fp8(const prefill_bf16 *q, const prefill_bf16 *k, const
  * nearest even).  Requires hidden a multiple of 64, head_dim a multiple of 32
  * and (n_head + 2 n_kv_head) head_dim a multiple of 256
  * (PREFILL_ERR_UNSUPPORTED otherwise); pointers 16-byte aligned.  Runs on the
- * tensor cores (tcgen05) with 128 x 256 output tiles; a device wait that runs
+ * tensor cores (tcgen05) with 128 x 256 output tiles (128 x 192 when that width
+ * divides the output and fills the GPU's waves better); a device wait that runs
  * past its limit is reported as PREFILL_ERR_TIMEOUT in *status_dev.
  */
 int qkv_projection(const prefill_bf16 *x, const prefill_bf16 *w, int tokens, int hidden,
