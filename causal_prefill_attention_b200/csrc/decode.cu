@@ -116,11 +116,14 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
-// two e4m3 codes (low byte first) -> two f16 (exact: f16 holds every e4m3 value)
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    uint32_t d;
-    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(d) : "r"(two_codes));
-    return d;
+// four e4m3 codes (bytes 0-3 of w) -> two f16 pairs, exact (f16 holds every
+// e4m3 value): lo = (byte 0, byte 1), hi = (byte 2, byte 3), the lower byte in
+// the lower half; the word's 16-bit halves go to the conversions directly
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // byte offset of 16-byte slot `s` (0 .. D/8-1) of row `r` (0 .. 15) in a step tile:
@@ -434,10 +437,13 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
             for (int j = 0; j < D / 32; ++j) {
                 uint32_t w[4];
                 ldsm_x4(st + f8_off<D>(kr, 2 * j + (m >> 1)), w);
-                mma16816<true>(s0, qa[2 * j], e4m3x2_to_f16x2(w[0] & 0xffffu), e4m3x2_to_f16x2(w[0] >> 16));
-                mma16816<true>(s1, qa[2 * j], e4m3x2_to_f16x2(w[1] & 0xffffu), e4m3x2_to_f16x2(w[1] >> 16));
-                mma16816<true>(t0, qa[2 * j + 1], e4m3x2_to_f16x2(w[2] & 0xffffu), e4m3x2_to_f16x2(w[2] >> 16));
-                mma16816<true>(t1, qa[2 * j + 1], e4m3x2_to_f16x2(w[3] & 0xffffu), e4m3x2_to_f16x2(w[3] >> 16));
+                uint32_t f[4][2];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) e4m3x4_to_f16x2x2(w[e], f[e][0], f[e][1]);
+                mma16816<true>(s0, qa[2 * j], f[0][0], f[0][1]);
+                mma16816<true>(s1, qa[2 * j], f[1][0], f[1][1]);
+                mma16816<true>(t0, qa[2 * j + 1], f[2][0], f[2][1]);
+                mma16816<true>(t1, qa[2 * j + 1], f[3][0], f[3][1]);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -531,10 +537,12 @@ __global__ void __launch_bounds__(DTHREADS, kCtasPerSm) paged_decode_kernel(cons
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t lo = w[2 * h], hi = w[2 * h + 1];  // keys 0-7, keys 8-15
-                    mma16816<true>(o[4 * c + 2 * h], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0020)),
-                                   e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0020)));
-                    mma16816<true>(o[4 * c + 2 * h + 1], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0031)),
-                                   e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0031)));
+                    // even columns: (lo byte 0, lo byte 2 | hi byte 0, hi byte 2); odd: bytes 1, 3
+                    uint32_t ev[2], od[2];
+                    e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x6420), ev[0], ev[1]);
+                    e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x7531), od[0], od[1]);
+                    mma16816<true>(o[4 * c + 2 * h], pa, ev[0], ev[1]);
+                    mma16816<true>(o[4 * c + 2 * h + 1], pa, od[0], od[1]);
                 }
             }
         } else {
@@ -1001,10 +1009,13 @@ paged_decode_tma_kernel(const __grid_constant__ CUtensorMap tm, const DecodePara
                     for (int j = 0; j < D / 32; ++j) {
                         uint32_t w[4];
                         ldsm_x4(kt + f8_off<D>(kr, 2 * j + (m >> 1)), w);
-                        mma16816<true>(s0, qa[2 * j], e4m3x2_to_f16x2(w[0] & 0xffffu), e4m3x2_to_f16x2(w[0] >> 16));
-                        mma16816<true>(s1, qa[2 * j], e4m3x2_to_f16x2(w[1] & 0xffffu), e4m3x2_to_f16x2(w[1] >> 16));
-                        mma16816<true>(t0, qa[2 * j + 1], e4m3x2_to_f16x2(w[2] & 0xffffu), e4m3x2_to_f16x2(w[2] >> 16));
-                        mma16816<true>(t1, qa[2 * j + 1], e4m3x2_to_f16x2(w[3] & 0xffffu), e4m3x2_to_f16x2(w[3] >> 16));
+                        uint32_t f[4][2];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) e4m3x4_to_f16x2x2(w[e], f[e][0], f[e][1]);
+                        mma16816<true>(s0, qa[2 * j], f[0][0], f[0][1]);
+                        mma16816<true>(s1, qa[2 * j], f[1][0], f[1][1]);
+                        mma16816<true>(t0, qa[2 * j + 1], f[2][0], f[2][1]);
+                        mma16816<true>(t1, qa[2 * j + 1], f[3][0], f[3][1]);
                     }
                 } else {
                     const int kr = (m >> 1) * 8 + (lane & 7);  // matrices: keys 0-7 / 8-15 x columns +0 / +8
@@ -1083,10 +1094,12 @@ paged_decode_tma_kernel(const __grid_constant__ CUtensorMap tm, const DecodePara
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const uint32_t lo = w[2 * h], hi = w[2 * h + 1];
-                            mma16816<true>(o[4 * c + 2 * h], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0020)),
-                                           e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0020)));
-                            mma16816<true>(o[4 * c + 2 * h + 1], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0031)),
-                                           e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0031)));
+                            // even columns: (lo byte 0, lo byte 2 | hi byte 0, hi byte 2); odd: bytes 1, 3
+                            uint32_t ev[2], od[2];
+                            e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x6420), ev[0], ev[1]);
+                            e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x7531), od[0], od[1]);
+                            mma16816<true>(o[4 * c + 2 * h], pa, ev[0], ev[1]);
+                            mma16816<true>(o[4 * c + 2 * h + 1], pa, od[0], od[1]);
                         }
                     }
                 } else {
