@@ -1078,18 +1078,17 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(cons
     const int lane = threadIdx.x & 31;
     if (task >= (long long)p.total * p.n_head) return;
     const int t = (int)(task / p.n_head), h = (int)(task - (long long)t * p.n_head);
+    // the row's tag, maxima, sums and O partials are loaded together, for every
+    // split the launch may have used (all inside the workspace); only the row's
+    // own splits are used once the tag is known
     const uint32_t tag = p.part_nsp[t];
-    if ((tag >> 4) != (p.epoch & 0x0fffffffu)) return;  // not a row this launch split
-    int nsp = (int)(tag & 15u);
-    if (nsp <= 1) return;
-    if (nsp > p.nsplit) nsp = p.nsplit;
     const size_t row = (size_t)t * p.n_head + h, stride = (size_t)p.total * p.n_head;
     float2 ml = make_float2(-CUDART_INF_F, 0.f);
-    if (lane < nsp) ml = *reinterpret_cast<const float2 *>(p.part_ml + (row + lane * stride) * 2);
+    if (lane < p.nsplit) ml = *reinterpret_cast<const float2 *>(p.part_ml + (row + lane * stride) * 2);
     float v[kMaxSplits][E];
 #pragma unroll
     for (int sp = 0; sp < kMaxSplits; ++sp) {
-        if (sp < nsp) {
+        if (sp < p.nsplit) {
             const float *po = p.part_o + (row + sp * stride) * D + lane * E;
             if constexpr (E == 4) {
                 const float4 f = *reinterpret_cast<const float4 *>(po);
@@ -1100,6 +1099,11 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(cons
             }
         }
     }
+    if ((tag >> 4) != (p.epoch & 0x0fffffffu)) return;  // not a row this launch split
+    int nsp = (int)(tag & 15u);
+    if (nsp <= 1) return;
+    if (nsp > p.nsplit) nsp = p.nsplit;
+    if (lane >= nsp) ml = make_float2(-CUDART_INF_F, 0.f);
     float M = ml.x;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
