@@ -28,8 +28,10 @@ struct FwdParams {
     int max_ctx;                  // bound on every context length (chunked prefill; 0 otherwise)
     int window;                   // sliding window: row P sees keys P-window+1 .. P (<= 0: none)
     // split-KV: kv ranges split into up to nsplit parts; the partial results go to
-    // part_o [nsplit][total][n_head][D] (fp32, unnormalised) and part_ml
-    // [nsplit][total][n_head][2] (running max in log2 units, exp-sum), and
+    // part_o [nsplit][n_head][D / 4][total] float4 (fp32, unnormalised; the rows of
+    // one 4-column chunk contiguous, so that a warp's 32 rows store 512
+    // contiguous bytes) and part_ml [nsplit][n_head][total][2] (running max in
+    // log2 units, exp-sum), and
     // part_nsp [total] holds, for every row of a valid sequence, its pair's split
     // count tagged with this launch's epoch ((epoch << 4) | splits), so that the
     // merge kernel skips rows that this launch did not split (or did not reach)

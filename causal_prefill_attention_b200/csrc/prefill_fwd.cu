@@ -602,9 +602,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 p.part_nsp[it.c0 + a] = (p.epoch << 4) | (uint32_t)it.nsp;
             if (it.nsp > 1) {
                 // split-KV: unnormalised O, the running max (log2 units) and the
-                // exp-sum go to the workspace; the combine kernel merges the splits
-                const size_t prow = ((size_t)it.split * p.total + (it.c0 + a)) * p.n_head + it.h;
-                float *po = p.part_o + prow * D;
+                // exp-sum go to the workspace; the combine kernel merges the splits.
+                // O chunk-major ([split][head][column / 4][row]): a warp's 32 rows
+                // of one 4-column chunk are 512 contiguous bytes
+                const size_t sh = (size_t)it.split * p.n_head + it.h;
+                float4 *po = reinterpret_cast<float4 *>(p.part_o) + sh * (D / 4) * p.total + (it.c0 + a);
                 uint32_t r[32];
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
@@ -614,13 +616,15 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * vf);
                     }
                     if (a < it.n) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(po + cc * 32);
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
-                            d4[c] = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+                            po[(size_t)(cc * 8 + c) * p.total] = make_float4(
+                                __uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]), __uint_as_float(r[4 * c + 2]),
+                                __uint_as_float(r[4 * c + 3]));
                     }
                 }
-                if (a < it.n) *reinterpret_cast<float2 *>(p.part_ml + prow * 2) = make_float2(m_run * sl2, l_run);
+                if (a < it.n)
+                    *reinterpret_cast<float2 *>(p.part_ml + (sh * p.total + it.c0 + a) * 2) = make_float2(m_run * sl2, l_run);
             } else {
             const float inv_l = vf / l_run;
             uint16_t *dst = p.out + ((size_t)(it.c0 + a) * p.n_head + it.h) * D;
@@ -1061,74 +1065,97 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp == WARP_MMA) tmem_dealloc(tmem, 512);
 }
 
-// Split-KV merge: one warp per (packed row t, query head h), four per CTA.  The
-// row's split count comes from part_nsp, written by this launch's attention
-// kernel for every row of a valid sequence with the launch's epoch (a stale or
-// unsplit row is left alone).  All partial loads are issued before any use;
-// then O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s --
-// the merge rule the online softmax applies between blocks.
+// Split-KV merge: a warp merges 32 consecutive packed rows x 32 columns of one
+// query head, a lane per row (four warps per CTA, four heads; blockIdx.z picks
+// the 32 columns).  A row's split count comes from part_nsp, written by this
+// launch's attention kernel for every row of a valid sequence with the
+// launch's epoch (a stale or unsplit row is left alone).  The loads of the
+// splits' (max, sum) and of each 4-column chunk are 512 contiguous bytes per
+// warp (the partials' chunk-major layout), all issued before any use; the
+// lanes' rows then go through shared memory so that the output is written in
+// 64-byte row pieces: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with
+// M = max_s m_s -- the merge rule the online softmax applies between blocks.
 constexpr int kCombineWarps = 4;
 constexpr int kMaxSplits = 8;
 template <int D>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_splits_kernel(const FwdParams p) {
-    constexpr int E = D / 32;  // elements per lane
+    __shared__ __align__(16) uint16_t tile[kCombineWarps][32][40];  // 32 columns (+ 8: distinct banks)
     griddep_wait();  // the attention kernel's partials are complete
     griddep_launch_dependents();
-    const long long task = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (task >= (long long)p.total * p.n_head) return;
-    const int t = (int)(task / p.n_head), h = (int)(task - (long long)t * p.n_head);
-    // the row's tag, maxima, sums and O partials are loaded together, for every
-    // split the launch may have used (all inside the workspace); only the row's
-    // own splits are used once the tag is known
-    const uint32_t tag = p.part_nsp[t];
-    const size_t row = (size_t)t * p.n_head + h, stride = (size_t)p.total * p.n_head;
-    float2 ml = make_float2(-CUDART_INF_F, 0.f);
-    if (lane < p.nsplit) ml = *reinterpret_cast<const float2 *>(p.part_ml + (row + lane * stride) * 2);
-    float v[kMaxSplits][E];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y * kCombineWarps + warp;
+    const int t0 = blockIdx.x * 32, t = t0 + lane, c0 = blockIdx.z * 8;  // 4-column chunks c0 .. c0 + 7
+    if (h >= p.n_head) return;
+    // every load that the launch's split count allows is issued before the
+    // row's tag is known (speculative loads stay inside the workspace); the
+    // splits' O chunks two at a time
+    const bool in = t < p.total;
+    const uint32_t tag = in ? p.part_nsp[t] : 0u;
+    const float4 *po = reinterpret_cast<const float4 *>(p.part_o);
+    auto oaddr = [&](int sp, int c) -> size_t {
+        return (((size_t)sp * p.n_head + h) * (D / 4) + c0 + c) * p.total + t;
+    };
+    float2 ml[kMaxSplits];
 #pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) {
-        if (sp < p.nsplit) {
-            const float *po = p.part_o + (row + sp * stride) * D + lane * E;
-            if constexpr (E == 4) {
-                const float4 f = *reinterpret_cast<const float4 *>(po);
-                v[sp][0] = f.x; v[sp][1] = f.y; v[sp][2] = f.z; v[sp][3] = f.w;
-            } else {
-                const float2 f = *reinterpret_cast<const float2 *>(po);
-                v[sp][0] = f.x; v[sp][1] = f.y;
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+        if (in && sp < p.nsplit)
+            ml[sp] = *reinterpret_cast<const float2 *>(p.part_ml + (((size_t)sp * p.n_head + h) * p.total + t) * 2);
+    float4 f[2][8];
+#pragma unroll
+    for (int sp = 0; sp < 2; ++sp)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (in && sp < p.nsplit) f[sp][c] = po[oaddr(sp, c)];
+    int nsp = (in && (tag >> 4) == (p.epoch & 0x0fffffffu)) ? (int)(tag & 15u) : 0;  // else: not a row this launch split
+    if (nsp > p.nsplit) nsp = p.nsplit;
+    const bool mine = nsp > 1;
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+        if (mine && sp < nsp) M = fmaxf(M, ml[sp].x);
+    float L = 0.f;
+    float4 acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s0 = 0; s0 < kMaxSplits; s0 += 2) {
+        if (s0 >= nsp) break;
+        if (s0 > 0) {  // the next two splits (three or more splits: rare)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    if (s0 + j < nsp) f[j][c] = po[oaddr(s0 + j, c)];
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (mine && s0 + j < nsp) {
+                const float w = ex2(ml[s0 + j].x - M);
+                L += w * ml[s0 + j].y;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    acc[c].x = fmaf(w, f[j][c].x, acc[c].x);
+                    acc[c].y = fmaf(w, f[j][c].y, acc[c].y);
+                    acc[c].z = fmaf(w, f[j][c].z, acc[c].z);
+                    acc[c].w = fmaf(w, f[j][c].w, acc[c].w);
+                }
             }
         }
     }
-    if ((tag >> 4) != (p.epoch & 0x0fffffffu)) return;  // not a row this launch split
-    int nsp = (int)(tag & 15u);
-    if (nsp <= 1) return;
-    if (nsp > p.nsplit) nsp = p.nsplit;
-    if (lane >= nsp) ml = make_float2(-CUDART_INF_F, 0.f);
-    float M = ml.x;
+    const float inv = mine ? 1.f / L : 0.f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float wgt = lane < nsp ? ex2(ml.x - M) : 0.f;
-    float L = wgt * ml.y;
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint2 *>(&tile[warp][lane][4 * c]) =
+            make_uint2(pack_bf16x2(acc[c].x * inv, acc[c].y * inv), pack_bf16x2(acc[c].z * inv, acc[c].w * inv));
+    __syncwarp();
+    // 64-byte row pieces: 4 lanes per row, 8 rows per store
+    const uint32_t mask = __ballot_sync(0xffffffffu, mine);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) {
-        const float w_sp = __shfl_sync(0xffffffffu, wgt, sp);
-        if (sp < nsp) {
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] = fmaf(w_sp, v[sp][e], acc[e]);
-        }
-    }
-    const float inv = 1.f / L;
-    uint16_t *dst = p.out + row * D + lane * E;
-    if constexpr (E == 4) {
-        *reinterpret_cast<uint2 *>(dst) =
-            make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-    } else {
-        *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    for (int rb = 0; rb < 32; rb += 8) {
+        const int rr = rb + lane / 4, q = lane % 4;
+        if ((mask >> rr) & 1u)
+            *reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + rr) * p.n_head + h) * D + c0 * 4 + q * 8) =
+                *reinterpret_cast<const uint4 *>(&tile[warp][rr][q * 8]);
     }
 }
 
@@ -1185,8 +1212,7 @@ int launch_nst(const TensorMaps &maps, const FwdParams &p, void *stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, prefill_fwd_kernel<D, NST, MODE>, maps.q, maps.k, maps.v, maps.cache, p, P);
     if (e != cudaSuccess || p.nsplit <= 1) return (int)e;
-    const long long tasks = (long long)p.total * p.n_head;
-    cfg.gridDim = dim3((unsigned)((tasks + kCombineWarps - 1) / kCombineWarps));
+    cfg.gridDim = dim3((unsigned)cdiv(p.total, 32), (unsigned)cdiv(p.n_head, kCombineWarps), (unsigned)(D / 32));
     cfg.blockDim = dim3(32 * kCombineWarps);
     cfg.dynamicSmemBytes = 0;
     return (int)cudaLaunchKernelEx(&cfg, combine_splits_kernel<D>, p);
