@@ -43,6 +43,7 @@
 #include <math_constants.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "../../include/prefill.h"
 #include "block_rule.h"
@@ -1199,37 +1200,45 @@ __global__ void __launch_bounds__(128) decode_merge_pieces_kernel(const DecodePa
     if (np <= 1) return;
     const size_t base_row = (size_t)(c0 + i * nslab + slab) * ((size_t)TW * r) + (size_t)w * r + h;
     const size_t pstride = (size_t)TW * r;  // rows between consecutive pieces of the segment
-    constexpr int E = D / 32;
-    float M = -CUDART_INF_F;
-    for (int c = lane; c < np; c += 32) M = fmaxf(M, __ldcg(p.part_ml + (base_row + c * pstride) * 2));
+    constexpr int E = D / 32, PB = 4;       // the first PB pieces' O rows load with the maxima
+    using V = typename std::conditional<E == 4, float4, float2>::type;
+    V f[PB];
+#pragma unroll
+    for (int j = 0; j < PB; ++j)
+        if (j < np) f[j] = __ldcg(reinterpret_cast<const V *>(p.part_o + (base_row + j * pstride) * D + lane * E));
+    float2 mlane = make_float2(-CUDART_INF_F, 0.f);  // piece `lane` (first 32 pieces)
+    if (lane < np) mlane = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + (base_row + lane * pstride) * 2));
+    float M = mlane.x;
+    for (int c = lane + 32; c < np; c += 32) M = fmaxf(M, __ldcg(p.part_ml + (base_row + c * pstride) * 2));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float L = 0.f;
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    auto add = [&](float wgt, const V &v) {
+        const float *fv = reinterpret_cast<const float *>(&v);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, fv[e], acc[e]);
+    };
     for (int cb = 0; cb < np; cb += 32) {
         float wl = 0.f;
         if (cb + lane < np) {
-            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + (base_row + (cb + lane) * pstride) * 2));
+            const float2 ml = cb == 0 ? mlane
+                                      : __ldcg(reinterpret_cast<const float2 *>(p.part_ml + (base_row + (cb + lane) * pstride) * 2));
             wl = ex2(ml.x - M);
             L += wl * ml.y;
         }
         const int nb = min(32, np - cb);
-#pragma unroll 4
         for (int j = 0; j < nb; ++j) {
             const float wgt = __shfl_sync(0xffffffffu, wl, j);
-            const float *src = p.part_o + (base_row + (cb + j) * pstride) * D + lane * E;
-            if constexpr (E == 4) {
-                const float4 f = __ldcg(reinterpret_cast<const float4 *>(src));
-                acc[0] += wgt * f.x;
-                acc[1] += wgt * f.y;
-                acc[2] += wgt * f.z;
-                acc[3] += wgt * f.w;
+            const int c = cb + j;
+            if (c < PB) {
+#pragma unroll
+                for (int k = 0; k < PB; ++k)
+                    if (k == c) add(wgt, f[k]);
             } else {
-                const float2 f = __ldcg(reinterpret_cast<const float2 *>(src));
-                acc[0] += wgt * f.x;
-                acc[1] += wgt * f.y;
+                add(wgt, __ldcg(reinterpret_cast<const V *>(p.part_o + (base_row + c * pstride) * D + lane * E)));
             }
         }
     }
