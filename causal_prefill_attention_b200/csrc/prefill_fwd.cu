@@ -961,14 +961,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             for (int b = 0; b < BATCH; ++b) {
                                 const int r = (rb + b) * 2 * RPW + cw * RPW + lane / LPR;
                                 uint32_t h[8];
-                                h[0] = e4m3x2_to_f16x2_exact(c[b].x & 0xffffu);
-                                h[1] = e4m3x2_to_f16x2_exact(c[b].x >> 16);
-                                h[2] = e4m3x2_to_f16x2_exact(c[b].y & 0xffffu);
-                                h[3] = e4m3x2_to_f16x2_exact(c[b].y >> 16);
-                                h[4] = e4m3x2_to_f16x2_exact(c[b].z & 0xffffu);
-                                h[5] = e4m3x2_to_f16x2_exact(c[b].z >> 16);
-                                h[6] = e4m3x2_to_f16x2_exact(c[b].w & 0xffffu);
-                                h[7] = e4m3x2_to_f16x2_exact(c[b].w >> 16);
+                                e4m3x4_to_f16x2x2_exact(c[b].x, h[0], h[1]);
+                                e4m3x4_to_f16x2x2_exact(c[b].y, h[2], h[3]);
+                                e4m3x4_to_f16x2x2_exact(c[b].z, h[4], h[5]);
+                                e4m3x4_to_f16x2x2_exact(c[b].w, h[6], h[7]);
                                 uint8_t *row = tile + ch * CHUNK + r * 128;
                                 *reinterpret_cast<uint4 *>(row + ((u0 ^ (r & 7)) << 4)) =
                                     make_uint4(h[0], h[1], h[2], h[3]);

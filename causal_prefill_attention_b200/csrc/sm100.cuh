@@ -322,11 +322,14 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
-// Two e4m3 codes (low byte first) to their values as packed f16x2 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_exact(uint32_t two_codes) {
-    uint32_t d;
-    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(d) : "r"(two_codes));
-    return d;
+// Four e4m3 codes (bytes 0-3 of w) to their values as two packed f16x2
+// (exact): lo from bytes 0-1, hi from bytes 2-3, the lower byte in the lower
+// half; the word's 16-bit halves go to the conversions directly.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2_exact(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
