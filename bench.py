@@ -146,7 +146,7 @@ def prefill_splits(num_seqs: int, n_head: int, max_q: int, max_ctx: int, sms: in
     """Key splits the library chooses for a prefill call (the rule of its
     split selection, restated: split only when the call has fewer work items
     than SMs; then the count up to 8 that minimises waves x blocks per split
-    plus a fixed cost of 6 blocks, with at least 4 blocks per split).  A split
+    plus a fixed cost of 4 blocks, with at least 4 blocks per split).  A split
     call launches the attention kernel and then the merge kernel."""
     items = num_seqs * n_head * -(-max_q // 256)
     if items <= 0 or items >= sms:
@@ -156,7 +156,7 @@ def prefill_splits(num_seqs: int, n_head: int, max_q: int, max_ctx: int, sms: in
     for sp in range(2, 9):
         if nk // sp < 4:
             break
-        cost = -(-(items * sp) // sms) * -(-nk // sp) + 6.0
+        cost = -(-(items * sp) // sms) * -(-nk // sp) + 4.0
         if cost < best_cost - 1e-9:
             best, best_cost = sp, cost
     return best

@@ -1248,10 +1248,12 @@ bool fwd_pipelined_supported(const FwdParams &p, int head_dim) {
     return smem <= kMaxSmem;
 }
 
-// Fixed cost of splitting (the partial writes and the combine kernel), in
-// units of one kv block step of a work item: measured ~12 us against ~2 us
-// per step on the 512-row chunks of an 8k GQA prompt.
-constexpr double kSplitCostSteps = 6.0;
+// Fixed cost of splitting (the partial writes and the merge kernel), in units
+// of one kv block step of a work item: the merge path of a 512-row chunk of an
+// 8k GQA prompt takes ~6 us (release of the merge launch, merging, release of
+// the next launch) against ~2 us per step; on the 16 chunks of that prompt a
+// cost of 4 steps ran fastest (6: 0.859 ms, 4: 0.851, 3: 0.858, 2: 0.863).
+constexpr double kSplitCostSteps = 4.0;
 
 int device_sm_count() { return sm_count(); }
 
