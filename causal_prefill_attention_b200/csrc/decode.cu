@@ -1037,6 +1037,26 @@ paged_decode_tma_kernel(const __grid_constant__ CUtensorMap tm, const DecodePara
                     s1[e] += t1[e];
                 }
             }
+            // FP8: the step's V codes widened to f16 fragments here -- they do not depend
+            // on the scores, so their loads and conversions overlap the S products and
+            // the softmax instead of following them
+            uint32_t vf[kFp8 ? D / 32 : 1][2][4];
+            if constexpr (kFp8) {
+                const int m = lane >> 3;
+                const int vr = (m & 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t w[4];
+                    ldsm_x4_t(vt + f8_off<D>(vr, 2 * c + (m >> 1)), w);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t lo = w[2 * h], hi = w[2 * h + 1];
+                        // even columns: (lo byte 0, lo byte 2 | hi byte 0, hi byte 2); odd: bytes 1, 3
+                        e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x6420), vf[c][h][0], vf[c][h][1]);
+                        e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x7531), vf[c][h][2], vf[c][h][3]);
+                    }
+                }
+            }
             const int nvalid = uc.k1 - p0;
             if (c2 >= nvalid) s0[0] = s0[2] = -CUDART_INF_F;
             if (c2 + 1 >= nvalid) s0[1] = s0[3] = -CUDART_INF_F;
@@ -1089,20 +1109,12 @@ paged_decode_tma_kernel(const __grid_constant__ CUtensorMap tm, const DecodePara
                 const int vr = (m & 1) * 8 + (lane & 7);
                 if constexpr (kFp8) {
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t w[4];
-                        ldsm_x4_t(vt + f8_off<D>(vr, 2 * c + (m >> 1)), w);
+                    for (int c = 0; c < D / 32; ++c)
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            const uint32_t lo = w[2 * h], hi = w[2 * h + 1];
-                            // even columns: (lo byte 0, lo byte 2 | hi byte 0, hi byte 2); odd: bytes 1, 3
-                            uint32_t ev[2], od[2];
-                            e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x6420), ev[0], ev[1]);
-                            e4m3x4_to_f16x2x2(__byte_perm(lo, hi, 0x7531), od[0], od[1]);
-                            mma16816<true>(o[4 * c + 2 * h], pa, ev[0], ev[1]);
-                            mma16816<true>(o[4 * c + 2 * h + 1], pa, od[0], od[1]);
+                            mma16816<true>(o[4 * c + 2 * h], pa, vf[c][h][0], vf[c][h][1]);
+                            mma16816<true>(o[4 * c + 2 * h + 1], pa, vf[c][h][2], vf[c][h][3]);
                         }
-                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < NT / 2; ++c) {
